@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer forward on B200: tokens/s and TFLOPS.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed
+
+One step = one moe_forward (router GEMM + TopK/softmax, permutation, grouped
+SwiGLU FFN, combine) over one batch of synthetic tokens already resident in
+HBM.  With N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica of the layer on its own batch (the forward has no data
+exchange when dropless), the timed region is bracketed by a barrier and a
+device synchronise, and the time is the max over ranks.  Rank 0 prints one
+JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "mixtral_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (profiling runs on a smaller batch)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=None,
+                    help="tokens per oracle sample (default: sized to ~10-20 s)")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------- accounting
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic(w, n_kept, tokens_with_kept):
+    """FLOPs and HBM bytes of each stage for one forward (padding and dropped
+    assignments are never counted)."""
+    s = 2 if w.dtype == "bf16" else 4
+    T, d, E, k, H = w.T, w.d, w.E, w.k, w.H
+    c_up = 4 if w.act == "swiglu" else 2
+    flop = {
+        "route": 2.0 * T * d * E,
+        "ffn_up": c_up * float(d) * H * n_kept,
+        "ffn_down": 2.0 * d * H * n_kept,
+    }
+    n_w_up = (2 if w.act == "swiglu" else 1) * E * d * H
+    byts = {
+        # read x and W_g once; write idx, gate (T*k each) and margin
+        "route": T * d * s + d * E * s + T * k * 8 + T * 4,
+        # read idx twice, the rows of x that are kept somewhere, write kept rows and pos
+        "permute": 2 * T * k * 4 + tokens_with_kept * d * s + n_kept * d * s + T * k * 4,
+        # weights once, activations in and out
+        "ffn_up": n_w_up * s + n_kept * d * s + n_kept * H * s,
+        "ffn_down": E * H * d * s + n_kept * H * s + n_kept * d * 4,
+        # read kept rows of o (fp32), pos and gate; write y
+        "combine": n_kept * d * 4 + T * k * 8 + T * d * s,
+    }
+    total_flop = flop["route"] + flop["ffn_up"] + flop["ffn_down"]
+    return flop, byts, total_flop
+
+
+def traffic_for(kernel_file, kernel):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, "mixture_experts_layer_51_b200", "csrc", kernel_file)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if rec.get("source_sha") != sha:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sms.append(float(r[1]))
+                maxs.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "samples": len(sms), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------- CPU oracle
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_seconds(w, cpu_inp, T_s):
+    """Run the fp64 oracle as it stands on the first T_s tokens (routing,
+    capacity over that sample batch, expert FFNs, combine); wall seconds."""
+    import oracle
+    x = cpu_inp["x"][:T_s]
+    t0 = time.perf_counter()
+    logits = oracle.router_logits(x, cpu_inp["Wg"], cpu_inp["bias"])
+    idx, _, _ = oracle.top_k(logits, w.k)
+    C = oracle.capacity(T_s, w.E, w.k, w.cf)
+    _, _, _, kept = oracle.assign_capacity(idx, w.E, C)
+    oracle.moe_forward_tokens(x, logits, idx, kept, cpu_inp["W1"], cpu_inp["W3"],
+                              cpu_inp["W2"], w.act)
+    return time.perf_counter() - t0
+
+
+def default_cpu_sample(w):
+    # ~10-20 s of fp64 work on a few host cores for the large layers.
+    per_token = 2.0 * w.k * (3 if w.act == "swiglu" else 2) * w.d * w.H
+    return int(max(16, min(w.T, 2.5e11 / per_token / 8)))
+
+
+# ----------------------------------------------------------------- main
+def main(argv=None):
+    a = parse_args(argv)
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_51_b200 import moe as M
+    from mixture_experts_layer_51_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[a.workload]
+    if a.tokens:
+        w = w.replace(T=a.tokens)
+    peaks, peak_src = load_peaks()
+
+    if a.impl == "reference":
+        return run_reference(a, w, rank, world)
+
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    inp = make_inputs(w, dev)
+    layer = M.MoELayer(inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], w.k, w.cf, w.act,
+                       max_tokens=w.T)
+    x = inp["x"]
+    y = torch.empty_like(x)
+
+    # Routing statistics for the FLOP count (kept assignments only).
+    _, st = layer(x, y=y, stats=True)
+    n_kept = int(st.kept)
+    pos = layer.intermediates(w.T)["pos"]
+    tokens_with_kept = int((pos >= 0).any(dim=1).sum().item())
+    flop, byts, total_flop = algorithmic(w, n_kept, tokens_with_kept)
+
+    for _ in range(a.warmup):
+        layer(x, y=y)
+    torch.cuda.synchronize(dev)
+
+    # Stage events for every timed step (recorded on the launching stream).
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(M.MOE_NUM_STAGE_EVENTS)]
+           for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local) if not a.no_clocks else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    start.record(stream)
+    for i in range(a.steps):
+        M.moe_set_stage_events(evs[i])
+        layer(x, y=y)
+    end.record(stream)
+    M.moe_set_stage_events(None)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop() if clocks else None
+    elapsed_ms = start.elapsed_time(end)
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    stage_ms = {s: 0.0 for s in M.STAGES}
+    for i in range(a.steps):
+        for s, v in M.stage_times_ms(evs[i]).items():
+            stage_ms[s] += v / a.steps
+
+    ms_per_step = elapsed_ms / a.steps
+    tokens_per_s = world * w.T * a.steps / (elapsed_ms / 1e3)
+    tflops = total_flop * world * a.steps / (elapsed_ms / 1e3) / 1e12
+
+    # End to end: tokens in pinned host memory, copies inside the timed call.
+    e2e = None
+    if not a.no_e2e:
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty_like(x_host).pin_memory()
+        x_dev, y_dev = torch.empty_like(x), torch.empty_like(x)
+        ws = layer.workspace(w.T)
+        for _ in range(2):
+            M.moe_forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
+                               w.k, w.cf, w.act, y_host=y_host, x_dev=x_dev, y_dev=y_dev, ws=ws)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.steps):
+            M.moe_forward_host(x_host, inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"],
+                               w.k, w.cf, w.act, y_host=y_host, x_dev=x_dev, y_dev=y_dev, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        nbytes = x.numel() * x.element_size()
+        e2e = {"value": world * w.T * a.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "ms_per_step": e2e_ms / a.steps}
+
+    # CPU baseline: the oracle as it stands, bounded sample, rank 0 at N=1.
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu_inp = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+        T_s = a.cpu_sample or default_cpu_sample(w)
+        secs = oracle_sample_seconds(w, cpu_inp, T_s)
+        cpu = {"value": T_s / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"first {T_s} tokens of the {w.name} batch (routing, capacity, expert "
+                         f"FFNs, combine in fp64 NumPy), {secs:.1f} s"}
+
+    up_ms = stage_ms["ffn_up"]
+    hbm = peaks["hbm_gbs"]
+    stages = {}
+    for s in M.STAGES:
+        ms = stage_ms[s]
+        rec = {"ms": round(ms, 5)}
+        if s in flop:
+            rec["tflops"] = round(flop[s] / (ms / 1e3) / 1e12, 2) if ms > 0 else None
+        rec["gbs"] = round(byts[s] / (ms / 1e3) / 1e9, 1) if ms > 0 else None
+        if s in ("route", "permute", "combine") and rec["gbs"]:
+            rec["frac_hbm"] = round(rec["gbs"] / hbm, 4)
+        stages[s] = rec
+    roof_peak = peaks["bf16_tflops_sustained"]
+    achieved = flop["ffn_up"] / (up_ms / 1e3) / 1e12 if up_ms > 0 else None
+    roofline = {
+        "kernel": "ffn_tc_kernel<SwiGLU> (grouped up projection)",
+        "bound": "tensor", "achieved": round(achieved, 2) if achieved else None,
+        "peak": roof_peak, "unit": "TFLOP/s",
+        "frac": round(achieved / roof_peak, 4) if achieved else None,
+        "traffic": traffic_for("ffn_tc.cu", "ffn_up"),
+        "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",
+    }
+
+    if rank == 0:
+        line = {
+            "metric": "MoE layer fwd tokens/s (and TFLOPS as a fraction of bf16 dense peak) on 1 B200",
+            "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded; random-init weights)",
+            "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "H": w.H,
+                       "act": w.act, "capacity_factor": w.cf, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (expert weights "
+                             f"{(3 if w.act == 'swiglu' else 2) * w.E * w.d * w.H * (2 if w.dtype == 'bf16' else 4) / 1e9:.2f} GB"
+                             " stream from HBM every step)"},
+            "tflops": round(tflops, 2),
+            "frac_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+            "frac_bf16_peak_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
+            "kept_assignments": n_kept, "flop_per_step": total_flop,
+            "stages": stages, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 6 * a.steps, "clocks": clk, "peaks": {**peaks, "source": peak_src},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(a, w, rank, world):
+    """The oracle as it stands, on the host cores, on bounded samples of the
+    same workload (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import torch
+    from mixture_experts_layer_51_b200.workloads import make_inputs
+    inp = make_inputs(w, "cuda" if torch.cuda.is_available() else "cpu")
+    cpu_inp = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    del inp
+    T_s = a.cpu_sample or max(8, default_cpu_sample(w) // 4)
+    for _ in range(a.warmup):
+        oracle_sample_seconds(w, cpu_inp, T_s)
+    secs = [oracle_sample_seconds(w, cpu_inp, T_s) for _ in range(a.steps)]
+    total = sum(secs)
+    value = T_s * a.steps / total
+    cores = cpu_threads()
+    line = {
+        "metric": "MoE layer fwd tokens/s (and TFLOPS as a fraction of bf16 dense peak) on 1 B200",
+        "impl": "reference", "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(total / a.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "H": w.H,
+                   "act": w.act, "capacity_factor": w.cf},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"each step: first {T_s} tokens of the {w.name} batch"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

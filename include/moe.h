@@ -1,0 +1,228 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the forward pass of one token-choice
+ * Mixture-of-Experts FFN layer on an NVIDIA B200 (sm_100a).
+ *
+ * The layer (pages: "How do Mixture of Expert Models Work?", section "The
+ * Math Behind MoEs"; "[Paper Club] Upcycling Large Language Models into
+ * Mixture of Experts", the walk-through of the MoE layer's steps):
+ *
+ *     logits = x . W_g (+ bias)                  router GEMM
+ *     G(x)   = Softmax(TopK(logits))             k gates, summing to one
+ *     permute tokens into one block per expert, keeping at most C per expert
+ *     E_e(x) = (SiLU(x W1_e) * (x W3_e)) W2_e    SwiGLU expert (or GELU)
+ *     y_t    = sum_j G_tj E_{idx_tj}(x_t)        un-permute + weighted sum
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer argument is a DEVICE pointer unless the name says host.
+ *   The caller allocates and owns every buffer; the library never allocates
+ *   or frees device memory and keeps no pointer after a call returns.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  All work is enqueued on it; calls return without waiting for
+ *   the GPU, except that moe_forward with a non-NULL `stats` and
+ *   moe_forward_host wait for their own stream before returning.
+ * - Layouts are row-major and dense: x [T, d]; W_g [d, E]; W1, W3 [E, d, H];
+ *   W2 [E, H, d]; y [T, d]; idx, gate, pos [T, k].
+ * - Element types: MOE_BF16 means x, W_g, W1, W3, W2, xp, h and y are bf16;
+ *   MOE_FP32 means they are fp32.  Router bias, gates, margins and the
+ *   expert output `o` are always fp32; indices and counts are int32.
+ * - Limits: 1 <= k <= E <= 64, k <= 8, d % 8 == 0, H % 8 == 0, T >= 0.
+ *   T == 0 is valid and does nothing.  Pointers must be 16-byte aligned.
+ * - Errors: arguments are checked on the host before anything is enqueued;
+ *   a bad argument returns MOE_ERR_ARG and enqueues nothing.  A failed CUDA
+ *   call returns MOE_ERR_CUDA.  Kernels that wait on on-chip barriers give
+ *   up after a bounded time and set a device error word, reported as
+ *   MOE_ERR_DEVICE by moe_forward (when it synchronises) or readable by the
+ *   caller.  Nothing aborts the process or throws across the ABI.
+ *
+ * Permuted layout (moe_permute -> moe_grouped_ffn -> moe_unpermute_combine)
+ * -------------------------------------------------------------------------
+ * Expert e's kept assignments occupy rows [offsets[e], offsets[e] +
+ * kept_counts[e]) of xp/h/o, in ascending token position.  Each expert's
+ * block starts on a multiple of MOE_ROW_ALIGN rows:
+ *     offsets[0] = 0,  offsets[e+1] = offsets[e] + roundup(kept_counts[e], 128).
+ * Rows between kept_counts[e] and the next block are padding: never read
+ * into y, and their contents are unspecified.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_MAX_EXPERTS 64
+#define MOE_MAX_TOPK 8
+#define MOE_ROW_ALIGN 128
+#define MOE_ABI_VERSION 1
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,          /* invalid argument; nothing was enqueued */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. no sm_100 GPU) */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE = 4        /* a kernel reported an error through its error word */
+} moe_status;
+
+typedef enum { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype;
+typedef enum { MOE_SWIGLU = 0, MOE_GELU = 1 } moe_act;
+
+/* Filled by moe_forward when `stats` is non-NULL (after the stream drains). */
+typedef struct {
+  int32_t counts[MOE_MAX_EXPERTS];      /* assignments routed to each expert */
+  int32_t kept_counts[MOE_MAX_EXPERTS]; /* min(counts, C)                    */
+  int64_t assignments;                  /* T * k                             */
+  int64_t kept;                         /* sum of kept_counts                */
+  int32_t capacity;                     /* C, or -1 when dropless            */
+  int32_t device_error;                 /* 0 = no kernel reported an error   */
+} moe_stats;
+
+/* Byte offsets of the intermediates inside the moe_forward workspace, so a
+ * caller can read them after a forward (all 256-byte aligned). */
+typedef struct {
+  size_t idx;          /* int32 [T, k]   selected experts, slot order       */
+  size_t gate;         /* fp32  [T, k]   Softmax(TopK) gates                */
+  size_t margin;       /* fp32  [T]      k-th minus (k+1)-th largest logit  */
+  size_t pos;          /* int32 [T, k]   row in xp/h/o, or -1 if dropped    */
+  size_t counts;       /* int32 [E]                                         */
+  size_t kept_counts;  /* int32 [E]                                         */
+  size_t offsets;      /* int32 [E + 1]                                     */
+  size_t dev_error;    /* int32 [1]      device error word                  */
+  size_t scratch;      /* permute scratch (moe_permute_workspace_bytes)     */
+  size_t xp;           /* dtype [rows, d] permuted tokens                   */
+  size_t h;            /* dtype [rows, H] expert hidden activations         */
+  size_t o;            /* fp32  [rows, d] expert outputs                    */
+  size_t total;        /* == moe_workspace_bytes(...)                       */
+  int64_t rows;        /* rows of xp/h/o (moe_max_permuted_rows)            */
+} moe_ws_layout;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status s);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int32_t moe_abi_version(void);
+
+/* Per-expert capacity C = ceil(cf * T * k / E), evaluated in double
+ * ("How do Mixture of Expert Models Work?", "Expert Capacity").  Returns -1
+ * when the layer is dropless (cf <= 0, NaN or +inf). */
+int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double capacity_factor);
+
+/* Rows a permuted buffer (xp, h, o) needs for any routing of T tokens:
+ * min(T*k, E*C) kept assignments plus up to 127 padding rows per expert.
+ * Returns -1 on invalid sizes. */
+int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double capacity_factor);
+
+/* Scratch bytes moe_permute needs in `ws` (per-block counts and a counter). */
+size_t moe_permute_workspace_bytes(int32_t T, int32_t E);
+
+/* Workspace bytes moe_forward needs; 0 on invalid sizes. */
+size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                           double capacity_factor, moe_dtype dtype, moe_act act);
+
+/* Where each intermediate lives inside the moe_forward workspace.
+ * Returns MOE_ERR_ARG on invalid sizes or a NULL `out`. */
+moe_status moe_workspace_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                double capacity_factor, moe_dtype dtype, moe_act act,
+                                moe_ws_layout* out);
+
+/* Router GEMM + TopK + gating softmax ("The Math Behind MoEs":
+ * Softmax(TopK(x . W_g)); "[Paper Club] Upcycling ...": the router is a
+ * learnable matrix and the expert indices are the highest-probability
+ * experts).
+ *   x [T, d], Wg [d, E] (dtype); bias [E] fp32 or NULL (added to the logits
+ *   before TopK and kept in the softmax).
+ *   Out: idx [T, k] int32 in descending-logit order, equal logits -> lower
+ *   expert first; gate [T, k] fp32 = softmax over the k selected logits;
+ *   margin [T] fp32 or NULL = k-th minus (k+1)-th largest logit (+inf when
+ *   k == E).  Logits are accumulated in fp32 and never stored. */
+moe_status moe_route(const void* x, const void* Wg, const float* bias,
+                     int32_t T, int32_t d, int32_t E, int32_t k, moe_dtype dtype,
+                     int32_t* idx, float* gate, float* margin, void* stream);
+
+/* Permutation with optional capacity ("[Paper Club] Upcycling ...": tokens
+ * that selected expert e are gathered into one matrix for e, and some are
+ * dropped depending on the capacity factor; "Take a Closer Look at the MoE
+ * LLM Routing", "Drop-towards-the-End": the earliest C assignments of each
+ * expert, in token position, are kept).
+ *   x [T, d] (dtype), idx [T, k] int32 from moe_route.
+ *   capacity_factor <= 0 (or +inf) = dropless; else C = moe_capacity(...).
+ *   Out: xp [xp_rows, d] (dtype) with the permuted layout above (xp_rows >=
+ *   moe_max_permuted_rows); pos [T, k] int32 = row of (t, j) in xp, or -1
+ *   if dropped; counts [E], kept_counts [E], offsets [E+1] int32.
+ *   ws: device scratch of at least moe_permute_workspace_bytes(T, E).
+ *   Deterministic: the result does not depend on scheduling. */
+moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d,
+                       int32_t E, int32_t k, double capacity_factor, moe_dtype dtype,
+                       void* xp, int64_t xp_rows, int32_t* pos, int32_t* counts,
+                       int32_t* kept_counts, int32_t* offsets,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped expert FFN over the per-expert blocks ("[Paper Club] Upcycling
+ * ...": one grouped GEMM over any number of experts and tokens instead of a
+ * loop over experts; Mixtral's SwiGLU expert in "The Math Behind MoEs").
+ *   xp [rows, d] (dtype), offsets [E+1], kept_counts [E] as from moe_permute.
+ *   W1, W3 [E, d, H] (W3 unused and may be NULL for MOE_GELU), W2 [E, H, d].
+ *   Out: h [rows, H] (dtype) = SiLU(xp W1_e) * (xp W3_e)  or GELU(xp W1_e);
+ *        o [rows, d] fp32 = h W2_e.  Only kept rows are written.
+ *   dev_error: int32 device word; a kernel that gives up on a bounded wait
+ *   ORs a nonzero code into it (the caller zeroes it beforehand).
+ *   bf16 runs on the tcgen05 tensor cores with fp32 accumulation (h is
+ *   rounded to bf16 before the second GEMM); fp32 runs on fp32 FMA. */
+moe_status moe_grouped_ffn(const void* xp, int64_t rows, const int32_t* offsets,
+                           const int32_t* kept_counts, const void* W1, const void* W3,
+                           const void* W2, int32_t E, int32_t d, int32_t H, moe_act act,
+                           moe_dtype dtype, void* h, float* o, int32_t* dev_error,
+                           void* stream);
+
+/* Un-permute and gate-weighted combine ("[Paper Club] Upcycling ...": the
+ * tokens are put back in their original order and scaled by the router
+ * probability; y = sum_i G(x)_i E_i(x)).
+ *   o [rows, d] fp32, pos [T, k], gate [T, k].
+ *   Out: y [T, d] (dtype), y_t = sum over kept j, in slot order, of
+ *   gate[t,j] * o[pos[t,j]], accumulated in fp32 and rounded once; a token
+ *   with every slot dropped gets y_t = 0.  No atomics: deterministic. */
+moe_status moe_unpermute_combine(const float* o, const int32_t* pos, const float* gate,
+                                 int32_t T, int32_t d, int32_t k, moe_dtype dtype,
+                                 void* y, void* stream);
+
+/* The whole layer: moe_route -> moe_permute -> moe_grouped_ffn ->
+ * moe_unpermute_combine on one stream with no host synchronisation (unless
+ * `stats` is non-NULL).  ws: device workspace of at least
+ * moe_workspace_bytes(...); its intermediates stay readable afterwards at
+ * the offsets moe_workspace_layout reports. */
+moe_status moe_forward(const void* x, const void* Wg, const float* bias,
+                       const void* W1, const void* W3, const void* W2,
+                       int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                       double capacity_factor, moe_act act, moe_dtype dtype,
+                       void* y, void* ws, size_t ws_bytes, moe_stats* stats,
+                       void* stream);
+
+/* moe_forward with the tokens in HOST memory: copies x_host [T, d] to
+ * x_dev, runs the layer, copies y back to y_host [T, d], and waits for the
+ * stream.  x_dev and y_dev are caller-owned device buffers of T*d elements.
+ * Host buffers may be pageable; pinned memory gives full PCIe bandwidth. */
+moe_status moe_forward_host(const void* x_host, void* y_host, void* x_dev, void* y_dev,
+                            const void* Wg, const float* bias, const void* W1,
+                            const void* W3, const void* W2, int32_t T, int32_t d,
+                            int32_t H, int32_t E, int32_t k, double capacity_factor,
+                            moe_act act, moe_dtype dtype, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Stage timing.  `events` points to MOE_NUM_STAGE_EVENTS cudaEvent_t
+ * handles (passed as void*) created by the caller, or is NULL to stop.  The
+ * next moe_forward / moe_forward_host calls on the calling host thread
+ * record them on their stream: [0] before the router, [1] after the router,
+ * [2] after the permutation, [3] after the up projection, [4] after the down
+ * projection, [5] after the combine.  The handles are copied; the events
+ * themselves stay owned by the caller and must outlive those calls. */
+#define MOE_NUM_STAGE_EVENTS 6
+moe_status moe_set_stage_events(void* const* events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

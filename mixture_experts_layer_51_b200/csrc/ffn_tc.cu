@@ -1,0 +1,530 @@
+// Grouped expert FFN on the B200 5th-generation tensor cores (tcgen05).
+//
+// Pages: "[Paper Club] Upcycling Large Language Models into Mixture of
+// Experts" -- the per-expert loop of GEMMs is replaced by one grouped GEMM
+// that takes any number of experts and any number of tokens per expert;
+// "How do Mixture of Expert Models Work?", "The Math Behind MoEs" -- Mixtral's
+// experts are SwiGLU FFNs.  The pages name a CUTLASS grouped GEMM for this
+// step but give no design; this kernel is written for sm_100a from scratch.
+//
+// Two launches of one persistent, warp-specialised kernel:
+//   up:   h[rows, H] = SiLU(xp W1_e) * (xp W3_e)   (bf16 out; GELU variant)
+//   down: o[rows, d] = h W2_e                      (fp32 out)
+// Tiles are 128 rows x 256 accumulator columns.  For the up projection the
+// 256 columns are 128 columns of W1 next to the same 128 columns of W3, so
+// one accumulator holds both halves of the SwiGLU and the epilogue writes
+// SiLU(gate) * up directly: the two pre-activations never reach HBM.
+//
+// Roles (192 threads):
+//   warp 0      one thread issues TMA loads of A (K-major, 128B swizzle) and
+//               B (weights [E, K, N] read N-major, 128B swizzle) into a
+//               4-stage shared-memory ring;
+//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
+//               fp32 accumulate in tensor memory) and commits stage releases;
+//               the warp also owns the 512-column TMEM allocation (two
+//               accumulators, so the epilogue of tile i overlaps the MMAs of
+//               tile i+1);
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, activation,
+//               16-byte global stores of the kept rows.
+// The tile list (expert, m-block, n-block) is built on the device from the
+// per-expert offsets, with the experts that have the most m-blocks first and
+// m-blocks fastest, so concurrent CTAs share weight tiles in L2.  No host
+// synchronisation is needed between the permutation and this kernel.
+//
+// Every wait on an mbarrier is bounded; on timeout a thread records an error
+// bit, raises an abort flag, lets in-flight copies and MMAs land, frees TMEM
+// and returns.  No TMA multicast is used anywhere.
+
+#include <math.h>
+#include <stdio.h>
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int TM = 128;  // tile rows (UMMA M)
+constexpr int TN = 256;  // accumulator columns (UMMA N)
+constexpr int TK = 64;   // K per stage: one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = TM * TK * 2;    // 16 KB
+constexpr int B_BYTES = TN * TK * 2;    // 32 KB
+constexpr int B_BOX_BYTES = 64 * TK * 2;  // one 64-column x 64-row box: 8 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * TN;
+constexpr int CONTROL_BYTES = 2048;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CONTROL_BYTES + 1024;  // + alignment slack
+
+enum Epi { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_PLAIN_F32 = 2 };
+
+struct TcParams {
+  void* out;
+  int64_t ld_out;  // elements per output row
+  int n_out;       // valid output columns
+  int K;           // reduction length
+  int E;
+  int n_tiles;     // column tiles per expert
+  int64_t rows;    // rows of the A and output buffers
+  const int32_t* offsets;
+  const int32_t* kept;
+  int32_t* err;
+};
+
+struct Control {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+  int total_tiles;
+  int n_sched;
+  int sched_e[kMaxE];
+  int sched_mt[kMaxE];
+  int sched_prefix[kMaxE + 1];
+  int off[kMaxE];
+  int kept[kMaxE];
+};
+static_assert(sizeof(Control) <= CONTROL_BYTES, "control block too large");
+
+__device__ __forceinline__ void decode_tile(const Control& c, int t, int& e, int& m, int& n) {
+  int s = 0;
+  while (s + 1 < c.n_sched && c.sched_prefix[s + 1] <= t) ++s;
+  e = c.sched_e[s];
+  const int local = t - c.sched_prefix[s];
+  const int mt = c.sched_mt[s];
+  n = local / mt;
+  m = local - n * mt;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float gelu_f(float z) {
+  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                  const __grid_constant__ CUtensorMap tmB1, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Control& c = *reinterpret_cast<Control*>(smem + STAGES * STAGE_BYTES);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ------------------------------------------------------------ set-up
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&c.full[s]), 1);
+      mbar_init(smem_u32(&c.empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&c.tfull[a]), 1);
+      mbar_init(smem_u32(&c.tempty[a]), 4);  // one arrive per epilogue warp
+    }
+    mbar_init(smem_u32(&c.drain), 1);
+    c.abort_flag = 0;
+    fence_mbar_init();
+    fence_async_shared();
+  }
+  if (tid < p.E) {
+    c.off[tid] = p.offsets[tid];
+    c.kept[tid] = p.kept[tid];
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&c.tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // Schedule: experts with more m-blocks first (stable), empty ones skipped.
+    int n = 0;
+    for (int e = 0; e < p.E; ++e) {
+      const int mt = (c.kept[e] + TM - 1) / TM;
+      if (mt <= 0) continue;
+      // An expert block must start on a tile boundary and end inside the
+      // buffers; anything else is reported and skipped, never written.
+      if (c.off[e] < 0 || (c.off[e] % TM) != 0 ||
+          static_cast<int64_t>(c.off[e]) + static_cast<int64_t>(mt) * TM > p.rows) {
+        atomicOr(p.err, kErrRowOverflow);
+        continue;
+      }
+      int q = n;
+      while (q > 0 && c.sched_mt[q - 1] < mt) {
+        c.sched_mt[q] = c.sched_mt[q - 1];
+        c.sched_e[q] = c.sched_e[q - 1];
+        --q;
+      }
+      c.sched_mt[q] = mt;
+      c.sched_e[q] = e;
+      ++n;
+    }
+    int acc = 0;
+    for (int s = 0; s < n; ++s) {
+      c.sched_prefix[s] = acc;
+      acc += c.sched_mt[s] * p.n_tiles;
+    }
+    c.sched_prefix[n] = acc;
+    c.n_sched = n;
+    c.total_tiles = acc;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  const int total = c.total_tiles;
+  const int nk = (p.K + TK - 1) / TK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      bool ok = true, timed_out = false;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int e, m, n;
+        decode_tile(c, t, e, m, n);
+        const int row0 = c.off[e] + m * TM;
+        for (int kb = 0; kb < nk; ++kb) {
+          const uint32_t empty_bar = smem_u32(&c.empty[stage]);
+          if (!mbar_wait(empty_bar, phase ^ 1)) {
+            ok = false;
+            timed_out = true;
+            break;
+          }
+          if (c.abort_flag) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_bar = smem_u32(&c.full[stage]);
+          const uint32_t a_dst = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t b_dst = a_dst + A_BYTES;
+          mbar_arrive_expect_tx(full_bar, STAGE_BYTES);
+          tma_load_2d(a_dst, &tmA, full_bar, kb * TK, row0);
+          if (EPI == EPI_SWIGLU) {
+            const int n0 = n * (TN / 2);
+            tma_load_3d(b_dst + 0 * B_BOX_BYTES, &tmB0, full_bar, n0, kb * TK, e);
+            tma_load_3d(b_dst + 1 * B_BOX_BYTES, &tmB0, full_bar, n0 + 64, kb * TK, e);
+            tma_load_3d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_bar, n0, kb * TK, e);
+            tma_load_3d(b_dst + 3 * B_BOX_BYTES, &tmB1, full_bar, n0 + 64, kb * TK, e);
+          } else {
+            const int n0 = n * TN;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tma_load_3d(b_dst + q * B_BOX_BYTES, &tmB0, full_bar, n0 + 64 * q, kb * TK, e);
+          }
+#pragma unroll
+          for (int s = 0; s < STAGES; ++s)
+            if (s == stage) ++issued[s];
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (ok) {
+        // Tail: wait until the MMA warp has released every stage, so no
+        // tcgen05.commit arrival is still in flight when the CTA exits.
+        for (int i = 0; i < STAGES; ++i) {
+          if (!mbar_wait(smem_u32(&c.empty[stage]), phase ^ 1)) {
+            timed_out = true;
+            break;
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok || timed_out) {
+        if (timed_out) atomicOr(p.err, kErrTimeoutProducer);
+        c.abort_flag = 1;
+        // Let every issued copy land before the shared memory goes away.
+        for (int s = 0; s < STAGES; ++s) {
+          if (issued[s] > 0 &&
+              !mbar_wait(smem_u32(&c.full[s]), static_cast<uint32_t>(issued[s] - 1) & 1u))
+            atomicOr(p.err, kErrTimeoutDrain);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TM, TN, false, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true, timed_out = false, issued_any = false;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (!mbar_wait(smem_u32(&c.tempty[acc]), acc_phase ^ 1)) {
+          ok = false;
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * TN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&c.full[stage]), phase)) {
+            ok = false;
+            timed_out = true;
+            break;
+          }
+          if (c.abort_flag) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TK / 16; ++kk) {
+            // A: K-major, advance 16 elements (32 bytes) inside the swizzled row.
+            const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            // B: N-major, 64-column boxes 8 KB apart; advance 16 K-rows (2 KB).
+            const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, B_BOX_BYTES, 1024);
+            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(smem_u32(&c.empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&c.tfull[acc]));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      if (!ok) {
+        if (timed_out) atomicOr(p.err, kErrTimeoutMma);
+        c.abort_flag = 1;
+        if (issued_any) {
+          // Wait for the MMAs already issued before TMEM is freed.
+          tc_commit(smem_u32(&c.drain));
+          if (!mbar_wait(smem_u32(&c.drain), 0)) atomicOr(p.err, kErrTimeoutDrain);
+        }
+      }
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
+    const int row = quad * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      int e, m, n;
+      decode_tile(c, t, e, m, n);
+      if (!mbar_wait(smem_u32(&c.tfull[acc]), acc_phase)) {
+        atomicOr(p.err, kErrTimeoutEpilogue);
+        c.abort_flag = 1;
+        break;
+      }
+      if (c.abort_flag) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(acc * TN);
+      const bool row_ok = row < c.kept[e] - m * TM;
+      const int64_t grow = static_cast<int64_t>(c.off[e]) + m * TM + row;
+      if (EPI == EPI_SWIGLU) {
+        const int n0 = n * (TN / 2);
+        __nv_bfloat16* dst_row = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float g[32], u[32];
+          tc_ld_32cols(tbase + cc * 32, g);
+          tc_ld_32cols(tbase + TN / 2 + cc * 32, u);
+          tc_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = n0 + cc * 32 + v * 8;
+              if (col < p.n_out) {
+                uint4 pk;
+                pk.x = pack_bf16x2(silu_f(g[v * 8 + 0]) * u[v * 8 + 0],
+                                   silu_f(g[v * 8 + 1]) * u[v * 8 + 1]);
+                pk.y = pack_bf16x2(silu_f(g[v * 8 + 2]) * u[v * 8 + 2],
+                                   silu_f(g[v * 8 + 3]) * u[v * 8 + 3]);
+                pk.z = pack_bf16x2(silu_f(g[v * 8 + 4]) * u[v * 8 + 4],
+                                   silu_f(g[v * 8 + 5]) * u[v * 8 + 5]);
+                pk.w = pack_bf16x2(silu_f(g[v * 8 + 6]) * u[v * 8 + 6],
+                                   silu_f(g[v * 8 + 7]) * u[v * 8 + 7]);
+                *reinterpret_cast<uint4*>(dst_row + col) = pk;
+              }
+            }
+          }
+        }
+      } else if (EPI == EPI_GELU) {
+        const int n0 = n * TN;
+        __nv_bfloat16* dst_row = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out;
+#pragma unroll 1
+        for (int cc = 0; cc < TN / 32; ++cc) {
+          float g[32];
+          tc_ld_32cols(tbase + cc * 32, g);
+          tc_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int col = n0 + cc * 32 + v * 8;
+              if (col < p.n_out) {
+                uint4 pk;
+                pk.x = pack_bf16x2(gelu_f(g[v * 8 + 0]), gelu_f(g[v * 8 + 1]));
+                pk.y = pack_bf16x2(gelu_f(g[v * 8 + 2]), gelu_f(g[v * 8 + 3]));
+                pk.z = pack_bf16x2(gelu_f(g[v * 8 + 4]), gelu_f(g[v * 8 + 5]));
+                pk.w = pack_bf16x2(gelu_f(g[v * 8 + 6]), gelu_f(g[v * 8 + 7]));
+                *reinterpret_cast<uint4*>(dst_row + col) = pk;
+              }
+            }
+          }
+        }
+      } else {
+        const int n0 = n * TN;
+        float* dst_row = static_cast<float*>(p.out) + grow * p.ld_out;
+#pragma unroll 1
+        for (int cc = 0; cc < TN / 32; ++cc) {
+          float g[32];
+          tc_ld_32cols(tbase + cc * 32, g);
+          tc_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int col = n0 + cc * 32 + v * 4;
+              if (col < p.n_out)
+                *reinterpret_cast<float4*>(dst_row + col) =
+                    make_float4(g[v * 4 + 0], g[v * 4 + 1], g[v * 4 + 2], g[v * 4 + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&c.tempty[acc]));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  // ---------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 2-D bf16 matrix [rows, cols] (cols contiguous), box = 64 cols x box_rows.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D bf16 weights [E, K, N] (N contiguous), box = 64 (N) x 64 (K) x 1.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {N, K, E};
+  cuuint64_t strides[2] = {N * 2, K * N * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const TcParams& p, int grid, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  ffn_tc_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEvent_t between) {
+  if (a.rows <= 0) return MOE_OK;
+  CUtensorMap mx, mw1, mw3, mh, mw2;
+  const bool swiglu = a.act == MOE_SWIGLU;
+  if (!make_map_2d(&mx, a.xp, a.rows, a.d, TM) || !make_map_3d(&mw1, a.W1, a.E, a.d, a.H) ||
+      (swiglu && !make_map_3d(&mw3, a.W3, a.E, a.d, a.H)) ||
+      !make_map_2d(&mh, a.h, a.rows, a.H, TM) || !make_map_3d(&mw2, a.W2, a.E, a.H, a.d))
+    return MOE_ERR_CUDA;
+  const int64_t mtiles_max = (a.rows + TM - 1) / TM;
+
+  TcParams up{};
+  up.out = a.h;
+  up.ld_out = a.H;
+  up.n_out = a.H;
+  up.K = a.d;
+  up.E = a.E;
+  up.n_tiles = swiglu ? (a.H + TN / 2 - 1) / (TN / 2) : (a.H + TN - 1) / TN;
+  up.rows = a.rows;
+  up.offsets = a.offsets;
+  up.kept = a.kept_counts;
+  up.err = a.dev_error;
+  int grid = static_cast<int>(std::min<int64_t>(num_sms, mtiles_max * up.n_tiles));
+  cudaError_t err = swiglu ? launch_one<EPI_SWIGLU>(mx, mw1, mw3, up, grid, s)
+                           : launch_one<EPI_GELU>(mx, mw1, mw1, up, grid, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (between && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  TcParams dn{};
+  dn.out = a.o;
+  dn.ld_out = a.d;
+  dn.n_out = a.d;
+  dn.K = a.H;
+  dn.E = a.E;
+  dn.n_tiles = (a.d + TN - 1) / TN;
+  dn.rows = a.rows;
+  dn.offsets = a.offsets;
+  dn.kept = a.kept_counts;
+  dn.err = a.dev_error;
+  grid = static_cast<int>(std::min<int64_t>(num_sms, mtiles_max * dn.n_tiles));
+  err = launch_one<EPI_PLAIN_F32>(mh, mw2, mw2, dn, grid, s);
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

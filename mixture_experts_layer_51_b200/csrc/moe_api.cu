@@ -1,0 +1,347 @@
+// C ABI of libmoe.so: argument checks, workspace layout and the one-stream
+// orchestration of route -> permute -> grouped FFN -> combine.  Every entry
+// point is declared and documented in include/moe.h.
+
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "moe_internal.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t elt_size(moe_dtype dt) { return dt == MOE_BF16 ? 2 : 4; }
+
+bool valid_dtype(moe_dtype dt) { return dt == MOE_BF16 || dt == MOE_FP32; }
+bool valid_act(moe_act a) { return a == MOE_SWIGLU || a == MOE_GELU; }
+
+bool valid_route_sizes(int32_t T, int32_t d, int32_t E, int32_t k) {
+  return T >= 0 && d > 0 && d % 8 == 0 && E >= 1 && E <= kMaxE && k >= 1 && k <= kMaxK && k <= E;
+}
+bool valid_ffn_sizes(int32_t d, int32_t H) { return d > 0 && d % 8 == 0 && H > 0 && H % 8 == 0; }
+
+int capacity_or_max(int32_t T, int32_t E, int32_t k, double cf) {
+  const int32_t C = moe_capacity(T, E, k, cf);
+  return C < 0 ? INT32_MAX : C;
+}
+
+// Stage events set by moe_set_stage_events for this host thread.
+thread_local cudaEvent_t g_stage_events[MOE_NUM_STAGE_EVENTS] = {};
+thread_local bool g_stage_events_on = false;
+
+moe_status record_stage(int i, cudaStream_t s) {
+  if (!g_stage_events_on) return MOE_OK;
+  return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+struct DeviceInfo {
+  int device = -1;
+  int num_sms = 0;
+  int major = 0;
+};
+
+moe_status device_info(DeviceInfo* out) {
+  static std::atomic<int> sms_cache[64];
+  static std::atomic<int> major_cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  out->device = dev;
+  if (dev >= 0 && dev < 64 && sms_cache[dev].load() > 0) {
+    out->num_sms = sms_cache[dev].load();
+    out->major = major_cache[dev].load();
+  } else {
+    if (cudaDeviceGetAttribute(&out->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&out->major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (dev >= 0 && dev < 64) {
+      major_cache[dev].store(out->major);
+      sms_cache[dev].store(out->num_sms);
+    }
+  }
+  // The library carries sm_100a code only.
+  return out->major == 10 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+bool compute_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, double cf,
+                    moe_dtype dt, moe_act act, moe_ws_layout* L) {
+  if (!valid_route_sizes(T, d, E, k) || !valid_ffn_sizes(d, H) || !valid_dtype(dt) ||
+      !valid_act(act))
+    return false;
+  const int64_t rows = moe_max_permuted_rows(T, E, k, cf);
+  if (rows < 0) return false;
+  const size_t tk = static_cast<size_t>(T) * k;
+  const size_t es = elt_size(dt);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  memset(L, 0, sizeof(*L));
+  L->idx = take(tk * 4);
+  L->gate = take(tk * 4);
+  L->margin = take(static_cast<size_t>(T) * 4);
+  L->pos = take(tk * 4);
+  L->counts = take(kMaxE * 4);
+  L->kept_counts = take(kMaxE * 4);
+  L->offsets = take((kMaxE + 1) * 4);
+  L->dev_error = take(4);
+  L->scratch = take(permute_scratch_bytes(T, E));
+  L->xp = take(static_cast<size_t>(rows) * d * es);
+  L->h = take(static_cast<size_t>(rows) * H * es);
+  L->o = take(static_cast<size_t>(rows) * d * 4);
+  L->total = off;
+  L->rows = rows;
+  return true;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+MOE_API const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_ARG: return "MOE_ERR_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: not supported on this device/config";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE: a kernel reported an error";
+  }
+  return "MOE_UNKNOWN_STATUS";
+}
+
+MOE_API int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+MOE_API int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double cf) {
+  if (!(cf > 0.0) || isinf(cf) || E <= 0 || T < 0 || k <= 0) return -1;
+  const double c = ceil(cf * static_cast<double>(T) * static_cast<double>(k) / static_cast<double>(E));
+  if (c > static_cast<double>(INT32_MAX)) return INT32_MAX;
+  return static_cast<int32_t>(c);
+}
+
+MOE_API int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double cf) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return -1;
+  if (T == 0) return 0;
+  const int64_t tk = static_cast<int64_t>(T) * k;
+  const int32_t C = moe_capacity(T, E, k, cf);
+  int64_t rows = tk + static_cast<int64_t>(E) * (kRowAlign - 1);
+  if (C >= 0) rows = std::min<int64_t>(rows, static_cast<int64_t>(E) * pad_rows(C));
+  return pad_rows(std::max<int64_t>(rows, kRowAlign));
+}
+
+MOE_API size_t moe_permute_workspace_bytes(int32_t T, int32_t E) {
+  if (T < 0 || E < 1 || E > kMaxE) return 0;
+  return permute_scratch_bytes(T, E);
+}
+
+MOE_API size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                   double cf, moe_dtype dt, moe_act act) {
+  moe_ws_layout L;
+  return compute_layout(T, d, H, E, k, cf, dt, act, &L) ? L.total : 0;
+}
+
+MOE_API moe_status moe_workspace_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                        double cf, moe_dtype dt, moe_act act, moe_ws_layout* out) {
+  if (!out) return MOE_ERR_ARG;
+  return compute_layout(T, d, H, E, k, cf, dt, act, out) ? MOE_OK : MOE_ERR_ARG;
+}
+
+MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, int32_t T,
+                             int32_t d, int32_t E, int32_t k, moe_dtype dt, int32_t* idx,
+                             float* gate, float* margin, void* stream) {
+  if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wg || !idx || !gate || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  RouteArgs a{x, Wg, bias, T, d, E, k, idx, gate, margin};
+  return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d, int32_t E,
+                               int32_t k, double cf, moe_dtype dt, void* xp, int64_t xp_rows,
+                               int32_t* pos, int32_t* counts, int32_t* kept_counts,
+                               int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
+  if (!counts || !kept_counts || !offsets) return MOE_ERR_ARG;
+  if (T > 0) {
+    if (!x || !idx || !xp || !pos || !ws || !aligned16(x) || !aligned16(xp) ||
+        !aligned16(ws))
+      return MOE_ERR_ARG;
+    if (xp_rows < moe_max_permuted_rows(T, E, k, cf)) return MOE_ERR_ARG;
+    if (ws_bytes < permute_scratch_bytes(T, E)) return MOE_ERR_ARG;
+  }
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  const size_t nblk = (static_cast<size_t>(T) + kPermBlock - 1) / kPermBlock;
+  int32_t* block_base = static_cast<int32_t*>(ws);
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(
+      static_cast<uint8_t*>(ws) + align_up(nblk * static_cast<size_t>(E) * 4));
+  PermuteArgs a{x, idx, T, d, E, k, capacity_or_max(T, E, k, cf), xp, pos, counts, kept_counts,
+                offsets, block_base, ticket};
+  return launch_permute(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_grouped_ffn(const void* xp, int64_t rows, const int32_t* offsets,
+                                   const int32_t* kept_counts, const void* W1, const void* W3,
+                                   const void* W2, int32_t E, int32_t d, int32_t H, moe_act act,
+                                   moe_dtype dt, void* h, float* o, int32_t* dev_error,
+                                   void* stream) {
+  if (!valid_ffn_sizes(d, H) || E < 1 || E > kMaxE || !valid_act(act) || !valid_dtype(dt) ||
+      rows < 0 || rows % kRowAlign != 0)
+    return MOE_ERR_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !offsets || !kept_counts || !W1 || !W2 || !h || !o || !dev_error) return MOE_ERR_ARG;
+  if (act == MOE_SWIGLU && !W3) return MOE_ERR_ARG;
+  if (!aligned16(xp) || !aligned16(W1) || (W3 && !aligned16(W3)) || !aligned16(W2) ||
+      !aligned16(h) || !aligned16(o))
+    return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  FfnArgs a{xp, rows, offsets, kept_counts, W1, W3, W2, E, d, H, act, h, o, dev_error};
+  cudaEvent_t between = g_stage_events_on ? g_stage_events[3] : nullptr;
+  if (dt == MOE_BF16)
+    return launch_ffn_tc(a, static_cast<cudaStream_t>(stream), di.num_sms, between);
+  return launch_ffn_simt(a, static_cast<cudaStream_t>(stream), between);
+}
+
+MOE_API moe_status moe_set_stage_events(void* const* events) {
+  if (!events) {
+    g_stage_events_on = false;
+    return MOE_OK;
+  }
+  for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i)
+    if (!events[i]) return MOE_ERR_ARG;
+  for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i)
+    g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  g_stage_events_on = true;
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_unpermute_combine(const float* o, const int32_t* pos, const float* gate,
+                                         int32_t T, int32_t d, int32_t k, moe_dtype dt, void* y,
+                                         void* stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || k < 1 || k > kMaxK || !valid_dtype(dt)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!o || !pos || !gate || !y || !aligned16(o) || !aligned16(y)) return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  CombineArgs a{o, pos, gate, T, d, k, y};
+  return launch_combine(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
+                                                                                 : MOE_ERR_CUDA;
+}
+
+namespace {
+
+moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, const void* W1,
+                           const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
+                           int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
+                           void* ws, size_t ws_bytes, const moe_ws_layout& L, cudaStream_t s) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
+  float* gate = reinterpret_cast<float*>(w + L.gate);
+  float* margin = reinterpret_cast<float*>(w + L.margin);
+  int32_t* pos = reinterpret_cast<int32_t*>(w + L.pos);
+  int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* kept = reinterpret_cast<int32_t*>(w + L.kept_counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* err = reinterpret_cast<int32_t*>(w + L.dev_error);
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  moe_status st = record_stage(0, s);
+  if (st != MOE_OK) return st;
+  st = moe_route(x, Wg, bias, T, d, E, k, dt, idx, gate, margin, s);
+  if (st == MOE_OK) st = record_stage(1, s);
+  if (st != MOE_OK) return st;
+  st = moe_permute(x, idx, T, d, E, k, cf, dt, w + L.xp, L.rows, pos, counts, kept, offsets,
+                   w + L.scratch, permute_scratch_bytes(T, E), s);
+  if (st == MOE_OK) st = record_stage(2, s);
+  if (st != MOE_OK) return st;
+  st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,
+                       reinterpret_cast<float*>(w + L.o), err, s);
+  if (st == MOE_OK) st = record_stage(4, s);
+  if (st != MOE_OK) return st;
+  st = moe_unpermute_combine(reinterpret_cast<float*>(w + L.o), pos, gate, T, d, k, dt, y, s);
+  if (st == MOE_OK) st = record_stage(5, s);
+  return st;
+}
+
+moe_status read_device_error(const moe_ws_layout& L, void* ws, cudaStream_t s, int32_t* out) {
+  if (cudaMemcpyAsync(out, static_cast<uint8_t*>(ws) + L.dev_error, sizeof(int32_t),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API moe_status moe_forward(const void* x, const void* Wg, const float* bias, const void* W1,
+                               const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
+                               int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
+                               void* ws, size_t ws_bytes, moe_stats* stats, void* stream) {
+  moe_ws_layout L;
+  if (!compute_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
+  if (T > 0 && (!y || !ws || ws_bytes < L.total || !aligned16(ws))) return MOE_ERR_ARG;
+  if (T == 0) {
+    if (stats) {
+      memset(stats, 0, sizeof(*stats));
+      stats->capacity = moe_capacity(T, E, k, cf);
+    }
+    return MOE_OK;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  moe_status st = forward_enqueue(x, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, y, ws,
+                                  ws_bytes, L, s);
+  if (st != MOE_OK || !stats) return st;
+  memset(stats, 0, sizeof(*stats));
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  if (cudaMemcpyAsync(stats->counts, w + L.counts, sizeof(int32_t) * E, cudaMemcpyDeviceToHost,
+                      s) != cudaSuccess ||
+      cudaMemcpyAsync(stats->kept_counts, w + L.kept_counts, sizeof(int32_t) * E,
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = read_device_error(L, ws, s, &stats->device_error);
+  if (st != MOE_OK) return st;
+  stats->assignments = static_cast<int64_t>(T) * k;
+  for (int e = 0; e < E; ++e) stats->kept += stats->kept_counts[e];
+  stats->capacity = moe_capacity(T, E, k, cf);
+  return stats->device_error ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+MOE_API moe_status moe_forward_host(const void* x_host, void* y_host, void* x_dev, void* y_dev,
+                                    const void* Wg, const float* bias, const void* W1,
+                                    const void* W3, const void* W2, int32_t T, int32_t d,
+                                    int32_t H, int32_t E, int32_t k, double cf, moe_act act,
+                                    moe_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+  moe_ws_layout L;
+  if (!compute_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host || !x_dev || !y_dev || !ws || ws_bytes < L.total) return MOE_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * d * elt_size(dt);
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  moe_status st = forward_enqueue(x_dev, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, y_dev,
+                                  ws, ws_bytes, L, s);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int32_t derr = 0;
+  st = read_device_error(L, ws, s, &derr);
+  if (st != MOE_OK) return st;
+  return derr ? MOE_ERR_DEVICE : MOE_OK;
+}

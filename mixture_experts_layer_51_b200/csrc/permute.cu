@@ -1,0 +1,233 @@
+// Permutation of tokens into one contiguous block per expert, with an
+// optional capacity.
+//
+// Pages: "[Paper Club] Upcycling Large Language Models into Mixture of
+// Experts" -- after routing, the tokens that chose expert e are gathered
+// into one matrix for e, and depending on the capacity factor some tokens are
+// dropped (Megatron-Core: dropless by default, or dropping with padding);
+// "How do Mixture of Expert Models Work?", "Expert Capacity"; "Take a Closer
+// Look at the MoE LLM Routing", "Drop-towards-the-End" -- the tokens that
+// arrive later in the sequence are the ones dropped.
+//
+// The kept assignments of expert e are its first C in token position, so
+// the permutation is a stable counting sort by expert:
+//   pass 1 (count): per 256-token block, per-expert counts from warp ballots;
+//     the last block to finish (atomic ticket) turns them into exclusive
+//     per-expert bases, the counts, kept counts (min(count, C)) and the
+//     128-row aligned block offsets.
+//   pass 2 (scatter): per 32-token chunk, rank = block base + counts of the
+//     preceding chunks in the block + ballot prefix inside the chunk; then
+//     the chunk's rows are copied to xp with 16-byte loads and stores.
+// Every rank is computed from counts in token order: no atomics decide
+// placement, so the output is deterministic.
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpsPerBlock = kPermBlock / 32;  // 8 chunks per block
+
+// Bit e set when token t selected expert e.  Ids outside [0, E) (possible
+// only when a caller passes its own idx) select nothing and are never kept.
+__device__ __forceinline__ uint64_t expert_mask(const int32_t* __restrict__ idx, int t, int T,
+                                                int k, int E) {
+  uint64_t m = 0;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      if (e >= 0 && e < E) m |= 1ull << e;
+    }
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(kPermBlock)
+    permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int C, int nblk,
+                         int32_t* __restrict__ block_base, unsigned int* __restrict__ ticket,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ kept_counts,
+                         int32_t* __restrict__ offsets) {
+  __shared__ int wcnt[kWarpsPerBlock][kMaxE];
+  __shared__ int padded[kMaxE];
+  __shared__ bool is_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t = blockIdx.x * kPermBlock + tid;
+  const uint64_t mask = expert_mask(idx, t, T, k, E);
+  for (int e = 0; e < E; ++e) {
+    const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
+    if (lane == 0) wcnt[warp][e] = __popc(b);
+  }
+  __syncthreads();
+  if (tid < E) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < kWarpsPerBlock; ++w) s += wcnt[w][tid];
+    block_base[(int64_t)blockIdx.x * E + tid] = s;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = (atomicAdd(ticket, 1u) == static_cast<unsigned>(nblk - 1));
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  // Last block: exclusive scan over blocks for every expert.
+  if (tid < E) {
+    int run = 0;
+    int b = 0;
+    for (; b + 8 <= nblk; b += 8) {
+      int v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __ldcg(block_base + (int64_t)(b + i) * E + tid);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        block_base[(int64_t)(b + i) * E + tid] = run;
+        run += v[i];
+      }
+    }
+    for (; b < nblk; ++b) {
+      const int v = __ldcg(block_base + (int64_t)b * E + tid);
+      block_base[(int64_t)b * E + tid] = run;
+      run += v;
+    }
+    const int kept = run < C ? run : C;
+    counts[tid] = run;
+    kept_counts[tid] = kept;
+    padded[tid] = (kept + kRowAlign - 1) / kRowAlign * kRowAlign;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int off = 0;
+    for (int e = 0; e < E; ++e) {
+      offsets[e] = off;
+      off += padded[e];
+    }
+    offsets[E] = off;
+    *ticket = 0u;  // ready for the next call on this workspace
+  }
+}
+
+template <int UNROLL>
+__global__ void __launch_bounds__(kPermBlock)
+    permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx, int T,
+                           int dvec, int E, int k, int C, const int32_t* __restrict__ block_base,
+                           const int32_t* __restrict__ offsets, int32_t* __restrict__ pos,
+                           uint4* __restrict__ xp) {
+  __shared__ int wcnt[kWarpsPerBlock][kMaxE];
+  __shared__ int base[kMaxE];
+  __shared__ int spos[kPermChunk * kMaxK];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x;
+  const int blk = chunk / kWarpsPerBlock;
+  const int cw = chunk % kWarpsPerBlock;
+
+  // Counts of the chunks that precede this one inside its 256-token block.
+  if (warp < cw) {
+    const int t = (blk * kWarpsPerBlock + warp) * kPermChunk + lane;
+    const uint64_t mask = expert_mask(idx, t, T, k, E);
+    for (int e = 0; e < E; ++e) {
+      const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
+      if (lane == 0) wcnt[warp][e] = __popc(b);
+    }
+  }
+  __syncthreads();
+  if (tid < E) {
+    int s = block_base[(int64_t)blk * E + tid];
+    for (int w = 0; w < cw; ++w) s += wcnt[w][tid];
+    base[tid] = s;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int t = chunk * kPermChunk + lane;
+    int ej[kMaxK];
+    uint64_t mask = 0;
+    for (int j = 0; j < k; ++j) {
+      ej[j] = (t < T) ? idx[(int64_t)t * k + j] : -1;
+      if (ej[j] >= 0 && ej[j] < E) mask |= 1ull << ej[j];
+    }
+    int rj[kMaxK];
+    for (int j = 0; j < k; ++j) rj[j] = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int e = 0; e < E; ++e) {
+      const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
+      if ((mask >> e) & 1ull) {
+        const int r = base[e] + __popc(b & lt);
+        for (int j = 0; j < k; ++j)
+          if (ej[j] == e) rj[j] = r;
+      }
+    }
+    for (int j = 0; j < k; ++j) {
+      int p = -1;
+      if (t < T && ej[j] >= 0 && ej[j] < E && rj[j] < C) p = offsets[ej[j]] + rj[j];
+      if (t < T) pos[(int64_t)t * k + j] = p;
+      spos[lane * k + j] = p;
+    }
+  }
+  __syncthreads();
+
+  // Copy each kept token row to its k destinations.
+  for (int i = warp; i < kPermChunk; i += kWarpsPerBlock) {
+    const int t = chunk * kPermChunk + i;
+    if (t >= T) break;
+    int p[kMaxK];
+    bool any = false;
+    for (int j = 0; j < k; ++j) {
+      p[j] = spos[i * k + j];
+      any |= p[j] >= 0;
+    }
+    if (!any) continue;
+    const uint4* src = x + (int64_t)t * dvec;
+    for (int v0 = lane; v0 < dvec; v0 += 32 * UNROLL) {
+      uint4 buf[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int v = v0 + u * 32;
+        if (v < dvec) buf[u] = __ldg(src + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        if (p[j] < 0) continue;
+        uint4* dst = xp + (int64_t)p[j] * dvec;
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          const int v = v0 + u * 32;
+          if (v < dvec) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t permute_scratch_bytes(int T, int E) {
+  const size_t nblk = (static_cast<size_t>(T) + kPermBlock - 1) / kPermBlock;
+  size_t b = nblk * static_cast<size_t>(E) * sizeof(int32_t);
+  b = (b + 255) / 256 * 256;
+  return b + 256;  // + ticket counter
+}
+
+cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s) {
+  if (a.T == 0) {
+    // Still produce well-defined counts/offsets for an empty batch.
+    cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(a.kept_counts, 0, sizeof(int32_t) * a.E, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), s);
+    return err;
+  }
+  const int nblk = (a.T + kPermBlock - 1) / kPermBlock;
+  const int nchunk = (a.T + kPermChunk - 1) / kPermChunk;
+  const int elt = dtype == MOE_BF16 ? 2 : 4;
+  const int dvec = a.d * elt / 16;
+  cudaError_t err = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned int), s);
+  if (err != cudaSuccess) return err;
+  permute_count_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.T, a.E, a.k, a.capacity, nblk,
+                                                   a.block_base, a.ticket, a.counts,
+                                                   a.kept_counts, a.offsets);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  permute_scatter_kernel<4><<<nchunk, kPermBlock, 0, s>>>(
+      static_cast<const uint4*>(a.x), a.idx, a.T, dvec, a.E, a.k, a.capacity, a.block_base,
+      a.offsets, a.pos, static_cast<uint4*>(a.xp));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

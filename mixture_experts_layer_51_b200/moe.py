@@ -1,0 +1,350 @@
+"""Thin Python binding of libmoe.so (include/moe.h), by the same names.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  Functions
+accept torch tensors, allocate missing outputs with torch, pass raw pointers
+through ctypes and raise ``MoeError`` on any non-OK status.  There is no
+fallback: if libmoe.so is missing or was not built, the first call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+MOE_OK, MOE_ERR_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(5)
+MOE_BF16, MOE_FP32 = 0, 1
+MOE_SWIGLU, MOE_GELU = 0, 1
+MOE_MAX_EXPERTS = 64
+MOE_MAX_TOPK = 8
+MOE_ROW_ALIGN = 128
+
+EXPORTED = (
+    "moe_status_string", "moe_abi_version", "moe_capacity", "moe_max_permuted_rows",
+    "moe_permute_workspace_bytes", "moe_workspace_bytes", "moe_workspace_layout",
+    "moe_route", "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine",
+    "moe_forward", "moe_forward_host", "moe_set_stage_events",
+)
+MOE_NUM_STAGE_EVENTS = 6
+STAGES = ("route", "permute", "ffn_up", "ffn_down", "combine")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class moe_stats(ctypes.Structure):
+    _fields_ = [
+        ("counts", ctypes.c_int32 * MOE_MAX_EXPERTS),
+        ("kept_counts", ctypes.c_int32 * MOE_MAX_EXPERTS),
+        ("assignments", ctypes.c_int64),
+        ("kept", ctypes.c_int64),
+        ("capacity", ctypes.c_int32),
+        ("device_error", ctypes.c_int32),
+    ]
+
+
+class moe_ws_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "idx", "gate", "margin", "pos", "counts", "kept_counts", "offsets", "dev_error",
+        "scratch", "xp", "h", "o", "total")] + [("rows", ctypes.c_int64)]
+
+
+_lib_handle = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_D = ctypes.c_double
+_SZ = ctypes.c_size_t
+
+
+def lib():
+    """The loaded libmoe.so (raises if it has not been built)."""
+    global _lib_handle
+    if _lib_handle is not None:
+        return _lib_handle
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(
+            f"{_LIB_PATH} is missing: build it with "
+            "`python -m mixture_experts_layer_51_b200.build` (there is no CPU fallback)")
+    L = ctypes.CDLL(_LIB_PATH)
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [ctypes.c_int]
+    L.moe_abi_version.restype = _I32
+    L.moe_capacity.restype = _I32
+    L.moe_capacity.argtypes = [_I32, _I32, _I32, _D]
+    L.moe_max_permuted_rows.restype = _I64
+    L.moe_max_permuted_rows.argtypes = [_I32, _I32, _I32, _D]
+    L.moe_permute_workspace_bytes.restype = _SZ
+    L.moe_permute_workspace_bytes.argtypes = [_I32, _I32]
+    L.moe_workspace_bytes.restype = _SZ
+    L.moe_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, _I32, _D, ctypes.c_int, ctypes.c_int]
+    L.moe_workspace_layout.restype = ctypes.c_int
+    L.moe_workspace_layout.argtypes = [_I32, _I32, _I32, _I32, _I32, _D, ctypes.c_int,
+                                       ctypes.c_int, ctypes.POINTER(moe_ws_layout)]
+    L.moe_route.restype = ctypes.c_int
+    L.moe_route.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, ctypes.c_int, _P, _P, _P, _P]
+    L.moe_permute.restype = ctypes.c_int
+    L.moe_permute.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _D, ctypes.c_int, _P, _I64, _P,
+                              _P, _P, _P, _P, _SZ, _P]
+    L.moe_grouped_ffn.restype = ctypes.c_int
+    L.moe_grouped_ffn.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _I32, _I32, _I32, ctypes.c_int,
+                                  ctypes.c_int, _P, _P, _P, _P]
+    L.moe_unpermute_combine.restype = ctypes.c_int
+    L.moe_unpermute_combine.argtypes = [_P, _P, _P, _I32, _I32, _I32, ctypes.c_int, _P, _P]
+    L.moe_forward.restype = ctypes.c_int
+    L.moe_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _D,
+                              ctypes.c_int, ctypes.c_int, _P, _P, _SZ,
+                              ctypes.POINTER(moe_stats), _P]
+    L.moe_forward_host.restype = ctypes.c_int
+    L.moe_forward_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
+                                   _I32, _D, ctypes.c_int, ctypes.c_int, _P, _SZ, _P]
+    L.moe_set_stage_events.restype = ctypes.c_int
+    L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+    _lib_handle = L
+    return L
+
+
+# ------------------------------------------------------------------ helpers
+def status_string(status):
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}: use bfloat16 or float32")
+
+
+def _act_code(act):
+    if act in ("swiglu", MOE_SWIGLU):
+        return MOE_SWIGLU
+    if act in ("gelu", MOE_GELU):
+        return MOE_GELU
+    raise ValueError(act)
+
+
+def _stream(device, stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cf(capacity_factor):
+    return 0.0 if capacity_factor is None else float(capacity_factor)
+
+
+def moe_capacity(T, E, k, capacity_factor):
+    return lib().moe_capacity(T, E, k, _cf(capacity_factor))
+
+
+def moe_max_permuted_rows(T, E, k, capacity_factor):
+    return lib().moe_max_permuted_rows(T, E, k, _cf(capacity_factor))
+
+
+def moe_permute_workspace_bytes(T, E):
+    return lib().moe_permute_workspace_bytes(T, E)
+
+
+def moe_workspace_bytes(T, d, H, E, k, capacity_factor, dtype, act):
+    code = MOE_BF16 if dtype in (torch.bfloat16, "bf16") else MOE_FP32
+    return lib().moe_workspace_bytes(T, d, H, E, k, _cf(capacity_factor), code, _act_code(act))
+
+
+def moe_workspace_layout(T, d, H, E, k, capacity_factor, dtype, act):
+    code = MOE_BF16 if dtype in (torch.bfloat16, "bf16") else MOE_FP32
+    L = moe_ws_layout()
+    _check(lib().moe_workspace_layout(T, d, H, E, k, _cf(capacity_factor), code, _act_code(act),
+                                      ctypes.byref(L)), "moe_workspace_layout")
+    return L
+
+
+def workspace_views(ws, layout, T, d, H, E, k, dtype):
+    """Tensor views of the intermediates inside a moe_forward workspace."""
+    def view(off, n, dt):
+        nbytes = n * torch.empty((), dtype=dt).element_size()
+        return ws[off:off + nbytes].view(dt)
+    rows = layout.rows
+    return dict(
+        idx=view(layout.idx, T * k, torch.int32).view(T, k),
+        gate=view(layout.gate, T * k, torch.float32).view(T, k),
+        margin=view(layout.margin, T, torch.float32),
+        pos=view(layout.pos, T * k, torch.int32).view(T, k),
+        counts=view(layout.counts, E, torch.int32),
+        kept_counts=view(layout.kept_counts, E, torch.int32),
+        offsets=view(layout.offsets, E + 1, torch.int32),
+        dev_error=view(layout.dev_error, 1, torch.int32),
+        xp=view(layout.xp, rows * d, dtype).view(rows, d),
+        h=view(layout.h, rows * H, dtype).view(rows, H),
+        o=view(layout.o, rows * d, torch.float32).view(rows, d),
+    )
+
+
+# ------------------------------------------------------------- entry points
+def moe_route(x, Wg, bias, k, idx=None, gate=None, margin=None, stream=None):
+    T, d = x.shape
+    E = Wg.shape[1]
+    dev = x.device
+    idx = idx if idx is not None else torch.empty((T, k), dtype=torch.int32, device=dev)
+    gate = gate if gate is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
+    margin = margin if margin is not None else torch.empty((T,), dtype=torch.float32, device=dev)
+    _check(lib().moe_route(_ptr(x), _ptr(Wg), _ptr(bias), T, d, E, k, _dtype_code(x),
+                           _ptr(idx), _ptr(gate), _ptr(margin), _stream(dev, stream)),
+           "moe_route")
+    return idx, gate, margin
+
+
+def moe_permute(x, idx, E, capacity_factor, xp=None, pos=None, counts=None, kept_counts=None,
+                offsets=None, ws=None, stream=None):
+    T, d = x.shape
+    k = idx.shape[1]
+    dev = x.device
+    rows = moe_max_permuted_rows(T, E, k, capacity_factor)
+    xp = xp if xp is not None else torch.empty((max(rows, 0), d), dtype=x.dtype, device=dev)
+    pos = pos if pos is not None else torch.empty((T, k), dtype=torch.int32, device=dev)
+    counts = counts if counts is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    kept_counts = kept_counts if kept_counts is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = offsets if offsets is not None else torch.empty(E + 1, dtype=torch.int32, device=dev)
+    wsb = moe_permute_workspace_bytes(T, E)
+    ws = ws if ws is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
+    _check(lib().moe_permute(_ptr(x), _ptr(idx), T, d, E, k, _cf(capacity_factor),
+                             _dtype_code(x), _ptr(xp), xp.shape[0], _ptr(pos), _ptr(counts),
+                             _ptr(kept_counts), _ptr(offsets), _ptr(ws), ws.numel(),
+                             _stream(dev, stream)), "moe_permute")
+    return dict(xp=xp, pos=pos, counts=counts, kept_counts=kept_counts, offsets=offsets)
+
+
+def moe_grouped_ffn(xp, offsets, kept_counts, W1, W3, W2, act, h=None, o=None, dev_error=None,
+                    stream=None):
+    rows, d = xp.shape
+    E, _, H = W1.shape
+    dev = xp.device
+    h = h if h is not None else torch.empty((rows, H), dtype=xp.dtype, device=dev)
+    o = o if o is not None else torch.empty((rows, d), dtype=torch.float32, device=dev)
+    dev_error = dev_error if dev_error is not None else torch.zeros(1, dtype=torch.int32, device=dev)
+    _check(lib().moe_grouped_ffn(_ptr(xp), rows, _ptr(offsets), _ptr(kept_counts), _ptr(W1),
+                                 _ptr(W3), _ptr(W2), E, d, H, _act_code(act), _dtype_code(xp),
+                                 _ptr(h), _ptr(o), _ptr(dev_error), _stream(dev, stream)),
+           "moe_grouped_ffn")
+    return h, o, dev_error
+
+
+def moe_unpermute_combine(o, pos, gate, dtype, y=None, stream=None):
+    T, k = pos.shape
+    d = o.shape[1]
+    dev = o.device
+    y = y if y is not None else torch.empty((T, d), dtype=dtype, device=dev)
+    _check(lib().moe_unpermute_combine(_ptr(o), _ptr(pos), _ptr(gate), T, d, k,
+                                       _dtype_code(y), _ptr(y), _stream(dev, stream)),
+           "moe_unpermute_combine")
+    return y
+
+
+def moe_forward(x, Wg, bias, W1, W3, W2, k, capacity_factor, act, y=None, ws=None,
+                stats=False, stream=None):
+    """Whole layer.  Returns y, or (y, moe_stats) when stats=True."""
+    T, d = x.shape
+    E, _, H = W1.shape
+    dev = x.device
+    need = moe_workspace_bytes(T, d, H, E, k, capacity_factor, x.dtype, act)
+    ws = ws if ws is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+    y = y if y is not None else torch.empty((T, d), dtype=x.dtype, device=dev)
+    st = moe_stats() if stats else None
+    status = lib().moe_forward(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                               T, d, H, E, k, _cf(capacity_factor), _act_code(act),
+                               _dtype_code(x), _ptr(y), _ptr(ws), ws.numel(),
+                               ctypes.byref(st) if st is not None else None,
+                               _stream(dev, stream))
+    _check(status, "moe_forward")
+    return (y, st) if stats else y
+
+
+def moe_forward_host(x_host, Wg, bias, W1, W3, W2, k, capacity_factor, act, y_host=None,
+                     x_dev=None, y_dev=None, ws=None, stream=None):
+    """The layer on tokens in host memory (pinned for full bandwidth): copy in,
+    forward, copy out, all inside the library call."""
+    T, d = x_host.shape
+    E, _, H = W1.shape
+    dev = W1.device
+    y_host = y_host if y_host is not None else torch.empty((T, d), dtype=x_host.dtype, pin_memory=True)
+    x_dev = x_dev if x_dev is not None else torch.empty((T, d), dtype=x_host.dtype, device=dev)
+    y_dev = y_dev if y_dev is not None else torch.empty((T, d), dtype=x_host.dtype, device=dev)
+    need = moe_workspace_bytes(T, d, H, E, k, capacity_factor, x_host.dtype, act)
+    ws = ws if ws is not None else torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(lib().moe_forward_host(_ptr(x_host), _ptr(y_host), _ptr(x_dev), _ptr(y_dev),
+                                  _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2), T, d, H,
+                                  E, k, _cf(capacity_factor), _act_code(act),
+                                  _dtype_code(x_host), _ptr(ws), ws.numel(),
+                                  _stream(dev, stream)), "moe_forward_host")
+    return y_host
+
+
+def moe_set_stage_events(events):
+    """Record ``events`` (six torch.cuda.Event, created with timing enabled)
+    between the stages of the next forwards on this thread; None stops."""
+    if events is None:
+        _check(lib().moe_set_stage_events(None), "moe_set_stage_events")
+        return
+    arr = (ctypes.c_void_p * MOE_NUM_STAGE_EVENTS)()
+    for i, ev in enumerate(events):
+        arr[i] = ctypes.c_void_p(ev.cuda_event)
+    _check(lib().moe_set_stage_events(arr), "moe_set_stage_events")
+
+
+def stage_times_ms(events):
+    """Per-stage durations (ms) from six recorded events."""
+    return {name: events[i].elapsed_time(events[i + 1]) for i, name in enumerate(STAGES)}
+
+
+class MoELayer:
+    """Weights plus a persistent workspace for repeated forwards on one
+    device (no allocation per call)."""
+
+    def __init__(self, Wg, bias, W1, W3, W2, k, capacity_factor=0.0, act="swiglu",
+                 max_tokens=None):
+        self.Wg, self.bias, self.W1, self.W3, self.W2 = Wg, bias, W1, W3, W2
+        self.k, self.cf, self.act = k, capacity_factor, act
+        self.E, self.d, self.H = W1.shape
+        self.dtype = W1.dtype
+        self.device = W1.device
+        self._ws = None
+        self._ws_T = -1
+        if max_tokens:
+            self.workspace(max_tokens)
+
+    def workspace(self, T):
+        if self._ws is None or self._ws_T != T:
+            need = moe_workspace_bytes(T, self.d, self.H, self.E, self.k, self.cf, self.dtype,
+                                       self.act)
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self._ws_T = T
+        return self._ws
+
+    def layout(self, T):
+        return moe_workspace_layout(T, self.d, self.H, self.E, self.k, self.cf, self.dtype,
+                                    self.act)
+
+    def intermediates(self, T):
+        return workspace_views(self.workspace(T), self.layout(T), T, self.d, self.H, self.E,
+                               self.k, self.dtype)
+
+    def __call__(self, x, y=None, stats=False, stream=None):
+        return moe_forward(x, self.Wg, self.bias, self.W1, self.W3, self.W2, self.k, self.cf,
+                           self.act, y=y, ws=self.workspace(x.shape[0]), stats=stats,
+                           stream=stream)

@@ -1,0 +1,128 @@
+"""Shared parity protocol: run the CUDA path through the C ABI and compare
+every stage with the fp64 oracle.
+
+Routing near a tie can legitimately pick either expert, so each stage is
+checked twice:
+  * end to end -- expert indices must match the oracle's wherever the
+    oracle's margin (k-th minus (k+1)-th logit) exceeds 1e-3;
+  * teacher-forced -- the oracle's capacity/permutation step is fed the GPU's
+    indices (counts, kept counts, offsets, positions and drops must then be
+    bit-exact everywhere), and the oracle's expert FFNs and combine are fed
+    the GPU's selection (y must then meet the tolerance on every token).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_layer_51_b200 import moe as M
+
+NEAR_TIE = 1e-3
+BF16_MAX_ABS = 2e-2
+BF16_REL_FRO = 5e-3
+FP32_REL_FRO = 1e-5
+GATE_ABS = 1e-4
+
+
+def errors(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    diff = got - want
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    nrm = float(np.linalg.norm(want))
+    rel = float(np.linalg.norm(diff)) / nrm if nrm > 0 else float(np.linalg.norm(diff))
+    return max_abs, rel
+
+
+def assert_y_close(got, want, dtype, what="y"):
+    max_abs, rel = errors(got, want)
+    if dtype == "bf16":
+        assert max_abs <= BF16_MAX_ABS and rel <= BF16_REL_FRO, (
+            f"{what}: max_abs={max_abs:.3g} rel_fro={rel:.3g}")
+    else:
+        assert rel <= FP32_REL_FRO, f"{what}: rel_fro={rel:.3g} max_abs={max_abs:.3g}"
+    return max_abs, rel
+
+
+def to_np(t):
+    return t.detach().to("cpu").numpy()
+
+
+def run_gpu(w, inp, device="cuda"):
+    """moe_forward through the ABI; returns y and every intermediate (numpy)."""
+    dev = torch.device(device)
+    t = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
+    layer = M.MoELayer(t["Wg"], t["bias"], t["W1"], t["W3"], t["W2"], w.k, w.cf, w.act)
+    y, st = layer(t["x"], stats=True)
+    torch.cuda.synchronize(dev)
+    views = layer.intermediates(w.T)
+    out = {k: to_np(v) for k, v in views.items() if k in (
+        "idx", "gate", "margin", "pos", "counts", "kept_counts", "offsets", "dev_error")}
+    out["y"] = to_np(y.float())
+    out["stats"] = st
+    out["layer"] = layer
+    out["views"] = views
+    out["dev_inputs"] = t
+    return out
+
+
+def padded_offsets(kept_counts):
+    off = [0]
+    for c in kept_counts:
+        off.append(off[-1] + (int(c) + M.MOE_ROW_ALIGN - 1) // M.MOE_ROW_ALIGN * M.MOE_ROW_ALIGN)
+    return np.array(off)
+
+
+def check_routing(g, logits, k):
+    """Indices vs the oracle away from near-ties; gates vs the oracle's
+    softmax at the GPU's selection; returns the near-tie count."""
+    idx_o, _, margin_o = oracle.top_k(logits, k)
+    far = margin_o > NEAR_TIE
+    assert (g["idx"][far] == idx_o[far]).all(), "routing differs away from a near-tie"
+    gate_tf = oracle.gating_softmax(np.take_along_axis(logits, g["idx"].astype(np.int64), 1))
+    assert np.abs(g["gate"] - gate_tf).max() <= GATE_ABS
+    if k < logits.shape[1]:
+        assert np.abs(g["margin"][far] - margin_o[far]).max() <= 1e-3
+    return int((~far).sum()), idx_o
+
+
+def check_permutation(g, x_np, T, E, k, cf, xp_view=None):
+    """Teacher-forced permutation: bit-exact against the oracle's capacity
+    step run on the GPU's own indices."""
+    C = oracle.capacity(T, E, k, cf)
+    counts, kept_counts, rank, kept = oracle.assign_capacity(g["idx"], E, C)
+    assert (g["counts"] == counts).all()
+    assert (g["kept_counts"] == kept_counts).all()
+    off = padded_offsets(kept_counts)
+    assert (g["offsets"] == off).all()
+    want_pos = np.where(kept, off[g["idx"]] + rank, -1)
+    assert (g["pos"] == want_pos).all()
+    if xp_view is not None and kept.any():
+        tt, jj = np.nonzero(kept)
+        rows = torch.as_tensor(want_pos[tt, jj], device=xp_view.device, dtype=torch.long)
+        got = to_np(xp_view.index_select(0, rows).float())
+        assert np.array_equal(got, x_np[tt].astype(np.float32)), "xp rows are not exact copies"
+    return kept, C
+
+
+def full_parity(w, inp, check_xp=True):
+    """Whole-batch parity for sizes the oracle runs in seconds."""
+    g = run_gpu(w, inp)
+    assert int(g["dev_error"][0]) == 0
+    x_np = to_np(inp["x"].float())
+    logits = oracle.router_logits(inp["x"], inp["Wg"], inp["bias"])
+    near, idx_o = check_routing(g, logits, w.k)
+    kept, C = check_permutation(g, x_np, w.T, w.E, w.k, w.cf,
+                                g["views"]["xp"] if check_xp else None)
+    y_tf, _ = oracle.moe_forward_tokens(inp["x"], logits, g["idx"], kept, inp["W1"], inp["W3"],
+                                        inp["W2"], w.act)
+    errs = assert_y_close(g["y"], y_tf, w.dtype)
+    if near == 0 or (g["idx"] == idx_o).all():
+        ref = oracle.moe_forward(inp["x"], inp["Wg"], inp["bias"], inp["W1"], inp["W3"],
+                                 inp["W2"], w.k, w.cf, w.act)
+        assert (g["idx"] == ref["idx"]).all()
+        assert (g["kept_counts"] == ref["kept_counts"]).all()
+        assert_y_close(g["y"], ref["y"], w.dtype, "y (end to end)")
+    return g, dict(near_ties=near, max_abs=errs[0], rel_fro=errs[1])

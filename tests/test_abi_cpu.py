@@ -1,0 +1,135 @@
+"""CPU checks of the C ABI: libmoe.so loads without a GPU, exports every
+function include/moe.h declares, and its host-side logic (capacity, buffer
+sizes, argument validation) behaves as documented.  No kernel is launched."""
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_51_b200 import moe as M
+from mixture_experts_layer_51_b200.workloads import WORKLOADS
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(M._LIB_PATH):
+        from mixture_experts_layer_51_b200 import build
+        build.build()
+    return M.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(M.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.moe_abi_version() == 1
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert M.status_string(s).startswith("MOE_")
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_capacity_matches_oracle(lib, name):
+    w = WORKLOADS[name]
+    c = M.moe_capacity(w.T, w.E, w.k, w.cf)
+    o = oracle.capacity(w.T, w.E, w.k, w.cf)
+    assert c == (-1 if o is None else o)
+
+
+def test_capacity_edge_values(lib):
+    assert M.moe_capacity(100, 4, 2, 0.0) == -1
+    assert M.moe_capacity(100, 4, 2, -2.0) == -1
+    assert M.moe_capacity(100, 4, 2, math.inf) == -1
+    assert M.moe_capacity(100, 4, 2, math.nan) == -1
+    assert M.moe_capacity(10, 4, 1, 1.0) == 3
+    assert M.moe_capacity(0, 4, 1, 1.0) == 0
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(256, 4, 1, 1.25), (4096, 8, 2, 0.0), (16384, 32, 2, 1.0),
+                                       (16384, 64, 8, 0.0), (1, 1, 1, 0.0), (33, 7, 3, 0.5),
+                                       (1000, 64, 1, 0.0)])
+def test_max_permuted_rows_bounds_every_routing(lib, T, E, k, cf):
+    """sum_e roundup(kept_e, 128) <= moe_max_permuted_rows for random,
+    one-hot-skewed and spread-thin routings (kept counts from the oracle)."""
+    import numpy as np
+    rng = np.random.default_rng(T * 31 + E)
+    rows = M.moe_max_permuted_rows(T, E, k, cf)
+    assert rows % 128 == 0
+    C = oracle.capacity(T, E, k, cf)
+    routings = []
+    for _ in range(5):
+        routings.append(np.argsort(rng.standard_normal((T, E)), axis=1)[:, :k])
+    skew = np.tile(np.arange(k), (T, 1))                 # everyone on experts 0..k-1
+    routings.append(skew)
+    thin = (np.arange(T)[:, None] * k + np.arange(k)[None, :]) % E   # round robin
+    routings.append(thin)
+    for idx in routings:
+        _, kept_counts, _, _ = oracle.assign_capacity(idx, E, C)
+        need = int(sum(-(-int(c) // 128) * 128 for c in kept_counts))
+        assert need <= rows
+
+
+def test_workspace_layout_is_consistent(lib):
+    L = M.moe_workspace_layout(8192, 4096, 14336, 8, 2, 0.0, "bf16", "swiglu")
+    offs = [L.idx, L.gate, L.margin, L.pos, L.counts, L.kept_counts, L.offsets, L.dev_error,
+            L.scratch, L.xp, L.h, L.o]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert L.rows == M.moe_max_permuted_rows(8192, 8, 2, 0.0)
+    assert L.total >= L.o + L.rows * 4096 * 4
+    assert M.moe_workspace_bytes(8192, 4096, 14336, 8, 2, 0.0, "bf16", "swiglu") == L.total
+
+
+def test_invalid_arguments_are_rejected_before_any_cuda_call(lib):
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: validation fails first
+    # k > E
+    assert lib.moe_route(fake, fake, None, 16, 64, 2, 3, M.MOE_BF16, fake, fake, None, None) == M.MOE_ERR_ARG
+    # E > 64
+    assert lib.moe_route(fake, fake, None, 16, 64, 65, 2, M.MOE_BF16, fake, fake, None, None) == M.MOE_ERR_ARG
+    # d % 8 != 0
+    assert lib.moe_route(fake, fake, None, 16, 60, 8, 2, M.MOE_BF16, fake, fake, None, None) == M.MOE_ERR_ARG
+    # null output
+    assert lib.moe_route(fake, fake, None, 16, 64, 8, 2, M.MOE_BF16, None, fake, None, None) == M.MOE_ERR_ARG
+    # misaligned x
+    assert lib.moe_route(P(0x10004), fake, None, 16, 64, 8, 2, M.MOE_BF16, fake, fake, None, None) == M.MOE_ERR_ARG
+    # bad dtype enum
+    assert lib.moe_route(fake, fake, None, 16, 64, 8, 2, 7, fake, fake, None, None) == M.MOE_ERR_ARG
+    # permute buffer too small
+    assert lib.moe_permute(fake, fake, 64, 64, 8, 2, 0.0, M.MOE_BF16, fake, 128, fake, fake, fake,
+                           fake, fake, 1 << 20, None) == M.MOE_ERR_ARG
+    # grouped FFN: rows not a multiple of 128, missing W3 for SwiGLU
+    assert lib.moe_grouped_ffn(fake, 100, fake, fake, fake, fake, fake, 8, 64, 64, M.MOE_SWIGLU,
+                               M.MOE_BF16, fake, fake, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_grouped_ffn(fake, 128, fake, fake, fake, None, fake, 8, 64, 64, M.MOE_SWIGLU,
+                               M.MOE_BF16, fake, fake, fake, None) == M.MOE_ERR_ARG
+    # forward: workspace too small
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, 64, 64, 64, 8, 2, 0.0, M.MOE_SWIGLU,
+                         M.MOE_BF16, fake, fake, 16, None, None)
+    assert st == M.MOE_ERR_ARG
+
+
+def test_empty_batch_is_a_no_op(lib):
+    # T == 0 does nothing and touches no device state.
+    st = M.moe_stats()
+    assert lib.moe_forward(None, None, None, None, None, None, 0, 64, 64, 8, 2, 1.0,
+                           M.MOE_SWIGLU, M.MOE_BF16, None, None, 0, ctypes.byref(st), None) == M.MOE_OK
+    assert st.capacity == 0 and st.kept == 0
+    assert lib.moe_route(None, None, None, 0, 64, 8, 2, M.MOE_BF16, None, None, None, None) == M.MOE_OK

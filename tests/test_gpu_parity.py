@@ -1,0 +1,202 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small runs cover every stage on whole batches that still span several tiles
+and ragged tails; the full-size runs use the layer shapes and the launch
+configuration the benchmark times, checking every token's routing and
+permutation and a sample of tokens' outputs.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_51_b200 import moe as M
+from mixture_experts_layer_51_b200.workloads import WORKLOADS, Workload, make_inputs
+
+from parity import (assert_y_close, check_permutation, check_routing, full_parity, run_gpu,
+                    to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # the five layer families at sizes the oracle runs in a second or two
+    "switch_tiny_fp32": WORKLOADS["switch_tiny_fp32"],
+    "top2_bf16": WORKLOADS["top2_bf16"].replace(T=600, d=256, H=384),
+    "mixtral_bf16": WORKLOADS["mixtral_bf16"].replace(T=520, d=512, H=640),
+    "openmoe_skew_bf16": WORKLOADS["openmoe_skew_bf16"].replace(T=1100, d=256, H=512, seq_len=275),
+    "finegrained_bf16": WORKLOADS["finegrained_bf16"].replace(T=700, d=256, H=384),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_layer_parity(name):
+    w = SMALL[name]
+    inp = make_inputs(w, "cpu")
+    g, info = full_parity(w, inp)
+    print(name, info)
+
+
+def test_full_switch_tiny_fp32():
+    # The fp32 workload is small enough to check whole at its full size.
+    w = WORKLOADS["switch_tiny_fp32"]
+    g, info = full_parity(w, make_inputs(w, "cpu"))
+    assert g["stats"].capacity == 80
+
+
+@pytest.mark.parametrize("case", [
+    dict(T=1, d=64, E=4, k=2, H=128),            # single token
+    dict(T=33, d=128, E=8, k=2, H=256),          # ragged vs the 32-token chunk
+    dict(T=300, d=136, E=6, k=3, H=200),         # E not a multiple of 8, d/H tails
+    dict(T=257, d=64, E=1, k=1, H=128),          # one expert: dense FFN
+    dict(T=129, d=64, E=4, k=4, H=128),          # k == E
+    dict(T=400, d=192, E=3, k=1, H=72, act="gelu"),  # bf16 GELU, odd sizes
+    dict(T=2000, d=128, E=16, k=2, H=256, cf=0.25),  # heavy dropping
+    dict(T=513, d=64, E=64, k=8, H=64),          # many tiny experts
+])
+def test_edge_shapes(case):
+    act = case.pop("act", "swiglu")
+    cf = case.pop("cf", 0.0)
+    w = Workload("edge", act=act, dtype="bf16", cf=cf, seed=11, **case)
+    full_parity(w, make_inputs(w, "cpu"))
+
+
+def test_all_tokens_on_one_expert_with_capacity():
+    w = Workload("skew", T=700, d=128, E=8, k=2, H=256, act="swiglu", dtype="bf16", cf=1.0,
+                 seed=5)
+    inp = make_inputs(w, "cpu")
+    inp["bias"] = torch.tensor([40.0, 30.0] + [0.0] * 6)  # experts 0 and 1 win everywhere
+    g, _ = full_parity(w, inp)
+    C = oracle.capacity(w.T, w.E, w.k, w.cf)
+    assert g["counts"][0] == w.T and g["kept_counts"][0] == C
+    # drops are exactly the latest tokens
+    assert (g["pos"][:C, 0] >= 0).all() and (g["pos"][C:, 0] == -1).all()
+
+
+def test_upcycling_identity_on_gpu():
+    """Identical experts: the layer equals the dense FFN (within bf16)."""
+    w = Workload("upcycle", T=300, d=128, E=8, k=2, H=256, act="swiglu", dtype="bf16", cf=0.0,
+                 seed=6)
+    inp = make_inputs(w, "cpu")
+    for key in ("W1", "W3", "W2"):
+        inp[key] = inp[key][:1].expand_as(inp[key]).contiguous()
+    g = run_gpu(w, inp)
+    dense = oracle.expert_ffn(inp["x"], inp["W1"][0], inp["W3"][0], inp["W2"][0], "swiglu")
+    assert_y_close(g["y"], dense, "bf16", "upcycled layer vs dense FFN")
+
+
+def test_deterministic_bitwise():
+    w = SMALL["finegrained_bf16"]
+    inp = make_inputs(w, "cpu")
+    a = run_gpu(w, inp)
+    b = run_gpu(w, inp)
+    assert np.array_equal(a["y"], b["y"])
+    assert np.array_equal(a["pos"], b["pos"])
+
+
+def test_forward_host_matches_device_forward():
+    w = SMALL["top2_bf16"]
+    inp = make_inputs(w, "cpu")
+    g = run_gpu(w, inp)
+    t = g["dev_inputs"]
+    y_host = M.moe_forward_host(inp["x"].pin_memory(), t["Wg"], t["bias"], t["W1"], t["W3"],
+                                t["W2"], w.k, w.cf, w.act)
+    assert np.array_equal(y_host.float().numpy(), g["y"])
+
+
+def test_stage_entry_points_match_forward():
+    """moe_route -> moe_permute -> moe_grouped_ffn -> moe_unpermute_combine
+    called one by one give the same bits as moe_forward."""
+    w = SMALL["openmoe_skew_bf16"]
+    inp = make_inputs(w, "cpu")
+    g = run_gpu(w, inp)
+    t = g["dev_inputs"]
+    idx, gate, margin = M.moe_route(t["x"], t["Wg"], t["bias"], w.k)
+    p = M.moe_permute(t["x"], idx, w.E, w.cf)
+    h, o, err = M.moe_grouped_ffn(p["xp"], p["offsets"], p["kept_counts"], t["W1"], t["W3"],
+                                  t["W2"], w.act)
+    y = M.moe_unpermute_combine(o, p["pos"], gate, t["x"].dtype)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(to_np(idx), g["idx"])
+    assert np.array_equal(to_np(p["pos"]), g["pos"])
+    assert np.array_equal(to_np(y.float()), g["y"])
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_grouped_ffn_against_oracle(act):
+    """The tcgen05 grouped GEMM alone, on hand-made expert blocks (sizes that
+    are not tile multiples, an empty expert, a one-row expert)."""
+    torch.manual_seed(0)
+    E, d, H = 5, 320, 392
+    kept = [130, 0, 257, 1, 128]
+    off = [0]
+    for c in kept:
+        off.append(off[-1] + (c + 127) // 128 * 128)
+    rows = off[-1]
+    xp = torch.randn(rows, d).bfloat16()
+    W1 = (torch.randn(E, d, H) / d ** 0.5).bfloat16()
+    W3 = (torch.randn(E, d, H) / d ** 0.5).bfloat16() if act == "swiglu" else None
+    W2 = (torch.randn(E, H, d) / H ** 0.5).bfloat16()
+    dev = torch.device("cuda")
+    offs = torch.tensor(off, dtype=torch.int32, device=dev)
+    kc = torch.tensor(kept, dtype=torch.int32, device=dev)
+    h, o, err = M.moe_grouped_ffn(xp.to(dev), offs, kc, W1.to(dev),
+                                  None if W3 is None else W3.to(dev), W2.to(dev), act)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    h = to_np(h.float())
+    o = to_np(o)
+    for e in range(E):
+        r = slice(off[e], off[e] + kept[e])
+        if kept[e] == 0:
+            continue
+        xr = xp[r]
+        if act == "swiglu":
+            h_ref = oracle.silu(xr.double().numpy() @ W1[e].double().numpy()) * (
+                xr.double().numpy() @ W3[e].double().numpy())
+        else:
+            h_ref = oracle.gelu(xr.double().numpy() @ W1[e].double().numpy())
+        # h is rounded to bf16 once: relative error <= 2^-8 per element.
+        assert np.all(np.abs(h[r] - h_ref) <= 2.0 ** -8 * np.abs(h_ref) + 1e-6), f"h expert {e}"
+        # o given the GPU's own h: only fp32 accumulation differs.
+        o_ref = h[r].astype(np.float64) @ W2[e].double().numpy()
+        _, rel = assert_y_close(o[r], o_ref, "fp32", f"o expert {e}")
+
+
+# ------------------------------------------------------ full-size layers
+FULL = ["top2_bf16", "mixtral_bf16", "openmoe_skew_bf16", "finegrained_bf16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_layer(name):
+    """The benchmark's shapes and launch configuration: every token's routing
+    (away from near-ties) and the whole permutation bit-exact; sampled
+    tokens' outputs against the oracle."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, "cuda")
+    g = run_gpu(w, inp)
+    assert int(g["dev_error"][0]) == 0
+    cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    logits = oracle.router_logits(cpu["x"], cpu["Wg"], cpu["bias"])
+    near, _ = check_routing(g, logits, w.k)
+    kept, C = check_permutation(g, None, w.T, w.E, w.k, w.cf)
+    rng = np.random.default_rng(w.seed)
+    sample = np.unique(np.concatenate([[0, w.T - 1], rng.choice(w.T, 96, replace=False)]))
+    experts = np.unique(g["idx"][sample])
+    W1 = {int(e): cpu["W1"][int(e)] for e in experts}
+    W3 = None if cpu["W3"] is None else {int(e): cpu["W3"][int(e)] for e in experts}
+    W2 = {int(e): cpu["W2"][int(e)] for e in experts}
+    y_ref, _ = oracle.moe_forward_tokens(cpu["x"][sample], logits[sample], g["idx"][sample],
+                                         kept[sample], W1, W3, W2, w.act)
+    max_abs, rel = assert_y_close(g["y"][sample], y_ref, w.dtype)
+    dropped = int((~kept).sum())
+    print(f"{name}: near_ties={near} dropped={dropped} max_abs={max_abs:.3g} rel_fro={rel:.3g}")
+    if w.cf > 0:
+        # Drop-towards-the-End, reported by position inside each sequence.
+        L = w.seq_len or w.T
+        for label, p, span in (("batch position", np.arange(w.T), w.T),
+                               ("position in sequence", np.arange(w.T) % L, L)):
+            rate = [float((~kept[(p >= a) & (p < a + span // 8)]).mean())
+                    for a in range(0, span, span // 8)]
+            print(f"drop rate by {label} octile:", [round(r, 4) for r in rate])
