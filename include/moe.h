@@ -160,6 +160,30 @@ moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d,
                        int32_t* kept_counts, int32_t* offsets,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* moe_permute without a caller-provided scratch buffer.  The pages have no
+ * counterpart to this entry point: it exists for callers that cannot
+ * allocate device memory where they run the layer -- for example a serving
+ * runtime that reserves all device memory for its own pool up front, or a
+ * plugin that its host framework forbids from allocating inside its execute
+ * call.  Arguments and results are those of moe_permute, minus ws/ws_bytes.
+ *   Scratch: a fixed array of MOE_PERMUTE_STATIC_MAX_INTS int32 (1 MiB) plus
+ *   256 bytes, held by every GPU that loads the library until the process
+ *   exits.  A call with ceil(T / 256) * E > MOE_PERMUTE_STATIC_MAX_INTS
+ *   (at E = 64: T > 1,048,576) returns MOE_ERR_ARG and enqueues nothing.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   The first call on a device looks up the array's device address with
+ *   that device current; make that first call before any stream capture.
+ *   Every call uses the same array, which keeps the last call's contents
+ *   (each call clears the counter that must start at zero, on its stream):
+ *   calls whose work overlaps on the GPU -- different streams, or different
+ *   host threads on one device -- race on it, so the caller must serialise
+ *   them. */
+#define MOE_PERMUTE_STATIC_MAX_INTS (1 << 18)
+moe_status moe_permute_static(const void* x, const int32_t* idx, int32_t T, int32_t d,
+                              int32_t E, int32_t k, double capacity_factor, moe_dtype dtype,
+                              void* xp, int64_t xp_rows, int32_t* pos, int32_t* counts,
+                              int32_t* kept_counts, int32_t* offsets, void* stream);
+
 /* Grouped expert FFN over the per-expert blocks ("[Paper Club] Upcycling
  * ...": one grouped GEMM over any number of experts and tokens instead of a
  * loop over experts; Mixtral's SwiGLU expert in "The Math Behind MoEs").

@@ -27,8 +27,9 @@ EXPORTED = (
     "moe_status_string", "moe_abi_version", "moe_capacity", "moe_max_permuted_rows",
     "moe_permute_workspace_bytes", "moe_workspace_bytes", "moe_workspace_layout",
     "moe_route", "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine",
-    "moe_forward", "moe_forward_host", "moe_set_stage_events",
+    "moe_forward", "moe_forward_host", "moe_set_stage_events", "moe_permute_static",
 )
+MOE_PERMUTE_STATIC_MAX_INTS = 1 << 18
 MOE_NUM_STAGE_EVENTS = 6
 STAGES = ("route", "permute", "ffn_up", "ffn_down", "combine")
 
@@ -105,6 +106,9 @@ def lib():
     L.moe_forward_host.restype = ctypes.c_int
     L.moe_forward_host.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                    _I32, _D, ctypes.c_int, ctypes.c_int, _P, _SZ, _P]
+    L.moe_permute_static.restype = ctypes.c_int
+    L.moe_permute_static.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _D, ctypes.c_int, _P, _I64,
+                                     _P, _P, _P, _P, _P]
     L.moe_set_stage_events.restype = ctypes.c_int
     L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
     _lib_handle = L
@@ -227,6 +231,26 @@ def moe_permute(x, idx, E, capacity_factor, xp=None, pos=None, counts=None, kept
                              _dtype_code(x), _ptr(xp), xp.shape[0], _ptr(pos), _ptr(counts),
                              _ptr(kept_counts), _ptr(offsets), _ptr(ws), ws.numel(),
                              _stream(dev, stream)), "moe_permute")
+    return dict(xp=xp, pos=pos, counts=counts, kept_counts=kept_counts, offsets=offsets)
+
+
+def moe_permute_static(x, idx, E, capacity_factor, xp=None, pos=None, counts=None,
+                       kept_counts=None, offsets=None, stream=None):
+    """moe_permute using the library's own fixed scratch (no allocation by the
+    library; outputs allocated here when not given)."""
+    T, d = x.shape
+    k = idx.shape[1]
+    dev = x.device
+    rows = moe_max_permuted_rows(T, E, k, capacity_factor)
+    xp = xp if xp is not None else torch.empty((max(rows, 0), d), dtype=x.dtype, device=dev)
+    pos = pos if pos is not None else torch.empty((T, k), dtype=torch.int32, device=dev)
+    counts = counts if counts is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    kept_counts = kept_counts if kept_counts is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = offsets if offsets is not None else torch.empty(E + 1, dtype=torch.int32, device=dev)
+    _check(lib().moe_permute_static(_ptr(x), _ptr(idx), T, d, E, k, _cf(capacity_factor),
+                                    _dtype_code(x), _ptr(xp), xp.shape[0], _ptr(pos),
+                                    _ptr(counts), _ptr(kept_counts), _ptr(offsets),
+                                    _stream(dev, stream)), "moe_permute_static")
     return dict(xp=xp, pos=pos, counts=counts, kept_counts=kept_counts, offsets=offsets)
 
 
