@@ -40,6 +40,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <stdlib.h>
+
 #include <algorithm>
 #include <mutex>
 
@@ -48,18 +50,25 @@
 namespace moe {
 namespace {
 
-constexpr int TM = 128;  // tile rows (UMMA M)
+constexpr int TM = 128;  // tile rows held by one CTA (UMMA M per CTA)
 constexpr int TN = 256;  // accumulator columns (UMMA N)
 constexpr int TK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = TM * TK * 2;    // 16 KB
-constexpr int B_BYTES = TN * TK * 2;    // 32 KB
+constexpr int A_BYTES = TM * TK * 2;      // 16 KB
 constexpr int B_BOX_BYTES = 64 * TK * 2;  // one 64-column x 64-row box: 8 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * TN;
 constexpr int CONTROL_BYTES = 2048;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CONTROL_BYTES + 1024;  // + alignment slack
+// One CTA per tile (CG = 1): each CTA holds all 256 B columns.  A CTA pair
+// (CG = 2): each CTA holds half of them, so a stage is 32 KB and the ring
+// gets 6 stages in the same shared memory.
+template <int CG>
+struct Cfg {
+  static constexpr int B_BOXES = 4 / CG;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BOXES * B_BOX_BYTES;
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CONTROL_BYTES + 1024;
+};
+constexpr int MAX_STAGES = 6;
 
 enum Epi { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_PLAIN_F32 = 2 };
 
@@ -77,8 +86,8 @@ struct TcParams {
 };
 
 struct Control {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -109,16 +118,31 @@ __device__ __forceinline__ float gelu_f(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
 }
 
-template <int EPI>
+// CG = 1: one CTA computes a 128 x 256 tile.  CG = 2: a cluster of two CTAs
+// computes a 256 x 256 tile with tcgen05 pair MMAs issued by the leader
+// (rank 0): each CTA loads its own 128 rows of A and its half of the 256
+// B columns; the pair MMA reads both CTAs' shared memory and writes each
+// CTA's 128 accumulator rows into that CTA's tensor memory.  Stage-full and
+// accumulator-empty barriers live in the leader; stage-empty and
+// accumulator-full barriers in each CTA (the leader's commits reach both).
+template <int EPI, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                   const __grid_constant__ CUtensorMap tmB1, const TcParams p) {
+  using C_ = Cfg<CG>;
+  constexpr int STAGES = C_::STAGES;
+  constexpr int STAGE_BYTES = C_::STAGE_BYTES;
+  constexpr int TILE_M = TM * CG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   Control& c = *reinterpret_cast<Control*>(smem + STAGES * STAGE_BYTES);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int group = blockIdx.x / CG;   // tile-processing unit (CTA or CTA pair)
+  const int ngroups = gridDim.x / CG;
 
   // ------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -128,7 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&c.tfull[a]), 1);
-      mbar_init(smem_u32(&c.tempty[a]), 4);  // one arrive per epilogue warp
+      mbar_init(smem_u32(&c.tempty[a]), 4 * CG);  // one arrive per epilogue warp of the group
     }
     mbar_init(smem_u32(&c.drain), 1);
     c.abort_flag = 0;
@@ -145,21 +169,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&c.tmem_base), TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(smem_u32(&c.tmem_base), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&c.tmem_base), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   __syncthreads();
   if (tid == 0) {
     // Schedule: experts with more m-blocks first (stable), empty ones skipped.
     int n = 0;
     for (int e = 0; e < p.E; ++e) {
-      const int mt = (c.kept[e] + TM - 1) / TM;
+      const int mt = (c.kept[e] + TILE_M - 1) / TILE_M;
       if (mt <= 0) continue;
-      // An expert block must start on a tile boundary and end inside the
-      // buffers; anything else is reported and skipped, never written.
+      // An expert block must start on a 128-row boundary and its kept rows
+      // must end inside the buffers; anything else is reported and skipped,
+      // never written.  (Rows a pair tile reads past the block are padding
+      // or the next block -- or past the buffer, where TMA reads zeros -- and
+      // are never stored.)
       if (c.off[e] < 0 || (c.off[e] % TM) != 0 ||
-          static_cast<int64_t>(c.off[e]) + static_cast<int64_t>(mt) * TM > p.rows) {
-        atomicOr(p.err, kErrRowOverflow);
+          static_cast<int64_t>(c.off[e]) + ((c.kept[e] + TM - 1) / TM) * TM > p.rows) {
+        if (leader) atomicOr(p.err, kErrRowOverflow);
         continue;
       }
       int q = n;
@@ -183,6 +215,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
   const int total = c.total_tiles;
@@ -197,13 +230,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
       bool ok = true, timed_out = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = group; t < total && ok; t += ngroups) {
         int e, m, n;
         decode_tile(c, t, e, m, n);
-        const int row0 = c.off[e] + m * TM;
+        const int row0 = c.off[e] + m * TILE_M + static_cast<int>(rank) * TM;
         for (int kb = 0; kb < nk; ++kb) {
-          const uint32_t empty_bar = smem_u32(&c.empty[stage]);
-          if (!mbar_wait(empty_bar, phase ^ 1)) {
+          if (!mbar_wait(smem_u32(&c.empty[stage]), phase ^ 1)) {
             ok = false;
             timed_out = true;
             break;
@@ -212,22 +244,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          const uint32_t full_bar = smem_u32(&c.full[stage]);
+          const uint32_t full_local = smem_u32(&c.full[stage]);
           const uint32_t a_dst = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t b_dst = a_dst + A_BYTES;
-          mbar_arrive_expect_tx(full_bar, STAGE_BYTES);
-          tma_load_2d(a_dst, &tmA, full_bar, kb * TK, row0);
-          if (EPI == EPI_SWIGLU) {
-            const int n0 = n * (TN / 2);
-            tma_load_3d(b_dst + 0 * B_BOX_BYTES, &tmB0, full_bar, n0, kb * TK, e);
-            tma_load_3d(b_dst + 1 * B_BOX_BYTES, &tmB0, full_bar, n0 + 64, kb * TK, e);
-            tma_load_3d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_bar, n0, kb * TK, e);
-            tma_load_3d(b_dst + 3 * B_BOX_BYTES, &tmB1, full_bar, n0 + 64, kb * TK, e);
-          } else {
-            const int n0 = n * TN;
+          if (CG == 1) {
+            mbar_arrive_expect_tx(full_local, STAGE_BYTES);
+            tma_load_2d(a_dst, &tmA, full_local, kb * TK, row0);
+            if (EPI == EPI_SWIGLU) {
+              const int n0 = n * (TN / 2);
+              tma_load_3d(b_dst + 0 * B_BOX_BYTES, &tmB0, full_local, n0, kb * TK, e);
+              tma_load_3d(b_dst + 1 * B_BOX_BYTES, &tmB0, full_local, n0 + 64, kb * TK, e);
+              tma_load_3d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_local, n0, kb * TK, e);
+              tma_load_3d(b_dst + 3 * B_BOX_BYTES, &tmB1, full_local, n0 + 64, kb * TK, e);
+            } else {
+              const int n0 = n * TN;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tma_load_3d(b_dst + q * B_BOX_BYTES, &tmB0, full_bar, n0 + 64 * q, kb * TK, e);
+              for (int q = 0; q < 4; ++q)
+                tma_load_3d(b_dst + q * B_BOX_BYTES, &tmB0, full_local, n0 + 64 * q, kb * TK, e);
+            }
+          } else {
+            // Both CTAs' bytes complete on the leader's full barrier, which
+            // the leader arms for the whole pair.
+            const uint32_t full_leader = mapa_shared(full_local, 0);
+            if (leader) mbar_arrive_expect_tx(full_local, CG * STAGE_BYTES);
+            tma_load_2d_pair(a_dst, &tmA, full_leader, kb * TK, row0);
+            if (EPI == EPI_SWIGLU) {
+              // leader: W1 columns (gate half); peer: W3 columns (up half)
+              const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
+              const int n0 = n * (TN / 2);
+              tma_load_3d_pair(b_dst, mb, full_leader, n0, kb * TK, e);
+              tma_load_3d_pair(b_dst + B_BOX_BYTES, mb, full_leader, n0 + 64, kb * TK, e);
+            } else {
+              const int n0 = n * TN + static_cast<int>(rank) * (TN / 2);
+              tma_load_3d_pair(b_dst, &tmB0, full_leader, n0, kb * TK, e);
+              tma_load_3d_pair(b_dst + B_BOX_BYTES, &tmB0, full_leader, n0 + 64, kb * TK, e);
+            }
           }
 #pragma unroll
           for (int s = 0; s < STAGES; ++s)
@@ -239,7 +290,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (ok) {
-        // Tail: wait until the MMA warp has released every stage, so no
+        // Tail: wait until the MMA has released every stage, so no
         // tcgen05.commit arrival is still in flight when the CTA exits.
         for (int i = 0; i < STAGES; ++i) {
           if (!mbar_wait(smem_u32(&c.empty[stage]), phase ^ 1)) {
@@ -256,23 +307,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (timed_out) atomicOr(p.err, kErrTimeoutProducer);
         c.abort_flag = 1;
         // Let every issued copy land before the shared memory goes away.
-        for (int s = 0; s < STAGES; ++s) {
-          if (issued[s] > 0 &&
-              !mbar_wait(smem_u32(&c.full[s]), static_cast<uint32_t>(issued[s] - 1) & 1u))
-            atomicOr(p.err, kErrTimeoutDrain);
+        if (CG == 1 || leader) {
+          for (int s = 0; s < STAGES; ++s) {
+            if (issued[s] > 0 &&
+                !mbar_wait(smem_u32(&c.full[s]), static_cast<uint32_t>(issued[s] - 1) & 1u))
+              atomicOr(p.err, kErrTimeoutDrain);
+          }
+        } else {
+          // The peer's copies complete on the leader's barrier, which this
+          // CTA cannot poll; give them time to land.
+          for (int i = 0; i < 100; ++i) __nanosleep(1000);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(TM, TN, false, true);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TILE_M, TN, false, true);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true, timed_out = false, issued_any = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = group; t < total && ok; t += ngroups) {
         if (!mbar_wait(smem_u32(&c.tempty[acc]), acc_phase ^ 1)) {
           ok = false;
           timed_out = true;
@@ -299,17 +356,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
             // B: N-major, 64-column boxes 8 KB apart; advance 16 K-rows (2 KB).
             const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, B_BOX_BYTES, 1024);
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if (CG == 2)
+              tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else
+              tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           issued_any = true;
-          tc_commit(smem_u32(&c.empty[stage]));
+          const uint32_t empty_local = smem_u32(&c.empty[stage]);
+          if (CG == 2) {
+            tc_commit_pair(empty_local);
+            tc_commit_pair(mapa_shared(empty_local, 1));
+          } else {
+            tc_commit(empty_local);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit(smem_u32(&c.tfull[acc]));
+        const uint32_t tfull_local = smem_u32(&c.tfull[acc]);
+        if (CG == 2) {
+          tc_commit_pair(tfull_local);
+          tc_commit_pair(mapa_shared(tfull_local, 1));
+        } else {
+          tc_commit(tfull_local);
+        }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
@@ -318,7 +390,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         c.abort_flag = 1;
         if (issued_any) {
           // Wait for the MMAs already issued before TMEM is freed.
-          tc_commit(smem_u32(&c.drain));
+          if (CG == 2)
+            tc_commit_pair(smem_u32(&c.drain));
+          else
+            tc_commit(smem_u32(&c.drain));
           if (!mbar_wait(smem_u32(&c.drain), 0)) atomicOr(p.err, kErrTimeoutDrain);
         }
       }
@@ -329,7 +404,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = quad * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (int t = group; t < total; t += ngroups) {
       int e, m, n;
       decode_tile(c, t, e, m, n);
       if (!mbar_wait(smem_u32(&c.tfull[acc]), acc_phase)) {
@@ -341,8 +416,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * TN);
-      const bool row_ok = row < c.kept[e] - m * TM;
-      const int64_t grow = static_cast<int64_t>(c.off[e]) + m * TM + row;
+      const int row_in_expert = m * TILE_M + static_cast<int>(rank) * TM + row;
+      const bool row_ok = row_in_expert < c.kept[e];
+      const int64_t grow = static_cast<int64_t>(c.off[e]) + row_in_expert;
       if (EPI == EPI_SWIGLU) {
         const int n0 = n * (TN / 2);
         __nv_bfloat16* dst_row = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out;
@@ -415,7 +491,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&c.tempty[acc]));
+      if (lane == 0) {
+        if (CG == 2)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&c.tempty[acc]), 0));
+        else
+          mbar_arrive(smem_u32(&c.tempty[acc]));
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -424,10 +505,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // ---------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // no CTA leaves while its pair may still touch its memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if (CG == 2)
+      tmem_dealloc_pair(tmem, TMEM_COLS);
+    else
+      tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -472,14 +557,47 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, int CG>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                       const TcParams& p, int grid, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                       const TcParams& p, int groups, cudaStream_t s) {
+  constexpr int smem = Cfg<CG>::SMEM_BYTES;
+  cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI, CG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  ffn_tc_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(a, b0, b1, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(groups * CG, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<EPI, CG>, a, b0, b1, p);
+}
+
+// CTA pairs by default; MOE_TC_CTA_PAIR=0 selects one CTA per tile.
+bool use_cta_pairs() {
+  static const bool pairs = [] {
+    const char* v = getenv("MOE_TC_CTA_PAIR");
+    return !(v && v[0] == '0');
+  }();
+  return pairs;
+}
+
+template <int EPI>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const TcParams& p, int num_sms, int64_t tiles_max, cudaStream_t s) {
+  if (use_cta_pairs()) {
+    const int groups = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>(num_sms / 2, (tiles_max + 1) / 2)));
+    return launch_one<EPI, 2>(a, b0, b1, p, groups, s);
+  }
+  const int groups = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms, tiles_max)));
+  return launch_one<EPI, 1>(a, b0, b1, p, groups, s);
 }
 
 }  // namespace
@@ -505,9 +623,9 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.offsets = a.offsets;
   up.kept = a.kept_counts;
   up.err = a.dev_error;
-  int grid = static_cast<int>(std::min<int64_t>(num_sms, mtiles_max * up.n_tiles));
-  cudaError_t err = swiglu ? launch_one<EPI_SWIGLU>(mx, mw1, mw3, up, grid, s)
-                           : launch_one<EPI_GELU>(mx, mw1, mw1, up, grid, s);
+  cudaError_t err =
+      swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, up, num_sms, mtiles_max * up.n_tiles, s)
+             : launch_gemm<EPI_GELU>(mx, mw1, mw1, up, num_sms, mtiles_max * up.n_tiles, s);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (between && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -522,8 +640,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
-  grid = static_cast<int>(std::min<int64_t>(num_sms, mtiles_max * dn.n_tiles));
-  err = launch_one<EPI_PLAIN_F32>(mh, mw2, mw2, dn, grid, s);
+  err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, dn, num_sms, mtiles_max * dn.n_tiles, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
