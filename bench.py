@@ -44,6 +44,8 @@ def parse_args(argv=None):
                     help="override T (profiling runs on a smaller batch)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (profiling runs with fewer experts' weights)")
+    ap.add_argument("--hidden", type=int, default=None,
+                    help="override H (profiling the router/permute/combine kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -104,6 +106,30 @@ def traffic_for(kernel_file, kernel):
         return float(rec["dram_bytes_per_launch"])
     except Exception:
         return None
+
+
+# ---------------------------------------------------------- ranks
+def rank_env():
+    """(rank, local_rank, world) from the torch.distributed launcher env."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def max_over_ranks(value, device=None):
+    """The largest of every rank's `value` (a time); identity on one rank.
+    Every rank must call it at the same point (it is a collective)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, steps, elapsed_ms):
+    """Units all ranks processed per second over the (max-over-ranks) time."""
+    return world * units_per_rank * steps / (elapsed_ms / 1e3)
 
 
 # --------------------------------------------------------------- clocks
@@ -202,14 +228,14 @@ def main(argv=None):
     from mixture_experts_layer_51_b200 import moe as M
     from mixture_experts_layer_51_b200.workloads import WORKLOADS, make_inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = rank_env()
     w = WORKLOADS[a.workload]
     if a.tokens:
         w = w.replace(T=a.tokens)
     if a.experts:
         w = w.replace(E=a.experts)
+    if a.hidden:
+        w = w.replace(H=a.hidden)
     peaks, peak_src = load_peaks()
 
     if a.impl == "reference":
@@ -265,16 +291,14 @@ def main(argv=None):
     elapsed_ms = start.elapsed_time(end)
     if world > 1:
         dist.barrier()
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     stage_ms = {s: 0.0 for s in M.STAGES}
     for i in range(a.steps):
         for s, v in M.stage_times_ms(evs[i]).items():
             stage_ms[s] += v / a.steps
 
     ms_per_step = elapsed_ms / a.steps
-    tokens_per_s = world * w.T * a.steps / (elapsed_ms / 1e3)
+    tokens_per_s = whole_job_rate(w.T, world, a.steps, elapsed_ms)
     tflops = total_flop * world * a.steps / (elapsed_ms / 1e3) / 1e12
 
     # End to end: tokens in pinned host memory, copies inside the timed call.
@@ -297,12 +321,9 @@ def main(argv=None):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev)
         nbytes = x.numel() * x.element_size()
-        e2e = {"value": world * w.T * a.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": whole_job_rate(w.T, world, a.steps, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                "ms_per_step": e2e_ms / a.steps}
 

@@ -19,57 +19,81 @@ namespace {
 
 constexpr int kCombineWarps = 8;
 
-template <bool OUT_BF16>
+// CH = 8-element chunks per lane per iteration: 2 for k <= 2 (more loads in
+// flight per lane), 1 otherwise (k rows already give 2k loads per chunk).
+template <bool OUT_BF16, int CH>
 __global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ pos,
                    const float* __restrict__ gate, int T, int d, int k, void* __restrict__ y) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= T) return;
-  int p[kMaxK];
-  float g[kMaxK];
+  constexpr int KJ = CH == 2 ? 2 : kMaxK;  // slots this instantiation handles
+  int p[KJ];
+  float g[KJ];
   {
     const int pl = lane < k ? pos[(int64_t)t * k + lane] : -1;
     const float gl = lane < k ? gate[(int64_t)t * k + lane] : 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
+    for (int j = 0; j < KJ; ++j) {
       p[j] = __shfl_sync(0xffffffffu, pl, j);
       g[j] = __shfl_sync(0xffffffffu, gl, j);
     }
   }
-  const int d4 = d / 4;  // float4 per row of o
-  // Each lane handles 8 consecutive elements (two float4) per step.
-  for (int c8 = lane; c8 * 8 < d; c8 += 32) {
-    float acc[8];
+  const int d4 = d / 4;   // float4 per row of o
+  const int n8 = d / 8;   // 8-element chunks per row
+  for (int c0 = lane; c0 < n8; c0 += 32 * CH) {
+    float4 v[KJ][CH][2];
+    // Issue every load of this iteration before any arithmetic.
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j = 0; j < KJ; ++j) {
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j < k && p[j] >= 0) {
-        const float4* row = o + (int64_t)p[j] * d4 + c8 * 2;
-        const float4 a = __ldcs(row);
-        const float4 b = __ldcs(row + 1);
-        acc[0] = fmaf(g[j], a.x, acc[0]);
-        acc[1] = fmaf(g[j], a.y, acc[1]);
-        acc[2] = fmaf(g[j], a.z, acc[2]);
-        acc[3] = fmaf(g[j], a.w, acc[3]);
-        acc[4] = fmaf(g[j], b.x, acc[4]);
-        acc[5] = fmaf(g[j], b.y, acc[5]);
-        acc[6] = fmaf(g[j], b.z, acc[6]);
-        acc[7] = fmaf(g[j], b.w, acc[7]);
+      for (int h = 0; h < CH; ++h) {
+        const int c8 = c0 + h * 32;
+        if (j < k && p[j] >= 0 && c8 < n8) {
+          const float4* row = o + (int64_t)p[j] * d4 + c8 * 2;
+          v[j][h][0] = __ldcs(row);
+          v[j][h][1] = __ldcs(row + 1);
+        } else {
+          v[j][h][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+          v[j][h][1] = v[j][h][0];
+        }
       }
     }
-    if (OUT_BF16) {
-      uint4 v;
-      v.x = pack_bf16x2(acc[0], acc[1]);
-      v.y = pack_bf16x2(acc[2], acc[3]);
-      v.z = pack_bf16x2(acc[4], acc[5]);
-      v.w = pack_bf16x2(acc[6], acc[7]);
-      reinterpret_cast<uint4*>(y)[(int64_t)t * (d / 8) + c8] = v;
-    } else {
-      float4* yr = reinterpret_cast<float4*>(y) + (int64_t)t * d4 + c8 * 2;
-      yr[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      yr[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+    for (int h = 0; h < CH; ++h) {
+      const int c8 = c0 + h * 32;
+      if (c8 >= n8) break;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KJ; ++j) {
+        // Slot order j = 0..k-1; absent slots hold zeros and add exactly 0.
+        if (j < k && p[j] >= 0) {
+          const float4 a = v[j][h][0], b = v[j][h][1];
+          acc[0] = fmaf(g[j], a.x, acc[0]);
+          acc[1] = fmaf(g[j], a.y, acc[1]);
+          acc[2] = fmaf(g[j], a.z, acc[2]);
+          acc[3] = fmaf(g[j], a.w, acc[3]);
+          acc[4] = fmaf(g[j], b.x, acc[4]);
+          acc[5] = fmaf(g[j], b.y, acc[5]);
+          acc[6] = fmaf(g[j], b.z, acc[6]);
+          acc[7] = fmaf(g[j], b.w, acc[7]);
+        }
+      }
+      if (OUT_BF16) {
+        uint4 q;
+        q.x = pack_bf16x2(acc[0], acc[1]);
+        q.y = pack_bf16x2(acc[2], acc[3]);
+        q.z = pack_bf16x2(acc[4], acc[5]);
+        q.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4*>(y)[(int64_t)t * n8 + c8] = q;
+      } else {
+        float4* yr = reinterpret_cast<float4*>(y) + (int64_t)t * d4 + c8 * 2;
+        yr[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        yr[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
     }
   }
 }
@@ -79,12 +103,19 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 cudaError_t launch_combine(const CombineArgs& a, moe_dtype dtype, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
   const int grid = (a.T + kCombineWarps - 1) / kCombineWarps;
-  if (dtype == MOE_BF16)
-    combine_kernel<true><<<grid, kCombineWarps * 32, 0, s>>>(
-        reinterpret_cast<const float4*>(a.o), a.pos, a.gate, a.T, a.d, a.k, a.y);
-  else
-    combine_kernel<false><<<grid, kCombineWarps * 32, 0, s>>>(
-        reinterpret_cast<const float4*>(a.o), a.pos, a.gate, a.T, a.d, a.k, a.y);
+  const float4* o = reinterpret_cast<const float4*>(a.o);
+  const int th = kCombineWarps * 32;
+  if (dtype == MOE_BF16) {
+    if (a.k <= 2)
+      combine_kernel<true, 2><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
+    else
+      combine_kernel<true, 1><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
+  } else {
+    if (a.k <= 2)
+      combine_kernel<false, 2><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
+    else
+      combine_kernel<false, 1><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
+  }
   return cudaGetLastError();
 }
 

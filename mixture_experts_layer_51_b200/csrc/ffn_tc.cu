@@ -57,7 +57,10 @@ constexpr int A_BYTES = TM * TK * 2;      // 16 KB
 constexpr int B_BOX_BYTES = 64 * TK * 2;  // one 64-column x 64-row box: 8 KB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * TN;
-constexpr int CONTROL_BYTES = 2048;
+constexpr int CONTROL_BYTES = 1536;
+#ifndef MOE_PAIR_STAGES
+#define MOE_PAIR_STAGES 6  // ring depth of the CTA-pair kernel (7 fills 227 KB)
+#endif
 // One CTA per tile (CG = 1): each CTA holds all 256 B columns.  A CTA pair
 // (CG = 2): each CTA holds half of them, so a stage is 32 KB and the ring
 // gets 6 stages in the same shared memory.
@@ -65,10 +68,11 @@ template <int CG>
 struct Cfg {
   static constexpr int B_BOXES = 4 / CG;
   static constexpr int STAGE_BYTES = A_BYTES + B_BOXES * B_BOX_BYTES;
-  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int STAGES = CG == 1 ? 4 : MOE_PAIR_STAGES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CONTROL_BYTES + 1024;
+  static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
 };
-constexpr int MAX_STAGES = 6;
+constexpr int MAX_STAGES = 8;
 
 enum Epi { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_PLAIN_F32 = 2 };
 

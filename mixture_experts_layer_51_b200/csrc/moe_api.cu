@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 #include "moe_internal.cuh"
 
@@ -250,7 +251,8 @@ namespace {
 moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, const void* W1,
                            const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
                            int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
-                           void* ws, size_t ws_bytes, const moe_ws_layout& L, cudaStream_t s) {
+                           void* ws, size_t ws_bytes, const moe_ws_layout& L, cudaStream_t s,
+                           bool clear_err = true) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
   float* gate = reinterpret_cast<float*>(w + L.gate);
@@ -260,7 +262,8 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
   int32_t* kept = reinterpret_cast<int32_t*>(w + L.kept_counts);
   int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
   int32_t* err = reinterpret_cast<int32_t*>(w + L.dev_error);
-  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (clear_err && cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   moe_status st = record_stage(0, s);
   if (st != MOE_OK) return st;
   st = moe_route(x, Wg, bias, T, d, E, k, dt, idx, gate, margin, s);
@@ -322,6 +325,52 @@ MOE_API moe_status moe_forward(const void* x, const void* Wg, const float* bias,
   return stats->device_error ? MOE_ERR_DEVICE : MOE_OK;
 }
 
+namespace {
+
+// Copy streams and events for the chunked host forward, created once per
+// device and kept for the life of the process (no device memory).
+constexpr int kMaxHostChunks = 8;
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in[kMaxHostChunks] = {}, out[kMaxHostChunks] = {};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+
+moe_status host_pipe(int dev, HostPipe** out) {
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  HostPipe& p = g_pipe[dev];
+  if (!p.ready) {
+    const unsigned f = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&p.start, f) != cudaSuccess ||
+        cudaEventCreateWithFlags(&p.done, f) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    for (int c = 0; c < kMaxHostChunks; ++c)
+      if (cudaEventCreateWithFlags(&p.in[c], f) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p.out[c], f) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    p.ready = true;
+  }
+  *out = &p;
+  return MOE_OK;
+}
+
+// Dropless layers are split into up to 4 token chunks of >= 1024 tokens so
+// the copy of chunk c+1 in and of chunk c-1 out overlap the forward of chunk
+// c.  Tokens are independent without a capacity, so y is unchanged; with a
+// capacity the batch stays whole (capacity is counted over the batch).
+int host_chunks(int32_t T, double cf) {
+  if (moe_capacity(T, 1, 1, cf) >= 0) return 1;
+  int n = T / 1024;
+  return n < 1 ? 1 : (n > 4 ? 4 : n);
+}
+
+}  // namespace
+
 MOE_API moe_status moe_forward_host(const void* x_host, void* y_host, void* x_dev, void* y_dev,
                                     const void* Wg, const float* bias, const void* W1,
                                     const void* W3, const void* W2, int32_t T, int32_t d,
@@ -332,16 +381,67 @@ MOE_API moe_status moe_forward_host(const void* x_host, void* y_host, void* x_de
   if (T == 0) return MOE_OK;
   if (!x_host || !y_host || !x_dev || !y_dev || !ws || ws_bytes < L.total) return MOE_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t bytes = static_cast<size_t>(T) * d * elt_size(dt);
-  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  moe_status st = forward_enqueue(x_dev, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, y_dev,
-                                  ws, ws_bytes, L, s);
+  const size_t row_bytes = static_cast<size_t>(d) * elt_size(dt);
+  const int nchunk = host_chunks(T, cf);
+  if (nchunk == 1) {
+    const size_t bytes = static_cast<size_t>(T) * row_bytes;
+    if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    moe_status st = forward_enqueue(x_dev, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt,
+                                    y_dev, ws, ws_bytes, L, s);
+    if (st != MOE_OK) return st;
+    if (cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    int32_t derr = 0;
+    st = read_device_error(L, ws, s, &derr);
+    if (st != MOE_OK) return st;
+    return derr ? MOE_ERR_DEVICE : MOE_OK;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* p = nullptr;
+  moe_status st = host_pipe(dev, &p);
   if (st != MOE_OK) return st;
-  if (cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+  // Every chunk reuses the workspace on `s` in order; its layout for the
+  // largest chunk fits inside the whole batch's.
+  const int32_t base = T / nchunk, rem = T % nchunk;
+  moe_ws_layout Lc;
+  if (!compute_layout(base + (rem ? 1 : 0), d, H, E, k, cf, dt, act, &Lc)) return MOE_ERR_ARG;
+  if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + Lc.dev_error, 0, sizeof(int32_t), s) !=
+          cudaSuccess ||
+      cudaEventRecord(p->start, s) != cudaSuccess ||
+      cudaStreamWaitEvent(p->h2d, p->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(p->d2h, p->start, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int32_t t0 = 0;
+  for (int c = 0; c < nchunk; ++c) {
+    const int32_t tc = base + (c < rem ? 1 : 0);
+    const size_t off = static_cast<size_t>(t0) * row_bytes, bytes = static_cast<size_t>(tc) * row_bytes;
+    const uint8_t* xh = static_cast<const uint8_t*>(x_host) + off;
+    uint8_t* xd = static_cast<uint8_t*>(x_dev) + off;
+    uint8_t* yd = static_cast<uint8_t*>(y_dev) + off;
+    uint8_t* yh = static_cast<uint8_t*>(y_host) + off;
+    if (cudaMemcpyAsync(xd, xh, bytes, cudaMemcpyHostToDevice, p->h2d) != cudaSuccess ||
+        cudaEventRecord(p->in[c], p->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(s, p->in[c], 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    // The largest chunk's layout serves every chunk (all regions are sized
+    // for at least tc tokens), so the error word stays in one place.
+    st = forward_enqueue(xd, Wg, bias, W1, W3, W2, tc, d, H, E, k, cf, act, dt, yd, ws, ws_bytes,
+                         Lc, s, /*clear_err=*/false);
+    if (st != MOE_OK) return st;
+    if (cudaEventRecord(p->out[c], s) != cudaSuccess ||
+        cudaStreamWaitEvent(p->d2h, p->out[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(yh, yd, bytes, cudaMemcpyDeviceToHost, p->d2h) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    t0 += tc;
+  }
+  if (cudaEventRecord(p->done, p->d2h) != cudaSuccess ||
+      cudaStreamWaitEvent(s, p->done, 0) != cudaSuccess)
     return MOE_ERR_CUDA;
   int32_t derr = 0;
-  st = read_device_error(L, ws, s, &derr);
+  st = read_device_error(Lc, ws, s, &derr);
   if (st != MOE_OK) return st;
   return derr ? MOE_ERR_DEVICE : MOE_OK;
 }

@@ -21,6 +21,8 @@
 // Every rank is computed from counts in token order: no atomics decide
 // placement, so the output is deterministic.
 
+#include <algorithm>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -106,10 +108,15 @@ __global__ void __launch_bounds__(kPermBlock)
   }
 }
 
+// Grid: (chunks of 32 tokens) x (slices of the row).  Every CTA of a chunk
+// recomputes the chunk's ranks (a few ballots); the slice-0 CTA writes pos;
+// each CTA copies its slice [v_begin, v_end) of the 16-byte vectors of every
+// kept row, so a small batch still spreads its copy over all SMs.
 template <int UNROLL>
 __global__ void __launch_bounds__(kPermBlock)
     permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx, int T,
-                           int dvec, int E, int k, int C, const int32_t* __restrict__ block_base,
+                           int dvec, int slice_vec, int E, int k, int C,
+                           const int32_t* __restrict__ block_base,
                            const int32_t* __restrict__ offsets, int32_t* __restrict__ pos,
                            uint4* __restrict__ xp) {
   __shared__ int wcnt[kWarpsPerBlock][kMaxE];
@@ -158,7 +165,7 @@ __global__ void __launch_bounds__(kPermBlock)
     for (int j = 0; j < k; ++j) {
       int p = -1;
       if (t < T && ej[j] >= 0 && ej[j] < E && rj[j] < C) p = offsets[ej[j]] + rj[j];
-      if (t < T) pos[(int64_t)t * k + j] = p;
+      if (t < T && blockIdx.y == 0) pos[(int64_t)t * k + j] = p;
       spos[lane * k + j] = p;
     }
   }
@@ -176,12 +183,14 @@ __global__ void __launch_bounds__(kPermBlock)
     }
     if (!any) continue;
     const uint4* src = x + (int64_t)t * dvec;
-    for (int v0 = lane; v0 < dvec; v0 += 32 * UNROLL) {
+    const int v_begin = blockIdx.y * slice_vec;
+    const int v_end = min(dvec, v_begin + slice_vec);
+    for (int v0 = v_begin + lane; v0 < v_end; v0 += 32 * UNROLL) {
       uint4 buf[UNROLL];
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
         const int v = v0 + u * 32;
-        if (v < dvec) buf[u] = __ldg(src + v);
+        if (v < v_end) buf[u] = __ldg(src + v);
       }
       for (int j = 0; j < k; ++j) {
         if (p[j] < 0) continue;
@@ -189,7 +198,7 @@ __global__ void __launch_bounds__(kPermBlock)
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
           const int v = v0 + u * 32;
-          if (v < dvec) dst[v] = buf[u];
+          if (v < v_end) dst[v] = buf[u];
         }
       }
     }
@@ -224,9 +233,16 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
                                                    a.kept_counts, a.offsets);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  permute_scatter_kernel<4><<<nchunk, kPermBlock, 0, s>>>(
-      static_cast<const uint4*>(a.x), a.idx, a.T, dvec, a.E, a.k, a.capacity, a.block_base,
-      a.offsets, a.pos, static_cast<uint4*>(a.xp));
+  // Enough row slices for ~4 CTAs per SM; each slice a multiple of 32 vectors.
+  constexpr int kTargetCtas = 4 * 148;
+  int nslice = (kTargetCtas + nchunk - 1) / nchunk;
+  nslice = std::max(1, std::min(nslice, (dvec + 31) / 32));
+  int slice_vec = (dvec + nslice - 1) / nslice;
+  slice_vec = (slice_vec + 31) / 32 * 32;
+  nslice = (dvec + slice_vec - 1) / slice_vec;
+  permute_scatter_kernel<4><<<dim3(nchunk, nslice), kPermBlock, 0, s>>>(
+      static_cast<const uint4*>(a.x), a.idx, a.T, dvec, slice_vec, a.E, a.k, a.capacity,
+      a.block_base, a.offsets, a.pos, static_cast<uint4*>(a.xp));
   return cudaGetLastError();
 }
 

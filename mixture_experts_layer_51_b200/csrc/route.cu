@@ -24,54 +24,72 @@
 namespace moe {
 namespace {
 
-constexpr int kRouteBM = 32;      // tokens per CTA
-constexpr int kRouteBK = 64;      // K (= d) per pipeline stage
-constexpr int kRouteStages = 6;
-constexpr int kRouteThreads = 64; // 2 warps x 16 tokens
-constexpr int kXStride = kRouteBK + 8;  // bf16 elements per smem row of x (pad: no bank conflicts)
+constexpr int kRouteThreads = 128; // 4 warps: (BM/16) token tiles x (4 / (BM/16)) K groups
 
+// Shared-memory row strides (bf16 elements), padded so ldmatrix rows fall
+// in different banks.
+__host__ __device__ constexpr int x_stride(int BK) { return BK + 8; }
 __host__ __device__ constexpr int wg_stride(int NT) { return NT * 8 + 8; }
-__host__ __device__ constexpr int stage_bytes(int NT) {
-  return kRouteBM * kXStride * 2 + kRouteBK * wg_stride(NT) * 2;
+__host__ __device__ constexpr int stage_bytes(int NT, int BM, int BK) {
+  return BM * x_stride(BK) * 2 + BK * wg_stride(NT) * 2;
 }
 
 // TopK over one token's E logits (descending; equal logits keep the lower
 // expert first), then softmax over the k selected ones.  `get(e)` returns
-// the logit of expert e.
-template <typename Get>
+// the logit of expert e.  The running top-(k+1) list lives in registers:
+// each new logit bubbles down a fixed compare-and-swap chain, and a strict
+// comparison leaves an equal earlier (lower-index) entry in front.
+template <int KM, typename Get>
 __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t, int32_t* idx,
                                                    float* gate, float* margin) {
-  float tv[kMaxK + 1];
-  int ti[kMaxK + 1];
-  const int keep = (k + 1 < E) ? k + 1 : E;  // also track the (k+1)-th for the margin
-  int n = 0;
+  float tv[KM];
+  int ti[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    tv[j] = -INFINITY;
+    ti[j] = -1;
+  }
   for (int e = 0; e < E; ++e) {
-    const float v = get(e);
-    if (n < keep || v > tv[n - 1]) {
-      int p = (n < keep) ? n : n - 1;
-      while (p > 0 && tv[p - 1] < v) {
-        tv[p] = tv[p - 1];
-        ti[p] = ti[p - 1];
-        --p;
+    float v = get(e);
+    int ei = e;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      // An unfilled slot (ti < 0) always takes the value, so -inf logits
+      // are still ranked in expert order.
+      if (v > tv[j] || ti[j] < 0) {
+        const float tvj = tv[j];
+        const int tij = ti[j];
+        tv[j] = v;
+        ti[j] = ei;
+        v = tvj;
+        ei = tij;
+        if (ei < 0) break;
       }
-      tv[p] = v;
-      ti[p] = e;
-      if (n < keep) ++n;
     }
   }
   const float m = tv[0];
-  float w[kMaxK];
+  float w[KM];
   float s = 0.f;
-  for (int j = 0; j < k; ++j) {
-    w[j] = expf(tv[j] - m);
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    w[j] = (j < k) ? expf(tv[j] - m) : 0.f;
     s += w[j];
   }
   const float inv = 1.0f / s;
-  for (int j = 0; j < k; ++j) {
-    idx[(int64_t)t * k + j] = ti[j];
-    gate[(int64_t)t * k + j] = w[j] * inv;
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    if (j < k) {
+      idx[(int64_t)t * k + j] = ti[j];
+      gate[(int64_t)t * k + j] = w[j] * inv;
+    }
   }
-  if (margin) margin[t] = (k < E) ? (tv[k - 1] - tv[k]) : INFINITY;
+  if (margin) {
+    float mg = INFINITY;
+#pragma unroll
+    for (int j = 1; j < KM; ++j)
+      if (j == k && k < E) mg = tv[j - 1] - tv[j];
+    margin[t] = mg;
+  }
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
@@ -114,8 +132,11 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// bf16 router.  NT = ceil(E / 8) column tiles of 8 experts.
-template <int NT>
+// bf16 router.  NT = ceil(E / 8) column tiles of 8 experts; BM tokens per
+// CTA.  The 4 warps split the work as (BM/16) token tiles x KG K-groups:
+// inside each 64-wide K stage, K-group g takes the 16-wide steps g, g+KG, ...
+// The KG partial sums of a token tile are added in a fixed order at the end.
+template <int NT, int BM, int BK, int STAGES, int KM>
 __global__ void __launch_bounds__(kRouteThreads)
     route_bf16_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wg,
                       const float* __restrict__ bias, int T, int d, int E, int k,
@@ -123,30 +144,35 @@ __global__ void __launch_bounds__(kRouteThreads)
                       float* __restrict__ margin) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int WS = wg_stride(NT);
-  constexpr int SB = stage_bytes(NT);
+  constexpr int XS = x_stride(BK);
+  constexpr int SB = stage_bytes(NT, BM, BK);
+  constexpr int CPR = BK / 8;        // 16-byte chunks per x row per stage
+  constexpr int MT = BM / 16;        // token tiles per CTA
+  constexpr int KG = 4 / MT;         // K groups
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int t0 = blockIdx.x * kRouteBM;
-  const int nk = (d + kRouteBK - 1) / kRouteBK;
+  const int mt = warp % MT, kg = warp / MT;
+  const int t0 = blockIdx.x * BM;
+  const int nk = (d + BK - 1) / BK;
   const bool vec_wg = (E % 8) == 0;
 
   auto x_tile = [&](int s) { return smem + s * SB; };
-  auto w_tile = [&](int s) { return smem + s * SB + kRouteBM * kXStride * 2; };
+  auto w_tile = [&](int s) { return smem + s * SB + BM * XS * 2; };
 
   auto load_stage = [&](int s, int kc) {
-    const int k0 = kc * kRouteBK;
-    // x: kRouteBM rows x 8 chunks of 16 bytes.
-    for (int i = tid; i < kRouteBM * 8; i += kRouteThreads) {
-      const int r = i >> 3, c = i & 7;
+    const int k0 = kc * BK;
+    // x: BM rows x CPR chunks of 16 bytes (each row segment contiguous).
+    for (int i = tid; i < BM * CPR; i += kRouteThreads) {
+      const int r = i / CPR, c = i % CPR;
       const int t = t0 + r, col = k0 + c * 8;
       const bool ok = (t < T) && (col < d);
       const __nv_bfloat16* src = ok ? x + (int64_t)t * d + col : x;
-      cp_async16(smem_u32(x_tile(s) + (r * kXStride + c * 8) * 2), src, ok ? 16 : 0);
+      cp_async16(smem_u32(x_tile(s) + (r * XS + c * 8) * 2), src, ok ? 16 : 0);
     }
-    // W_g rows k0 .. k0+63, columns 0 .. NT*8-1 (zero beyond E and d).
+    // W_g rows k0 .. k0+BK-1, columns 0 .. NT*8-1 (zero beyond E and d).
     if (vec_wg) {
       const int cpr = E / 8;  // 16-byte chunks per W_g row
-      for (int i = tid; i < kRouteBK * NT; i += kRouteThreads) {
+      for (int i = tid; i < BK * NT; i += kRouteThreads) {
         const int r = i / NT, c = i % NT;
         const int row = k0 + r;
         const bool ok = (row < d) && (c < cpr);
@@ -155,7 +181,7 @@ __global__ void __launch_bounds__(kRouteThreads)
       }
     } else {
       __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(w_tile(s));
-      for (int i = tid; i < kRouteBK * NT * 8; i += kRouteThreads) {
+      for (int i = tid; i < BK * NT * 8; i += kRouteThreads) {
         const int r = i / (NT * 8), c = i % (NT * 8);
         const int row = k0 + r;
         wt[r * WS + c] = (row < d && c < E) ? Wg[(int64_t)row * E + c] : __float2bfloat16(0.f);
@@ -170,22 +196,22 @@ __global__ void __launch_bounds__(kRouteThreads)
     for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
 
 #pragma unroll
-  for (int s = 0; s < kRouteStages - 1; ++s) {
+  for (int s = 0; s < STAGES - 1; ++s) {
     if (s < nk) load_stage(s, s);
     cp_async_commit();
   }
 
   for (int kc = 0; kc < nk; ++kc) {
-    cp_async_wait<kRouteStages - 2>();
+    cp_async_wait<STAGES - 2>();
     __syncthreads();
-    const int s = kc % kRouteStages;
+    const int s = kc % STAGES;
     const uint32_t xa = smem_u32(x_tile(s));
     const uint32_t wa = smem_u32(w_tile(s));
 #pragma unroll
-    for (int kk = 0; kk < kRouteBK / 16; ++kk) {
+    for (int kk = kg; kk < BK / 16; kk += KG) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(xa + ((warp * 16 + (lane & 15)) * kXStride + kk * 16 + (lane >> 4) * 8) * 2, a0, a1,
-              a2, a3);
+      ldsm_x4(xa + ((mt * 16 + (lane & 15)) * XS + kk * 16 + (lane >> 4) * 8) * 2, a0, a1, a2,
+              a3);
 #pragma unroll
       for (int n = 0; n + 1 < NT; n += 2) {
         uint32_t b0, b1, b2, b3;
@@ -200,34 +226,40 @@ __global__ void __launch_bounds__(kRouteThreads)
         mma_bf16_16816(acc[NT - 1], a0, a1, a2, a3, b0, b1);
       }
     }
-    const int nxt = kc + kRouteStages - 1;
-    if (nxt < nk) load_stage(nxt % kRouteStages, nxt);
+    const int nxt = kc + STAGES - 1;
+    if (nxt < nk) load_stage(nxt % STAGES, nxt);
     cp_async_commit();
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Logits to shared memory: [kRouteBM][NT*8 + 1] fp32 (reuses the ring).
+  // Partial logits to shared memory: [KG][BM][NT*8 + 1] fp32 (reuses the ring),
+  // then each token's KG partials are added in group order.
   float* lg = reinterpret_cast<float*>(smem);
   constexpr int LS = NT * 8 + 1;
   {
-    const int r = warp * 16 + (lane >> 2);
+    float* part = lg + kg * BM * LS;
+    const int r = mt * 16 + (lane >> 2);
     const int c = (lane & 3) * 2;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      lg[r * LS + n * 8 + c] = acc[n][0];
-      lg[r * LS + n * 8 + c + 1] = acc[n][1];
-      lg[(r + 8) * LS + n * 8 + c] = acc[n][2];
-      lg[(r + 8) * LS + n * 8 + c + 1] = acc[n][3];
+      part[r * LS + n * 8 + c] = acc[n][0];
+      part[r * LS + n * 8 + c + 1] = acc[n][1];
+      part[(r + 8) * LS + n * 8 + c] = acc[n][2];
+      part[(r + 8) * LS + n * 8 + c + 1] = acc[n][3];
     }
   }
   __syncthreads();
-  if (tid < kRouteBM) {
+  if (tid < BM) {
     const int t = t0 + tid;
     if (t < T) {
-      const float* row = lg + tid * LS;
-      auto get = [&](int e) { return bias ? row[e] + bias[e] : row[e]; };
-      topk_softmax_store(get, E, k, t, idx, gate, margin);
+      auto get = [&](int e) {
+        float v = lg[tid * LS + e];
+#pragma unroll
+        for (int g = 1; g < KG; ++g) v += lg[(g * BM + tid) * LS + e];
+        return bias ? v + bias[e] : v;
+      };
+      topk_softmax_store<KM>(get, E, k, t, idx, gate, margin);
     }
   }
 }
@@ -269,21 +301,46 @@ __global__ void __launch_bounds__(256)
   __syncwarp();
   if (lane == 0) {
     auto get = [&](int e) { return bias ? lg[warp][e] + bias[e] : lg[warp][e]; };
-    topk_softmax_store(get, E, k, t, idx, gate, margin);
+    topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin);
   }
 }
 
-template <int NT>
-cudaError_t launch_route_nt(const RouteArgs& a, cudaStream_t s) {
-  const int smem = kRouteStages * stage_bytes(NT);
-  cudaError_t err =
-      cudaFuncSetAttribute(route_bf16_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+template <int NT, int BM, int BK, int STAGES, int KM>
+cudaError_t launch_route_cfg(const RouteArgs& a, cudaStream_t s) {
+  constexpr int smem = STAGES * stage_bytes(NT, BM, BK);
+  static_assert(BM * (NT * 8 + 1) * 4 * (4 / (BM / 16)) <= smem, "epilogue buffer");
+  cudaError_t err = cudaFuncSetAttribute(route_bf16_kernel<NT, BM, BK, STAGES, KM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  const int grid = (a.T + kRouteBM - 1) / kRouteBM;
-  route_bf16_kernel<NT><<<grid, kRouteThreads, smem, s>>>(
+  const int grid = (a.T + BM - 1) / BM;
+  route_bf16_kernel<NT, BM, BK, STAGES, KM><<<grid, kRouteThreads, smem, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T,
       a.d, a.E, a.k, a.idx, a.gate, a.margin);
   return cudaGetLastError();
+}
+
+// Configurations chosen by a sweep on B200 (8192 x 4096, E = 8 and
+// 16384 x 2048, E = 64): 64-token tiles with 128-wide K stages were fastest,
+// because each stage re-streams a W_g chunk from L2 and larger token tiles
+// amortise it; fewer, longer-lived CTAs beat finer tiles here.
+template <int NT, int KM>
+cudaError_t launch_route_nt(const RouteArgs& a, cudaStream_t s) {
+  if (NT <= 2) return launch_route_cfg<NT, 64, 128, 4, KM>(a, s);
+  return launch_route_cfg<NT, 64, 128, 3, KM>(a, s);
+}
+
+template <int KM>
+cudaError_t launch_route_km(const RouteArgs& a, cudaStream_t s) {
+  switch ((a.E + 7) / 8) {
+    case 1: return launch_route_nt<1, KM>(a, s);
+    case 2: return launch_route_nt<2, KM>(a, s);
+    case 3: return launch_route_nt<3, KM>(a, s);
+    case 4: return launch_route_nt<4, KM>(a, s);
+    case 5: return launch_route_nt<5, KM>(a, s);
+    case 6: return launch_route_nt<6, KM>(a, s);
+    case 7: return launch_route_nt<7, KM>(a, s);
+    default: return launch_route_nt<8, KM>(a, s);
+  }
 }
 
 }  // namespace
@@ -296,16 +353,10 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
                                                     a.d, a.E, a.k, a.idx, a.gate, a.margin);
     return cudaGetLastError();
   }
-  switch ((a.E + 7) / 8) {
-    case 1: return launch_route_nt<1>(a, s);
-    case 2: return launch_route_nt<2>(a, s);
-    case 3: return launch_route_nt<3>(a, s);
-    case 4: return launch_route_nt<4>(a, s);
-    case 5: return launch_route_nt<5>(a, s);
-    case 6: return launch_route_nt<6>(a, s);
-    case 7: return launch_route_nt<7>(a, s);
-    default: return launch_route_nt<8>(a, s);
-  }
+  // KM = slots of the running top list (k + 1, rounded up to 3, 5 or 9).
+  if (a.k <= 2) return launch_route_km<3>(a, s);
+  if (a.k <= 4) return launch_route_km<5>(a, s);
+  return launch_route_km<kMaxK + 1>(a, s);
 }
 
 }  // namespace moe

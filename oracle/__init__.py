@@ -23,6 +23,7 @@ from .moe_oracle import (  # noqa: F401
     router_logits,
     top_k,
     gating_softmax,
+    gating_softmax_all,
     capacity,
     assign_capacity,
     silu,

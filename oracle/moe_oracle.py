@@ -37,6 +37,7 @@ __all__ = [
     "router_logits",
     "top_k",
     "gating_softmax",
+    "gating_softmax_all",
     "capacity",
     "assign_capacity",
     "silu",
@@ -102,6 +103,22 @@ def gating_softmax(sel_logits):
     s = _f64(sel_logits)
     z = np.exp(s - s.max(axis=1, keepdims=True))
     return z / z.sum(axis=1, keepdims=True)
+
+
+def gating_softmax_all(logits, idx):
+    """Switch order, Softmax then TopK: the softmax over all E logits of each
+    token, read at the selected experts.  The k gates no longer sum to one.
+
+    "[Paper Club] Upcycling ...": the original Switch Transformer applies the
+    softmax first, so the selected probabilities do not add up to one
+    (example 0.4 and 0.2); "How do Mixture of Expert Models Work?", "The Math
+    Behind MoEs": G(x) = Softmax(x . W_g).  TopK of the probabilities selects
+    the same experts as TopK of the logits (softmax is increasing).
+    """
+    logits = _f64(logits)
+    z = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p = z / z.sum(axis=1, keepdims=True)
+    return np.take_along_axis(p, np.asarray(idx, dtype=np.int64), axis=1)
 
 
 def capacity(T, E, k, cf):
@@ -179,14 +196,24 @@ def expert_ffn(xr, W1, W3, W2, act):
     return h @ _f64(W2)
 
 
-def _route(x, Wg, bias, k):
+def _gates(logits, idx, sel, gating, gate_scale):
+    if gating == "topk_softmax":
+        gate = gating_softmax(sel)
+    elif gating == "softmax_topk":
+        gate = gating_softmax_all(logits, idx)
+    else:
+        raise ValueError(gating)
+    return gate * float(gate_scale)
+
+
+def _route(x, Wg, bias, k, gating="topk_softmax", gate_scale=1.0):
     logits = router_logits(x, Wg, bias)
     idx, sel, margin = top_k(logits, k)
-    gate = gating_softmax(sel)
+    gate = _gates(logits, idx, sel, gating, gate_scale)
     return logits, idx, gate, margin
 
 
-def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act):
+def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act, gating="topk_softmax", gate_scale=1.0):
     """The whole layer: route -> TopK + softmax -> capacity -> permute ->
     expert FFN -> un-permute with the gate-weighted sum.
 
@@ -194,11 +221,16 @@ def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act):
     margin, C, counts, kept_counts, rank, kept.  Steps follow the MoE-layer
     walk-through on "[Paper Club] Upcycling ..." and the formula
     y = sum_i G(x)_i E_i(x) of "The Math Behind MoEs".
+
+    gating: "topk_softmax" (default, Mixtral) or "softmax_topk" (Switch
+    order); gate_scale multiplies every gate ("[Paper Club] Upcycling ...":
+    scaling the expert output by E/k restores the dense output scale when the
+    softmax comes first, x4 for 8 experts and top-2).
     """
     x = _f64(x)
     T, d = x.shape
     E = _f64(Wg).shape[1]
-    logits, idx, gate, margin = _route(x, Wg, bias, k)
+    logits, idx, gate, margin = _route(x, Wg, bias, k, gating, gate_scale)
     C = capacity(T, E, k, cf)
     counts, kept_counts, rank, kept = assign_capacity(idx, E, C)
     W1 = _f64(W1)
@@ -217,7 +249,8 @@ def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act):
                 counts=counts, kept_counts=kept_counts, rank=rank, kept=kept)
 
 
-def moe_forward_tokens(x_rows, logits_rows, sel_idx, kept, W1, W3, W2, act):
+def moe_forward_tokens(x_rows, logits_rows, sel_idx, kept, W1, W3, W2, act,
+                       gating="topk_softmax", gate_scale=1.0):
     """The layer output for a subset of tokens, given their routing.
 
     x_rows[n, d], logits_rows[n, E] (the oracle's own fp64 logits),
@@ -230,7 +263,8 @@ def moe_forward_tokens(x_rows, logits_rows, sel_idx, kept, W1, W3, W2, act):
     logits_rows = _f64(logits_rows)
     sel_idx = np.asarray(sel_idx, dtype=np.int64)
     kept = np.asarray(kept, dtype=bool)
-    gate = gating_softmax(np.take_along_axis(logits_rows, sel_idx, axis=1))
+    gate = _gates(logits_rows, sel_idx, np.take_along_axis(logits_rows, sel_idx, axis=1),
+                  gating, gate_scale)
     n = sel_idx.shape[0]
     # W1/W3/W2 may be full [E, ...] arrays or dicts {expert: matrix}; only the
     # experts that are used get converted to float64.

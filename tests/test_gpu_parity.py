@@ -104,6 +104,22 @@ def test_forward_host_matches_device_forward():
     assert np.array_equal(y_host.float().numpy(), g["y"])
 
 
+@pytest.mark.parametrize("T,cf", [(3001, 0.0), (4096, 0.0), (3001, 1.0)])
+def test_forward_host_chunked_matches_device_forward(T, cf):
+    """Dropless batches of >= 2048 tokens go through the chunked, overlapped
+    host path; per-token results must not change (bit-exact).  With a
+    capacity the batch stays whole."""
+    w = Workload("hostpipe", T=T, d=256, E=8, k=2, H=384, act="swiglu", dtype="bf16", cf=cf,
+                 seed=9)
+    inp = make_inputs(w, "cpu")
+    g = run_gpu(w, inp)
+    t = g["dev_inputs"]
+    for _ in range(2):
+        y_host = M.moe_forward_host(inp["x"].pin_memory(), t["Wg"], t["bias"], t["W1"], t["W3"],
+                                    t["W2"], w.k, w.cf, w.act)
+        assert np.array_equal(y_host.float().numpy(), g["y"])
+
+
 def test_stage_entry_points_match_forward():
     """moe_route -> moe_permute -> moe_grouped_ffn -> moe_unpermute_combine
     called one by one give the same bits as moe_forward."""

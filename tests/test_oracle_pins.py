@@ -376,3 +376,53 @@ def test_token_subset_matches_full_layer():
                                    r["kept"][rows], W1, W3, W2, "swiglu")
     np.testing.assert_allclose(y, r["y"][rows], rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(gate, r["gate"][rows], rtol=1e-15)
+
+
+# ------------------------------------------------ Switch-order gating
+def test_golden_switch_order_gates_04_02(golden_dir):
+    g = {r[0]: r[1:] for r in _read_golden(os.path.join(golden_dir, "gates_switch_order_04_02.txt"))}
+    logits = np.array([[float(v) for v in g["logits"]]])
+    k = int(g["k"][0])
+    idx, sel, _ = O.top_k(logits, k)
+    assert idx[0].tolist() == [int(v) for v in g["idx"]]
+    gate = O.gating_softmax_all(logits, idx)
+    np.testing.assert_allclose(gate[0], [float(v) for v in g["gates"]], rtol=0, atol=1e-15)
+    E = logits.shape[1]
+    r = O._gates(logits, idx, sel, "softmax_topk", E / k)
+    np.testing.assert_allclose(r[0], [float(v) for v in g["scaled"]], rtol=0, atol=1e-15)
+
+
+def test_switch_order_gates_are_the_dense_probabilities():
+    """Softmax-then-TopK gates are the dense softmax probabilities of the
+    selected experts: they sum to less than one unless k = E, and the
+    selection is the same as TopK of the logits."""
+    logits = RNG.standard_normal((300, 8)) * 2
+    idx, sel, _ = O.top_k(logits, 2)
+    g = O.gating_softmax_all(logits, idx)
+    dense = np.exp(logits) / np.exp(logits).sum(1, keepdims=True)
+    for t in range(300):
+        order = sorted(range(8), key=lambda e: (-dense[t, e], e))[:2]
+        assert idx[t].tolist() == order
+        np.testing.assert_allclose(g[t], dense[t, idx[t]], rtol=1e-13)
+    assert (g.sum(1) < 1).all()
+    idx8, sel8, _ = O.top_k(logits, 8)
+    np.testing.assert_allclose(O.gating_softmax_all(logits, idx8).sum(1), 1.0, atol=1e-14)
+
+
+def test_switch_order_upcycling_scale_restores_dense_output():
+    """Identical experts and a uniform router (all logits equal): every
+    softmax probability is 1/E, top-k gates sum to k/E, and the E/k scale of
+    "[Paper Club] Upcycling ..." brings the output back to the dense FFN."""
+    E, k, d, H = 8, 2, 8, 16
+    x, Wg, b, W1, W3, W2 = rand_layer(10, d, E, H, "swiglu")
+    Wg[:] = 0.0
+    W1[:] = W1[0]
+    W3[:] = W3[0]
+    W2[:] = W2[0]
+    dense = dense_ffn(x, W1[0], W3[0], W2[0], "swiglu")
+    r = O.moe_forward(x, Wg, None, W1, W3, W2, k, 0.0, "swiglu", gating="softmax_topk",
+                      gate_scale=E / k)
+    np.testing.assert_allclose(r["gate"], 0.5, atol=1e-15)
+    np.testing.assert_allclose(r["y"], dense, rtol=1e-12, atol=1e-12)
+    r1 = O.moe_forward(x, Wg, None, W1, W3, W2, k, 0.0, "swiglu", gating="softmax_topk")
+    np.testing.assert_allclose(r1["y"], dense * k / E, rtol=1e-12, atol=1e-12)
