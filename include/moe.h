@@ -70,6 +70,33 @@ typedef enum {
 typedef enum { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype;
 typedef enum { MOE_SWIGLU = 0, MOE_GELU = 1 } moe_act;
 
+/* Gate formula.  TOPK_SOFTMAX: Softmax(TopK(logits)), the k gates sum to one
+ * ("The Math Behind MoEs"; Mixtral).  SOFTMAX_TOPK: the softmax over all E
+ * logits read at the TopK experts, the Switch order ("[Paper Club]
+ * Upcycling ...": the selected gates no longer sum to one, e.g. 0.4 and 0.2).
+ * Both select the same experts. */
+typedef enum { MOE_GATE_TOPK_SOFTMAX = 0, MOE_GATE_SOFTMAX_TOPK = 1 } moe_gating;
+
+/* Which assignments a full expert keeps.  POSITION: the earliest tokens
+ * ("Take a Closer Look at the MoE LLM Routing", "Drop-towards-the-End").
+ * GATE: Batch Priority Routing ("Scaling Vision with Sparse Mixture of
+ * Experts", "Priority Routing"): tokens reach the queues in descending order
+ * of their largest gate, equal gates in position order, so the least
+ * important tokens are dropped. */
+typedef enum { MOE_PRIORITY_POSITION = 0, MOE_PRIORITY_GATE = 1 } moe_priority;
+
+/* Options of the *_ex entry points; NULL means all defaults. */
+typedef struct {
+  int32_t gating;      /* moe_gating; default MOE_GATE_TOPK_SOFTMAX                */
+  float gate_scale;    /* multiplies every gate, > 0; default 1.  E/k restores the
+                          dense output scale under SOFTMAX_TOPK ("[Paper Club]
+                          Upcycling ...": scale the expert output by the number
+                          of experts over top-k, x4 for 8 experts and top-2)   */
+  int32_t priority;    /* moe_priority; default MOE_PRIORITY_POSITION; only
+                          matters when a capacity is set                       */
+  int32_t reserved[5]; /* must be zero                                         */
+} moe_options;
+
 /* Filled by moe_forward when `stats` is non-NULL (after the stream drains). */
 typedef struct {
   int32_t counts[MOE_MAX_EXPERTS];      /* assignments routed to each expert */
@@ -97,6 +124,8 @@ typedef struct {
   size_t o;            /* fp32  [rows, d] expert outputs                    */
   size_t total;        /* == moe_workspace_bytes(...)                       */
   int64_t rows;        /* rows of xp/h/o (moe_max_permuted_rows)            */
+  size_t order;        /* int32 [T] queue order (priority routing only)     */
+  size_t prio_scratch; /* sort scratch (moe_priority_workspace_bytes)       */
 } moe_ws_layout;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -142,6 +171,12 @@ moe_status moe_route(const void* x, const void* Wg, const float* bias,
                      int32_t T, int32_t d, int32_t E, int32_t k, moe_dtype dtype,
                      int32_t* idx, float* gate, float* margin, void* stream);
 
+/* moe_route with options (gate formula and scale); opt may be NULL. */
+moe_status moe_route_ex(const void* x, const void* Wg, const float* bias,
+                        int32_t T, int32_t d, int32_t E, int32_t k, moe_dtype dtype,
+                        const moe_options* opt, int32_t* idx, float* gate, float* margin,
+                        void* stream);
+
 /* Permutation with optional capacity ("[Paper Club] Upcycling ...": tokens
  * that selected expert e are gathered into one matrix for e, and some are
  * dropped depending on the capacity factor; "Take a Closer Look at the MoE
@@ -159,6 +194,25 @@ moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d,
                        void* xp, int64_t xp_rows, int32_t* pos, int32_t* counts,
                        int32_t* kept_counts, int32_t* offsets,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* moe_permute serving the expert queues in a given order: queue position i
+ * is token order[i] (a permutation of 0..T-1, e.g. from moe_priority_order);
+ * order == NULL is token position, i.e. moe_permute.  Rows inside an expert
+ * block follow the queue order.  ws as for moe_permute. */
+moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order, int32_t T,
+                          int32_t d, int32_t E, int32_t k, double capacity_factor,
+                          moe_dtype dtype, void* xp, int64_t xp_rows, int32_t* pos,
+                          int32_t* counts, int32_t* kept_counts, int32_t* offsets,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Batch Priority Routing order ("Scaling Vision with Sparse Mixture of
+ * Experts", "Priority Routing"): order[T] = the tokens sorted by descending
+ * gate[t, 0] (each token's largest gate), equal gates in ascending position
+ * -- a stable, deterministic device radix sort.  gate [T, k] fp32 as from
+ * moe_route.  ws: at least moe_priority_workspace_bytes(T). */
+size_t moe_priority_workspace_bytes(int32_t T);
+moe_status moe_priority_order(const float* gate, int32_t T, int32_t k, int32_t* order,
+                              void* ws, size_t ws_bytes, void* stream);
 
 /* moe_permute without a caller-provided scratch buffer.  The pages have no
  * counterpart to this entry point: it exists for callers that cannot
@@ -223,6 +277,14 @@ moe_status moe_forward(const void* x, const void* Wg, const float* bias,
                        double capacity_factor, moe_act act, moe_dtype dtype,
                        void* y, void* ws, size_t ws_bytes, moe_stats* stats,
                        void* stream);
+
+/* moe_forward with options (gate formula and scale); opt may be NULL. */
+moe_status moe_forward_ex(const void* x, const void* Wg, const float* bias,
+                          const void* W1, const void* W3, const void* W2,
+                          int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                          double capacity_factor, moe_act act, moe_dtype dtype,
+                          const moe_options* opt, void* y, void* ws, size_t ws_bytes,
+                          moe_stats* stats, void* stream);
 
 /* moe_forward with the tokens in HOST memory: copies x_host [T, d] to
  * x_dev, runs the layer, copies y back to y_host [T, d], and waits for the

@@ -84,6 +84,7 @@ struct TcParams {
   int E;
   int n_tiles;     // column tiles per expert
   int64_t rows;    // rows of the A and output buffers
+  int b_chunked;   // 1: B maps are 4-D {64, K, N/64, E}; one load covers a CTA's chunks
   const int32_t* offsets;
   const int32_t* kept;
   int32_t* err;
@@ -251,7 +252,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t full_local = smem_u32(&c.full[stage]);
           const uint32_t a_dst = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t b_dst = a_dst + A_BYTES;
-          if (CG == 1) {
+          if (CG == 1 && p.b_chunked) {
+            mbar_arrive_expect_tx(full_local, STAGE_BYTES);
+            tma_load_2d(a_dst, &tmA, full_local, kb * TK, row0);
+            if (EPI == EPI_SWIGLU) {
+              const int c0 = n * (TN / 2) / 64;  // W1 then W3, two 64-column chunks each
+              tma_load_4d(b_dst, &tmB0, full_local, 0, kb * TK, c0, e);
+              tma_load_4d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_local, 0, kb * TK, c0, e);
+            } else {
+              tma_load_4d(b_dst, &tmB0, full_local, 0, kb * TK, n * TN / 64, e);
+            }
+          } else if (CG == 1) {
             mbar_arrive_expect_tx(full_local, STAGE_BYTES);
             tma_load_2d(a_dst, &tmA, full_local, kb * TK, row0);
             if (EPI == EPI_SWIGLU) {
@@ -272,7 +283,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t full_leader = mapa_shared(full_local, 0);
             if (leader) mbar_arrive_expect_tx(full_local, CG * STAGE_BYTES);
             tma_load_2d_pair(a_dst, &tmA, full_leader, kb * TK, row0);
-            if (EPI == EPI_SWIGLU) {
+            if (p.b_chunked) {
+              // leader: W1 columns (gate half), peer: W3 columns (up half) for
+              // SwiGLU; otherwise the two halves of the 256 columns
+              const CUtensorMap* mb = (EPI == EPI_SWIGLU && !leader) ? &tmB1 : &tmB0;
+              const int c0 = EPI == EPI_SWIGLU ? n * (TN / 2) / 64
+                                               : (n * TN + static_cast<int>(rank) * (TN / 2)) / 64;
+              tma_load_4d_pair(b_dst, mb, full_leader, 0, kb * TK, c0, e);
+            } else if (EPI == EPI_SWIGLU) {
               // leader: W1 columns (gate half); peer: W3 columns (up half)
               const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
               const int n0 = n * (TN / 2);
@@ -561,6 +579,23 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D view {64, K, N/64, E} of bf16 weights [E, K, N] (N % 64 == 0): a box of
+// {64, 64, chunks, 1} loads `chunks` adjacent 64-column chunks of 64 K-rows
+// in one instruction, in the same shared-memory layout as separate 3-D boxes
+// (chunk-major, 8 KB per chunk).
+bool make_map_w4d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N,
+                  uint32_t chunks) {
+  auto fn = encode_fn();
+  if (!fn || N % 64 != 0) return false;
+  cuuint64_t dims[4] = {64, K, N / 64, E};
+  cuuint64_t strides[3] = {N * 2, 128, K * N * 2};
+  cuuint32_t box[4] = {64, 64, chunks, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPI, int CG>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const TcParams& p, int groups, cudaStream_t s) {
@@ -610,10 +645,20 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   if (a.rows <= 0) return MOE_OK;
   CUtensorMap mx, mw1, mw3, mh, mw2;
   const bool swiglu = a.act == MOE_SWIGLU;
-  if (!make_map_2d(&mx, a.xp, a.rows, a.d, TM) || !make_map_3d(&mw1, a.W1, a.E, a.d, a.H) ||
-      (swiglu && !make_map_3d(&mw3, a.W3, a.E, a.d, a.H)) ||
-      !make_map_2d(&mh, a.h, a.rows, a.H, TM) || !make_map_3d(&mw2, a.W2, a.E, a.H, a.d))
+  const bool pairs = use_cta_pairs();
+  if (!make_map_2d(&mx, a.xp, a.rows, a.d, TM) || !make_map_2d(&mh, a.h, a.rows, a.H, TM))
     return MOE_ERR_CUDA;
+  // Weights: one 4-D load per K-step and CTA when the columns come in whole
+  // 64-wide chunks; per-chunk 3-D loads otherwise.
+  const bool up_chunked = a.H % 64 == 0, dn_chunked = a.d % 64 == 0;
+  const uint32_t up_chunks = pairs ? 2 : (swiglu ? 2 : 4), dn_chunks = pairs ? 2 : 4;
+  bool ok = up_chunked ? make_map_w4d(&mw1, a.W1, a.E, a.d, a.H, up_chunks) &&
+                             (!swiglu || make_map_w4d(&mw3, a.W3, a.E, a.d, a.H, up_chunks))
+                       : make_map_3d(&mw1, a.W1, a.E, a.d, a.H) &&
+                             (!swiglu || make_map_3d(&mw3, a.W3, a.E, a.d, a.H));
+  ok = ok && (dn_chunked ? make_map_w4d(&mw2, a.W2, a.E, a.H, a.d, dn_chunks)
+                         : make_map_3d(&mw2, a.W2, a.E, a.H, a.d));
+  if (!ok) return MOE_ERR_CUDA;
   const int64_t mtiles_max = (a.rows + TM - 1) / TM;
 
   TcParams up{};
@@ -624,6 +669,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.E = a.E;
   up.n_tiles = swiglu ? (a.H + TN / 2 - 1) / (TN / 2) : (a.H + TN - 1) / TN;
   up.rows = a.rows;
+  up.b_chunked = up_chunked ? 1 : 0;
   up.offsets = a.offsets;
   up.kept = a.kept_counts;
   up.err = a.dev_error;
@@ -641,6 +687,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.E = a.E;
   dn.n_tiles = (a.d + TN - 1) / TN;
   dn.rows = a.rows;
+  dn.b_chunked = dn_chunked ? 1 : 0;
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;

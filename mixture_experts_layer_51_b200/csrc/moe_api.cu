@@ -43,6 +43,23 @@ moe_status record_stage(int i, cudaStream_t s) {
   return cudaEventRecord(g_stage_events[i], s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Options with defaults filled in; false if they are invalid.
+bool read_options(const moe_options* opt, int* gating, float* gate_scale, int* priority = nullptr) {
+  *gating = MOE_GATE_TOPK_SOFTMAX;
+  *gate_scale = 1.0f;
+  if (priority) *priority = MOE_PRIORITY_POSITION;
+  if (!opt) return true;
+  if (opt->gating != MOE_GATE_TOPK_SOFTMAX && opt->gating != MOE_GATE_SOFTMAX_TOPK) return false;
+  if (!(opt->gate_scale > 0.0f) || isinf(opt->gate_scale)) return false;
+  if (opt->priority != MOE_PRIORITY_POSITION && opt->priority != MOE_PRIORITY_GATE) return false;
+  for (int i = 0; i < 5; ++i)
+    if (opt->reserved[i] != 0) return false;
+  *gating = opt->gating;
+  *gate_scale = opt->gate_scale;
+  if (priority) *priority = opt->priority;
+  return true;
+}
+
 struct DeviceInfo {
   int device = -1;
   int num_sms = 0;
@@ -96,6 +113,8 @@ bool compute_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, doubl
   L->offsets = take((kMaxE + 1) * 4);
   L->dev_error = take(4);
   L->scratch = take(permute_scratch_bytes(T, E));
+  L->order = take(static_cast<size_t>(T) * 4);
+  L->prio_scratch = take(priority_scratch_bytes(T));
   L->xp = take(static_cast<size_t>(rows) * d * es);
   L->h = take(static_cast<size_t>(rows) * H * es);
   L->o = take(static_cast<size_t>(rows) * d * 4);
@@ -154,25 +173,36 @@ MOE_API moe_status moe_workspace_layout(int32_t T, int32_t d, int32_t H, int32_t
   return compute_layout(T, d, H, E, k, cf, dt, act, out) ? MOE_OK : MOE_ERR_ARG;
 }
 
-MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, int32_t T,
-                             int32_t d, int32_t E, int32_t k, moe_dtype dt, int32_t* idx,
-                             float* gate, float* margin, void* stream) {
-  if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
+MOE_API moe_status moe_route_ex(const void* x, const void* Wg, const float* bias, int32_t T,
+                                int32_t d, int32_t E, int32_t k, moe_dtype dt,
+                                const moe_options* opt, int32_t* idx, float* gate, float* margin,
+                                void* stream) {
+  int gating;
+  float gate_scale;
+  if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt) || !read_options(opt, &gating, &gate_scale))
+    return MOE_ERR_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !Wg || !idx || !gate || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_ARG;
   DeviceInfo di;
   moe_status st = device_info(&di);
   if (st != MOE_OK) return st;
-  RouteArgs a{x, Wg, bias, T, d, E, k, idx, gate, margin};
+  RouteArgs a{x, Wg, bias, T, d, E, k, idx, gate, margin, gating, gate_scale};
   return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
 
-MOE_API moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d, int32_t E,
-                               int32_t k, double cf, moe_dtype dt, void* xp, int64_t xp_rows,
-                               int32_t* pos, int32_t* counts, int32_t* kept_counts,
-                               int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, int32_t T,
+                             int32_t d, int32_t E, int32_t k, moe_dtype dt, int32_t* idx,
+                             float* gate, float* margin, void* stream) {
+  return moe_route_ex(x, Wg, bias, T, d, E, k, dt, nullptr, idx, gate, margin, stream);
+}
+
+MOE_API moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order,
+                                  int32_t T, int32_t d, int32_t E, int32_t k, double cf,
+                                  moe_dtype dt, void* xp, int64_t xp_rows, int32_t* pos,
+                                  int32_t* counts, int32_t* kept_counts, int32_t* offsets,
+                                  void* ws, size_t ws_bytes, void* stream) {
   if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
   if (!counts || !kept_counts || !offsets) return MOE_ERR_ARG;
   if (T > 0) {
@@ -190,9 +220,36 @@ MOE_API moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int
   unsigned int* ticket = reinterpret_cast<unsigned int*>(
       static_cast<uint8_t*>(ws) + align_up(nblk * static_cast<size_t>(E) * 4));
   PermuteArgs a{x, idx, T, d, E, k, capacity_or_max(T, E, k, cf), xp, pos, counts, kept_counts,
-                offsets, block_base, ticket};
+                offsets, block_base, ticket, order};
   return launch_permute(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
                                                                                  : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d, int32_t E,
+                               int32_t k, double cf, moe_dtype dt, void* xp, int64_t xp_rows,
+                               int32_t* pos, int32_t* counts, int32_t* kept_counts,
+                               int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
+  return moe_permute_ex(x, idx, nullptr, T, d, E, k, cf, dt, xp, xp_rows, pos, counts,
+                        kept_counts, offsets, ws, ws_bytes, stream);
+}
+
+MOE_API size_t moe_priority_workspace_bytes(int32_t T) {
+  return T < 0 ? 0 : priority_scratch_bytes(T);
+}
+
+MOE_API moe_status moe_priority_order(const float* gate, int32_t T, int32_t k, int32_t* order,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || k < 1 || k > kMaxK) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!gate || !order || !ws || !aligned16(ws) || ws_bytes < priority_scratch_bytes(T))
+    return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_priority_order(gate, T, k, order, ws, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 MOE_API moe_status moe_grouped_ffn(const void* xp, int64_t rows, const int32_t* offsets,
@@ -252,7 +309,7 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
                            const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
                            int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
                            void* ws, size_t ws_bytes, const moe_ws_layout& L, cudaStream_t s,
-                           bool clear_err = true) {
+                           bool clear_err = true, const moe_options* opt = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   int32_t* idx = reinterpret_cast<int32_t*>(w + L.idx);
   float* gate = reinterpret_cast<float*>(w + L.gate);
@@ -266,11 +323,21 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
     return MOE_ERR_CUDA;
   moe_status st = record_stage(0, s);
   if (st != MOE_OK) return st;
-  st = moe_route(x, Wg, bias, T, d, E, k, dt, idx, gate, margin, s);
+  st = moe_route_ex(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, s);
   if (st == MOE_OK) st = record_stage(1, s);
   if (st != MOE_OK) return st;
-  st = moe_permute(x, idx, T, d, E, k, cf, dt, w + L.xp, L.rows, pos, counts, kept, offsets,
-                   w + L.scratch, permute_scratch_bytes(T, E), s);
+  int gating, priority;
+  float gate_scale;
+  read_options(opt, &gating, &gate_scale, &priority);
+  const int32_t* order = nullptr;
+  if (priority == MOE_PRIORITY_GATE && moe_capacity(T, E, k, cf) >= 0) {
+    st = moe_priority_order(gate, T, k, reinterpret_cast<int32_t*>(w + L.order),
+                            w + L.prio_scratch, priority_scratch_bytes(T), s);
+    if (st != MOE_OK) return st;
+    order = reinterpret_cast<const int32_t*>(w + L.order);
+  }
+  st = moe_permute_ex(x, idx, order, T, d, E, k, cf, dt, w + L.xp, L.rows, pos, counts, kept,
+                      offsets, w + L.scratch, permute_scratch_bytes(T, E), s);
   if (st == MOE_OK) st = record_stage(2, s);
   if (st != MOE_OK) return st;
   st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,
@@ -292,12 +359,17 @@ moe_status read_device_error(const moe_ws_layout& L, void* ws, cudaStream_t s, i
 
 }  // namespace
 
-MOE_API moe_status moe_forward(const void* x, const void* Wg, const float* bias, const void* W1,
-                               const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
-                               int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
-                               void* ws, size_t ws_bytes, moe_stats* stats, void* stream) {
+MOE_API moe_status moe_forward_ex(const void* x, const void* Wg, const float* bias,
+                                  const void* W1, const void* W3, const void* W2, int32_t T,
+                                  int32_t d, int32_t H, int32_t E, int32_t k, double cf,
+                                  moe_act act, moe_dtype dt, const moe_options* opt, void* y,
+                                  void* ws, size_t ws_bytes, moe_stats* stats, void* stream) {
   moe_ws_layout L;
+  int gating;
+  float gate_scale;
+  int priority;
   if (!compute_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
+  if (!read_options(opt, &gating, &gate_scale, &priority)) return MOE_ERR_ARG;
   if (T > 0 && (!y || !ws || ws_bytes < L.total || !aligned16(ws))) return MOE_ERR_ARG;
   if (T == 0) {
     if (stats) {
@@ -308,7 +380,7 @@ MOE_API moe_status moe_forward(const void* x, const void* Wg, const float* bias,
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   moe_status st = forward_enqueue(x, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, y, ws,
-                                  ws_bytes, L, s);
+                                  ws_bytes, L, s, true, opt);
   if (st != MOE_OK || !stats) return st;
   memset(stats, 0, sizeof(*stats));
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -323,6 +395,14 @@ MOE_API moe_status moe_forward(const void* x, const void* Wg, const float* bias,
   for (int e = 0; e < E; ++e) stats->kept += stats->kept_counts[e];
   stats->capacity = moe_capacity(T, E, k, cf);
   return stats->device_error ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+MOE_API moe_status moe_forward(const void* x, const void* Wg, const float* bias, const void* W1,
+                               const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
+                               int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
+                               void* ws, size_t ws_bytes, moe_stats* stats, void* stream) {
+  return moe_forward_ex(x, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, nullptr, y, ws,
+                        ws_bytes, stats, stream);
 }
 
 namespace {

@@ -107,6 +107,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                            int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 // tcgen05 (5th-generation tensor cores, accumulators in tensor memory) -----
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -202,6 +211,14 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                                 int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
                "r"(ncols)
@@ -273,6 +290,8 @@ struct RouteArgs {
   int32_t* idx;
   float* gate;
   float* margin;
+  int gating;        // moe_gating
+  float gate_scale;  // multiplies every gate
 };
 cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms);
 
@@ -288,9 +307,15 @@ struct PermuteArgs {
   int32_t* offsets;
   int32_t* block_base;  // [nblk * E] scratch
   unsigned int* ticket; // scratch counter
+  const int32_t* order = nullptr;  // queue order (token at position i), or null
 };
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s);
+
+size_t priority_scratch_bytes(int T);
+// Stable argsort of the tokens by descending slot-0 gate into order[T].
+cudaError_t launch_priority_order(const float* gate, int T, int k, int32_t* order, void* scratch,
+                                  cudaStream_t s);
 
 struct FfnArgs {
   const void* xp;

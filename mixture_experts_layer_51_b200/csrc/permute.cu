@@ -18,8 +18,11 @@
 //   pass 2 (scatter): per 32-token chunk, rank = block base + counts of the
 //     preceding chunks in the block + ballot prefix inside the chunk; then
 //     the chunk's rows are copied to xp with 16-byte loads and stores.
-// Every rank is computed from counts in token order: no atomics decide
-// placement, so the output is deterministic.
+// Every rank is computed from counts in queue order: no atomics decide
+// placement, so the output is deterministic.  The queue order is token
+// position, or -- Batch Priority Routing -- a given permutation `order`
+// (queue position i serves token order[i]); rows of an expert block then
+// follow that order.
 
 #include <algorithm>
 
@@ -44,17 +47,22 @@ __device__ __forceinline__ uint64_t expert_mask(const int32_t* __restrict__ idx,
   return m;
 }
 
+// Token served at queue position i: order[i] (Batch Priority Routing) or i.
+__device__ __forceinline__ int token_at(const int32_t* __restrict__ order, int i, int T) {
+  return (order && i < T) ? order[i] : i;
+}
+
 __global__ void __launch_bounds__(kPermBlock)
-    permute_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k, int C, int nblk,
-                         int32_t* __restrict__ block_base, unsigned int* __restrict__ ticket,
-                         int32_t* __restrict__ counts, int32_t* __restrict__ kept_counts,
-                         int32_t* __restrict__ offsets) {
+    permute_count_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ order, int T,
+                         int E, int k, int C, int nblk, int32_t* __restrict__ block_base,
+                         unsigned int* __restrict__ ticket, int32_t* __restrict__ counts,
+                         int32_t* __restrict__ kept_counts, int32_t* __restrict__ offsets) {
   __shared__ int wcnt[kWarpsPerBlock][kMaxE];
   __shared__ int padded[kMaxE];
   __shared__ bool is_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t = blockIdx.x * kPermBlock + tid;
-  const uint64_t mask = expert_mask(idx, t, T, k, E);
+  const int i = blockIdx.x * kPermBlock + tid;
+  const uint64_t mask = i < T ? expert_mask(idx, token_at(order, i, T), T, k, E) : 0ull;
   for (int e = 0; e < E; ++e) {
     const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
     if (lane == 0) wcnt[warp][e] = __popc(b);
@@ -114,7 +122,8 @@ __global__ void __launch_bounds__(kPermBlock)
 // kept row, so a small batch still spreads its copy over all SMs.
 template <int UNROLL>
 __global__ void __launch_bounds__(kPermBlock)
-    permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx, int T,
+    permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
+                           const int32_t* __restrict__ order, int T,
                            int dvec, int slice_vec, int E, int k, int C,
                            const int32_t* __restrict__ block_base,
                            const int32_t* __restrict__ offsets, int32_t* __restrict__ pos,
@@ -129,8 +138,8 @@ __global__ void __launch_bounds__(kPermBlock)
 
   // Counts of the chunks that precede this one inside its 256-token block.
   if (warp < cw) {
-    const int t = (blk * kWarpsPerBlock + warp) * kPermChunk + lane;
-    const uint64_t mask = expert_mask(idx, t, T, k, E);
+    const int i = (blk * kWarpsPerBlock + warp) * kPermChunk + lane;
+    const uint64_t mask = i < T ? expert_mask(idx, token_at(order, i, T), T, k, E) : 0ull;
     for (int e = 0; e < E; ++e) {
       const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
       if (lane == 0) wcnt[warp][e] = __popc(b);
@@ -144,7 +153,8 @@ __global__ void __launch_bounds__(kPermBlock)
   }
   __syncthreads();
   if (warp == 0) {
-    const int t = chunk * kPermChunk + lane;
+    const int i = chunk * kPermChunk + lane;
+    const int t = i < T ? token_at(order, i, T) : T;  // T: no token
     int ej[kMaxK];
     uint64_t mask = 0;
     for (int j = 0; j < k; ++j) {
@@ -173,8 +183,9 @@ __global__ void __launch_bounds__(kPermBlock)
 
   // Copy each kept token row to its k destinations.
   for (int i = warp; i < kPermChunk; i += kWarpsPerBlock) {
-    const int t = chunk * kPermChunk + i;
-    if (t >= T) break;
+    const int q = chunk * kPermChunk + i;
+    if (q >= T) break;
+    const int t = token_at(order, q, T);
     int p[kMaxK];
     bool any = false;
     for (int j = 0; j < k; ++j) {
@@ -228,7 +239,7 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
   const int dvec = a.d * elt / 16;
   cudaError_t err = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned int), s);
   if (err != cudaSuccess) return err;
-  permute_count_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.T, a.E, a.k, a.capacity, nblk,
+  permute_count_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.order, a.T, a.E, a.k, a.capacity, nblk,
                                                    a.block_base, a.ticket, a.counts,
                                                    a.kept_counts, a.offsets);
   err = cudaGetLastError();
@@ -241,7 +252,7 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
   slice_vec = (slice_vec + 31) / 32 * 32;
   nslice = (dvec + slice_vec - 1) / slice_vec;
   permute_scatter_kernel<4><<<dim3(nchunk, nslice), kPermBlock, 0, s>>>(
-      static_cast<const uint4*>(a.x), a.idx, a.T, dvec, slice_vec, a.E, a.k, a.capacity,
+      static_cast<const uint4*>(a.x), a.idx, a.order, a.T, dvec, slice_vec, a.E, a.k, a.capacity,
       a.block_base, a.offsets, a.pos, static_cast<uint4*>(a.xp));
   return cudaGetLastError();
 }

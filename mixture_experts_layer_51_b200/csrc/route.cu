@@ -41,7 +41,8 @@ __host__ __device__ constexpr int stage_bytes(int NT, int BM, int BK) {
 // comparison leaves an equal earlier (lower-index) entry in front.
 template <int KM, typename Get>
 __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t, int32_t* idx,
-                                                   float* gate, float* margin) {
+                                                   float* gate, float* margin, int gating,
+                                                   float gate_scale) {
   float tv[KM];
   int ti[KM];
 #pragma unroll
@@ -75,7 +76,12 @@ __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t,
     w[j] = (j < k) ? expf(tv[j] - m) : 0.f;
     s += w[j];
   }
-  const float inv = 1.0f / s;
+  if (gating == MOE_GATE_SOFTMAX_TOPK) {
+    // Switch order: normalise by the softmax denominator over all E logits.
+    s = 0.f;
+    for (int e = 0; e < E; ++e) s += expf(get(e) - m);
+  }
+  const float inv = gate_scale / s;
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
     if (j < k) {
@@ -141,7 +147,7 @@ __global__ void __launch_bounds__(kRouteThreads)
     route_bf16_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wg,
                       const float* __restrict__ bias, int T, int d, int E, int k,
                       int32_t* __restrict__ idx, float* __restrict__ gate,
-                      float* __restrict__ margin) {
+                      float* __restrict__ margin, int gating, float gate_scale) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int WS = wg_stride(NT);
   constexpr int XS = x_stride(BK);
@@ -259,7 +265,7 @@ __global__ void __launch_bounds__(kRouteThreads)
         for (int g = 1; g < KG; ++g) v += lg[(g * BM + tid) * LS + e];
         return bias ? v + bias[e] : v;
       };
-      topk_softmax_store<KM>(get, E, k, t, idx, gate, margin);
+      topk_softmax_store<KM>(get, E, k, t, idx, gate, margin, gating, gate_scale);
     }
   }
 }
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(256)
     route_fp32_kernel(const float* __restrict__ x, const float* __restrict__ Wg,
                       const float* __restrict__ bias, int T, int d, int E, int k,
                       int32_t* __restrict__ idx, float* __restrict__ gate,
-                      float* __restrict__ margin) {
+                      float* __restrict__ margin, int gating, float gate_scale) {
   __shared__ float lg[8][kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(256)
   __syncwarp();
   if (lane == 0) {
     auto get = [&](int e) { return bias ? lg[warp][e] + bias[e] : lg[warp][e]; };
-    topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin);
+    topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
   }
 }
 
@@ -315,7 +321,7 @@ cudaError_t launch_route_cfg(const RouteArgs& a, cudaStream_t s) {
   const int grid = (a.T + BM - 1) / BM;
   route_bf16_kernel<NT, BM, BK, STAGES, KM><<<grid, kRouteThreads, smem, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T,
-      a.d, a.E, a.k, a.idx, a.gate, a.margin);
+      a.d, a.E, a.k, a.idx, a.gate, a.margin, a.gating, a.gate_scale);
   return cudaGetLastError();
 }
 
@@ -350,7 +356,8 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
   if (dtype == MOE_FP32) {
     route_fp32_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(static_cast<const float*>(a.x),
                                                     static_cast<const float*>(a.Wg), a.bias, a.T,
-                                                    a.d, a.E, a.k, a.idx, a.gate, a.margin);
+                                                    a.d, a.E, a.k, a.idx, a.gate, a.margin,
+                                                    a.gating, a.gate_scale);
     return cudaGetLastError();
   }
   // KM = slots of the running top list (k + 1, rounded up to 3, 5 or 9).

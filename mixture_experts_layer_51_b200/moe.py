@@ -28,7 +28,11 @@ EXPORTED = (
     "moe_permute_workspace_bytes", "moe_workspace_bytes", "moe_workspace_layout",
     "moe_route", "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine",
     "moe_forward", "moe_forward_host", "moe_set_stage_events", "moe_permute_static",
+    "moe_route_ex", "moe_forward_ex", "moe_permute_ex", "moe_priority_order",
+    "moe_priority_workspace_bytes",
 )
+MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
+MOE_PRIORITY_POSITION, MOE_PRIORITY_GATE = 0, 1
 MOE_PERMUTE_STATIC_MAX_INTS = 1 << 18
 MOE_NUM_STAGE_EVENTS = 6
 STAGES = ("route", "permute", "ffn_up", "ffn_down", "combine")
@@ -51,10 +55,33 @@ class moe_stats(ctypes.Structure):
     ]
 
 
+class moe_options(ctypes.Structure):
+    _fields_ = [("gating", ctypes.c_int32), ("gate_scale", ctypes.c_float),
+                ("priority", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+
+
+def _options(gating="topk_softmax", gate_scale=1.0, priority="position"):
+    if gating in ("topk_softmax", MOE_GATE_TOPK_SOFTMAX):
+        g = MOE_GATE_TOPK_SOFTMAX
+    elif gating in ("softmax_topk", MOE_GATE_SOFTMAX_TOPK):
+        g = MOE_GATE_SOFTMAX_TOPK
+    else:
+        raise ValueError(gating)
+    if priority in ("position", MOE_PRIORITY_POSITION):
+        pr = MOE_PRIORITY_POSITION
+    elif priority in ("gate", MOE_PRIORITY_GATE):
+        pr = MOE_PRIORITY_GATE
+    else:
+        raise ValueError(priority)
+    return moe_options(gating=g, gate_scale=float(gate_scale), priority=pr)
+
+
 class moe_ws_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "idx", "gate", "margin", "pos", "counts", "kept_counts", "offsets", "dev_error",
-        "scratch", "xp", "h", "o", "total")] + [("rows", ctypes.c_int64)]
+        "scratch", "xp", "h", "o", "total")] + [("rows", ctypes.c_int64),
+                                                 ("order", ctypes.c_size_t),
+                                                 ("prio_scratch", ctypes.c_size_t)]
 
 
 _lib_handle = None
@@ -109,6 +136,20 @@ def lib():
     L.moe_permute_static.restype = ctypes.c_int
     L.moe_permute_static.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _D, ctypes.c_int, _P, _I64,
                                      _P, _P, _P, _P, _P]
+    L.moe_route_ex.restype = ctypes.c_int
+    L.moe_route_ex.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, ctypes.c_int,
+                               ctypes.POINTER(moe_options), _P, _P, _P, _P]
+    L.moe_forward_ex.restype = ctypes.c_int
+    L.moe_forward_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _D,
+                                 ctypes.c_int, ctypes.c_int, ctypes.POINTER(moe_options), _P, _P,
+                                 _SZ, ctypes.POINTER(moe_stats), _P]
+    L.moe_permute_ex.restype = ctypes.c_int
+    L.moe_permute_ex.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, _D, ctypes.c_int, _P, _I64,
+                                 _P, _P, _P, _P, _P, _SZ, _P]
+    L.moe_priority_workspace_bytes.restype = _SZ
+    L.moe_priority_workspace_bytes.argtypes = [_I32]
+    L.moe_priority_order.restype = ctypes.c_int
+    L.moe_priority_order.argtypes = [_P, _I32, _I32, _P, _P, _SZ, _P]
     L.moe_set_stage_events.restype = ctypes.c_int
     L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
     _lib_handle = L
@@ -193,6 +234,7 @@ def workspace_views(ws, layout, T, d, H, E, k, dtype):
         counts=view(layout.counts, E, torch.int32),
         kept_counts=view(layout.kept_counts, E, torch.int32),
         offsets=view(layout.offsets, E + 1, torch.int32),
+        order=view(layout.order, T, torch.int32),
         dev_error=view(layout.dev_error, 1, torch.int32),
         xp=view(layout.xp, rows * d, dtype).view(rows, d),
         h=view(layout.h, rows * H, dtype).view(rows, H),
@@ -201,21 +243,35 @@ def workspace_views(ws, layout, T, d, H, E, k, dtype):
 
 
 # ------------------------------------------------------------- entry points
-def moe_route(x, Wg, bias, k, idx=None, gate=None, margin=None, stream=None):
+def moe_route(x, Wg, bias, k, idx=None, gate=None, margin=None, stream=None,
+              gating="topk_softmax", gate_scale=1.0):
     T, d = x.shape
     E = Wg.shape[1]
     dev = x.device
     idx = idx if idx is not None else torch.empty((T, k), dtype=torch.int32, device=dev)
     gate = gate if gate is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
     margin = margin if margin is not None else torch.empty((T,), dtype=torch.float32, device=dev)
-    _check(lib().moe_route(_ptr(x), _ptr(Wg), _ptr(bias), T, d, E, k, _dtype_code(x),
-                           _ptr(idx), _ptr(gate), _ptr(margin), _stream(dev, stream)),
-           "moe_route")
+    opt = _options(gating, gate_scale)
+    _check(lib().moe_route_ex(_ptr(x), _ptr(Wg), _ptr(bias), T, d, E, k, _dtype_code(x),
+                              ctypes.byref(opt), _ptr(idx), _ptr(gate), _ptr(margin),
+                              _stream(dev, stream)), "moe_route_ex")
     return idx, gate, margin
 
 
+def moe_priority_order(gate, order=None, ws=None, stream=None):
+    """Tokens by descending slot-0 gate, ties in position order (int32 [T])."""
+    T, k = gate.shape
+    dev = gate.device
+    order = order if order is not None else torch.empty(T, dtype=torch.int32, device=dev)
+    need = lib().moe_priority_workspace_bytes(T)
+    ws = ws if ws is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().moe_priority_order(_ptr(gate), T, k, _ptr(order), _ptr(ws), ws.numel(),
+                                    _stream(dev, stream)), "moe_priority_order")
+    return order
+
+
 def moe_permute(x, idx, E, capacity_factor, xp=None, pos=None, counts=None, kept_counts=None,
-                offsets=None, ws=None, stream=None):
+                offsets=None, ws=None, stream=None, order=None):
     T, d = x.shape
     k = idx.shape[1]
     dev = x.device
@@ -227,10 +283,10 @@ def moe_permute(x, idx, E, capacity_factor, xp=None, pos=None, counts=None, kept
     offsets = offsets if offsets is not None else torch.empty(E + 1, dtype=torch.int32, device=dev)
     wsb = moe_permute_workspace_bytes(T, E)
     ws = ws if ws is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
-    _check(lib().moe_permute(_ptr(x), _ptr(idx), T, d, E, k, _cf(capacity_factor),
-                             _dtype_code(x), _ptr(xp), xp.shape[0], _ptr(pos), _ptr(counts),
-                             _ptr(kept_counts), _ptr(offsets), _ptr(ws), ws.numel(),
-                             _stream(dev, stream)), "moe_permute")
+    _check(lib().moe_permute_ex(_ptr(x), _ptr(idx), _ptr(order), T, d, E, k,
+                                _cf(capacity_factor), _dtype_code(x), _ptr(xp), xp.shape[0],
+                                _ptr(pos), _ptr(counts), _ptr(kept_counts), _ptr(offsets),
+                                _ptr(ws), ws.numel(), _stream(dev, stream)), "moe_permute_ex")
     return dict(xp=xp, pos=pos, counts=counts, kept_counts=kept_counts, offsets=offsets)
 
 
@@ -281,7 +337,8 @@ def moe_unpermute_combine(o, pos, gate, dtype, y=None, stream=None):
 
 
 def moe_forward(x, Wg, bias, W1, W3, W2, k, capacity_factor, act, y=None, ws=None,
-                stats=False, stream=None):
+                stats=False, stream=None, gating="topk_softmax", gate_scale=1.0,
+                priority="position"):
     """Whole layer.  Returns y, or (y, moe_stats) when stats=True."""
     T, d = x.shape
     E, _, H = W1.shape
@@ -290,12 +347,13 @@ def moe_forward(x, Wg, bias, W1, W3, W2, k, capacity_factor, act, y=None, ws=Non
     ws = ws if ws is not None else torch.empty(need, dtype=torch.uint8, device=dev)
     y = y if y is not None else torch.empty((T, d), dtype=x.dtype, device=dev)
     st = moe_stats() if stats else None
-    status = lib().moe_forward(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
-                               T, d, H, E, k, _cf(capacity_factor), _act_code(act),
-                               _dtype_code(x), _ptr(y), _ptr(ws), ws.numel(),
-                               ctypes.byref(st) if st is not None else None,
-                               _stream(dev, stream))
-    _check(status, "moe_forward")
+    opt = _options(gating, gate_scale, priority)
+    status = lib().moe_forward_ex(_ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                                  T, d, H, E, k, _cf(capacity_factor), _act_code(act),
+                                  _dtype_code(x), ctypes.byref(opt), _ptr(y), _ptr(ws),
+                                  ws.numel(), ctypes.byref(st) if st is not None else None,
+                                  _stream(dev, stream))
+    _check(status, "moe_forward_ex")
     return (y, st) if stats else y
 
 
@@ -341,9 +399,10 @@ class MoELayer:
     device (no allocation per call)."""
 
     def __init__(self, Wg, bias, W1, W3, W2, k, capacity_factor=0.0, act="swiglu",
-                 max_tokens=None):
+                 max_tokens=None, gating="topk_softmax", gate_scale=1.0, priority="position"):
         self.Wg, self.bias, self.W1, self.W3, self.W2 = Wg, bias, W1, W3, W2
         self.k, self.cf, self.act = k, capacity_factor, act
+        self.gating, self.gate_scale, self.priority = gating, gate_scale, priority
         self.E, self.d, self.H = W1.shape
         self.dtype = W1.dtype
         self.device = W1.device
@@ -371,4 +430,5 @@ class MoELayer:
     def __call__(self, x, y=None, stats=False, stream=None):
         return moe_forward(x, self.Wg, self.bias, self.W1, self.W3, self.W2, self.k, self.cf,
                            self.act, y=y, ws=self.workspace(x.shape[0]), stats=stats,
-                           stream=stream)
+                           stream=stream, gating=self.gating, gate_scale=self.gate_scale,
+                           priority=self.priority)

@@ -26,6 +26,7 @@ from .moe_oracle import (  # noqa: F401
     gating_softmax_all,
     capacity,
     assign_capacity,
+    priority_order,
     silu,
     gelu,
     expert_ffn,

@@ -40,6 +40,7 @@ __all__ = [
     "gating_softmax_all",
     "capacity",
     "assign_capacity",
+    "priority_order",
     "silu",
     "gelu",
     "expert_ffn",
@@ -137,17 +138,40 @@ def capacity(T, E, k, cf):
     return int(math.ceil(cf * T * k / E))
 
 
-def assign_capacity(idx, E, C):
-    """Queue every (token, slot) assignment at its expert in ascending token
-    position and keep the first C of each queue.
+def priority_order(gate):
+    """Batch Priority Routing order: tokens by descending importance, ties in
+    ascending position.
+
+    "Scaling Vision with Sparse Mixture of Experts", "Priority Routing":
+    tokens are sorted by an importance score and the least important are the
+    ones skipped when an expert is full.  The page does not define the score;
+    it is read here as the token's largest gate (slot 0).
+    """
+    g = _f64(gate)
+    return np.argsort(-g[:, 0], kind="stable")
+
+
+def assign_capacity(idx, E, C, order=None):
+    """Queue every (token, slot) assignment at its expert and keep the first
+    C of each queue.  Tokens arrive in ascending position, or in `order` (a
+    permutation of the tokens, e.g. priority_order) when given.
 
     Returns counts[E] (assignments per expert), kept_counts[E]
     (= min(count, C)), rank[T, k] (0-based place in the expert's queue) and
     kept[T, k] (bool).  "Take a Closer Look at the MoE LLM Routing",
-    "Drop-towards-the-End": later tokens are the ones dropped.
+    "Drop-towards-the-End": with position order, later tokens are the ones
+    dropped.
     """
     idx = np.asarray(idx, dtype=np.int64)
     T, k = idx.shape
+    if order is not None:
+        order = np.asarray(order, dtype=np.int64)
+        counts, kept_counts, rank_o, kept_o = assign_capacity(idx[order], E, C)
+        rank = np.empty_like(rank_o)
+        kept = np.empty_like(kept_o)
+        rank[order] = rank_o
+        kept[order] = kept_o
+        return counts, kept_counts, rank, kept
     flat = idx.reshape(-1)  # token-major: (t, j) -> t * k + j
     counts = np.bincount(flat, minlength=E).astype(np.int64)
     # Stable sort by expert keeps ascending token order inside each expert.
@@ -213,7 +237,8 @@ def _route(x, Wg, bias, k, gating="topk_softmax", gate_scale=1.0):
     return logits, idx, gate, margin
 
 
-def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act, gating="topk_softmax", gate_scale=1.0):
+def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act, gating="topk_softmax", gate_scale=1.0,
+                priority="position"):
     """The whole layer: route -> TopK + softmax -> capacity -> permute ->
     expert FFN -> un-permute with the gate-weighted sum.
 
@@ -225,14 +250,17 @@ def moe_forward(x, Wg, bias, W1, W3, W2, k, cf, act, gating="topk_softmax", gate
     gating: "topk_softmax" (default, Mixtral) or "softmax_topk" (Switch
     order); gate_scale multiplies every gate ("[Paper Club] Upcycling ...":
     scaling the expert output by E/k restores the dense output scale when the
-    softmax comes first, x4 for 8 experts and top-2).
+    softmax comes first, x4 for 8 experts and top-2).  priority: "position"
+    (default; drop the latest tokens) or "gate" (Batch Priority Routing: drop
+    the tokens with the smallest largest-gate first).
     """
     x = _f64(x)
     T, d = x.shape
     E = _f64(Wg).shape[1]
     logits, idx, gate, margin = _route(x, Wg, bias, k, gating, gate_scale)
     C = capacity(T, E, k, cf)
-    counts, kept_counts, rank, kept = assign_capacity(idx, E, C)
+    order = priority_order(gate) if priority == "gate" else None
+    counts, kept_counts, rank, kept = assign_capacity(idx, E, C, order)
     W1 = _f64(W1)
     W3 = _f64(W3) if W3 is not None else None
     W2 = _f64(W2)

@@ -90,7 +90,7 @@ def test_max_permuted_rows_bounds_every_routing(lib, T, E, k, cf):
 def test_workspace_layout_is_consistent(lib):
     L = M.moe_workspace_layout(8192, 4096, 14336, 8, 2, 0.0, "bf16", "swiglu")
     offs = [L.idx, L.gate, L.margin, L.pos, L.counts, L.kept_counts, L.offsets, L.dev_error,
-            L.scratch, L.xp, L.h, L.o]
+            L.scratch, L.order, L.prio_scratch, L.xp, L.h, L.o]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert L.rows == M.moe_max_permuted_rows(8192, 8, 2, 0.0)
     assert L.total >= L.o + L.rows * 4096 * 4
@@ -133,3 +133,19 @@ def test_empty_batch_is_a_no_op(lib):
                            M.MOE_SWIGLU, M.MOE_BF16, None, None, 0, ctypes.byref(st), None) == M.MOE_OK
     assert st.capacity == 0 and st.kept == 0
     assert lib.moe_route(None, None, None, 0, 64, 8, 2, M.MOE_BF16, None, None, None, None) == M.MOE_OK
+
+
+def test_invalid_options_are_rejected(lib):
+    fake = ctypes.c_void_p(0x10000)
+    for opt in (M.moe_options(gating=7, gate_scale=1.0), M.moe_options(gating=0, gate_scale=0.0),
+                M.moe_options(gating=1, gate_scale=-2.0),
+                M.moe_options(gating=0, gate_scale=float("inf"))):
+        assert lib.moe_route_ex(fake, fake, None, 16, 64, 8, 2, M.MOE_BF16, ctypes.byref(opt),
+                                fake, fake, None, None) == M.MOE_ERR_ARG
+    pr = M.moe_options(gating=0, gate_scale=1.0, priority=5)
+    assert lib.moe_route_ex(fake, fake, None, 16, 64, 8, 2, M.MOE_BF16, ctypes.byref(pr),
+                            fake, fake, None, None) == M.MOE_ERR_ARG
+    bad = M.moe_options(gating=0, gate_scale=1.0)
+    bad.reserved[3] = 1
+    assert lib.moe_route_ex(fake, fake, None, 16, 64, 8, 2, M.MOE_BF16, ctypes.byref(bad),
+                            fake, fake, None, None) == M.MOE_ERR_ARG

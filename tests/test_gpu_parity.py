@@ -85,6 +85,52 @@ def test_upcycling_identity_on_gpu():
     assert_y_close(g["y"], dense, "bf16", "upcycled layer vs dense FFN")
 
 
+@pytest.mark.parametrize("name,scale", [("mixtral_bf16", 4.0), ("finegrained_bf16", 1.0),
+                                        ("switch_tiny_fp32", 4.0)])
+def test_switch_order_gating_parity(name, scale):
+    """Softmax-then-TopK gates (Switch order) with the E/k output scale."""
+    w = SMALL[name]
+    full_parity(w, make_inputs(w, "cpu"), gating="softmax_topk", gate_scale=scale)
+
+
+def test_switch_order_upcycling_identity_on_gpu():
+    """Uniform router, identical experts, Softmax-then-TopK with gate scale
+    E/k: the layer equals the dense FFN (within bf16)."""
+    w = Workload("upcycle_switch", T=300, d=128, E=8, k=2, H=256, act="swiglu", dtype="bf16",
+                 cf=0.0, seed=6)
+    inp = make_inputs(w, "cpu")
+    inp["Wg"] = torch.zeros_like(inp["Wg"])
+    for key in ("W1", "W3", "W2"):
+        inp[key] = inp[key][:1].expand_as(inp[key]).contiguous()
+    g = run_gpu(w, inp, gating="softmax_topk", gate_scale=w.E / w.k)
+    np.testing.assert_allclose(g["gate"], 0.5, atol=1e-6)
+    dense = oracle.expert_ffn(inp["x"], inp["W1"][0], inp["W3"][0], inp["W2"][0], "swiglu")
+    assert_y_close(g["y"], dense, "bf16", "upcycled Switch-order layer vs dense FFN")
+
+
+@pytest.mark.parametrize("name", ["openmoe_skew_bf16", "switch_tiny_fp32", "finegrained_bf16"])
+def test_batch_priority_routing_parity(name):
+    """Capacity served by descending largest gate (Batch Priority Routing):
+    the device radix argsort equals the oracle's stable argsort of the same
+    gates, and the permutation and output follow the oracle."""
+    w = SMALL[name]
+    if w.cf <= 0:
+        w = w.replace(cf=0.5)
+    full_parity(w, make_inputs(w, "cpu"), priority="gate")
+
+
+def test_priority_order_ties_and_sizes():
+    """moe_priority_order alone: repeated gate values (stable ties) and sizes
+    around the 256-element sort block."""
+    rng = np.random.default_rng(3)
+    for T in (1, 255, 256, 257, 5000):
+        g = rng.integers(0, 7, size=(T, 2)).astype(np.float32) / 8 + 0.125
+        gate = torch.tensor(g, device="cuda")
+        order = M.moe_priority_order(gate)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_np(order), oracle.priority_order(g))
+
+
 def test_deterministic_bitwise():
     w = SMALL["finegrained_bf16"]
     inp = make_inputs(w, "cpu")

@@ -426,3 +426,52 @@ def test_switch_order_upcycling_scale_restores_dense_output():
     np.testing.assert_allclose(r["y"], dense, rtol=1e-12, atol=1e-12)
     r1 = O.moe_forward(x, Wg, None, W1, W3, W2, k, 0.0, "swiglu", gating="softmax_topk")
     np.testing.assert_allclose(r1["y"], dense * k / E, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------ Batch Priority Routing
+def brute_priority_queue(idx, prio, E, C):
+    """Sequential simulation: tokens arrive in descending priority (ties by
+    position); an expert accepts while it has room."""
+    T, k = idx.shape
+    arrival = sorted(range(T), key=lambda t: (-prio[t], t))
+    used = [0] * E
+    kept = np.zeros((T, k), dtype=bool)
+    for t in arrival:
+        for j in range(k):
+            e = int(idx[t, j])
+            if used[e] < C:
+                kept[t, j] = True
+            used[e] += 1
+    return kept
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(64, 4, 1, 0.5), (80, 8, 2, 1.0), (50, 6, 3, 0.6)])
+def test_priority_capacity_matches_sequential_queue(T, E, k, cf):
+    logits = RNG.standard_normal((T, E)) * 2
+    logits[:, 0] += 1.0
+    idx, sel, _ = O.top_k(logits, k)
+    gate = O.gating_softmax(sel)
+    # quantised gates make exact priority ties frequent
+    gate = np.round(gate * 8) / 8 + 1e-9 * (gate == 0)
+    C = O.capacity(T, E, k, cf)
+    _, kept_counts, _, kept = O.assign_capacity(idx, E, C, O.priority_order(gate))
+    assert (kept == brute_priority_queue(idx, gate[:, 0], E, C)).all()
+    assert (kept_counts == np.minimum(np.bincount(idx.ravel(), minlength=E), C)).all()
+
+
+def test_priority_drops_least_important_tokens():
+    """At every expert, each dropped assignment has a priority no higher than
+    every kept one ("Priority Routing": the least important are skipped)."""
+    T, E, k = 300, 8, 2
+    logits = RNG.standard_normal((T, E))
+    logits[:, :2] += 1.5
+    idx, sel, _ = O.top_k(logits, k)
+    gate = O.gating_softmax(sel)
+    C = O.capacity(T, E, k, 1.0)
+    _, _, _, kept = O.assign_capacity(idx, E, C, O.priority_order(gate))
+    assert not kept.all()
+    for e in range(E):
+        pk = gate[:, 0][np.nonzero((idx == e) & kept)[0]]
+        pd = gate[:, 0][np.nonzero((idx == e) & ~kept)[0]]
+        if pk.size and pd.size:
+            assert pd.max() <= pk.min()
