@@ -26,10 +26,14 @@ from .moe_oracle import (  # noqa: F401
     gating_softmax_all,
     capacity,
     assign_capacity,
+    assign_capacity_shard,
     priority_order,
     silu,
     gelu,
     expert_ffn,
     moe_forward,
     moe_forward_tokens,
+    expert_choice_scores,
+    expert_choice_select,
+    moe_forward_expert_choice,
 )

@@ -24,6 +24,15 @@ Readings of points the pages leave open (each also listed in the design doc):
   renormalisation).
 * SwiGLU expert: (SiLU(x W1) * (x W3)) W2, SiLU(z) = z / (1 + e^-z).
   GELU expert: GELU(x W1) W2 with the exact erf form.  No expert biases.
+* Expert-choice routing ("[Paper Club] Upcycling ...", the Q&A on expert
+  choice: the selection is reversed, every expert takes a fixed number of
+  tokens, a token may get no expert, several, or all): the token-to-expert
+  affinity is the router probability Softmax(x W_g) over all E experts (the
+  G(x) of "The Math Behind MoEs" before any TopK); each expert takes the
+  C = ceil(cf * T * k / E) tokens (at most T) with the largest affinity to it,
+  equal affinities -> lower position first, k read as the average number of
+  experts per token; the output is the affinity-weighted sum over the experts
+  that took the token, with no renormalisation.
 """
 
 from __future__ import annotations
@@ -46,6 +55,10 @@ __all__ = [
     "expert_ffn",
     "moe_forward",
     "moe_forward_tokens",
+    "assign_capacity_shard",
+    "expert_choice_scores",
+    "expert_choice_select",
+    "moe_forward_expert_choice",
 ]
 
 
@@ -190,6 +203,27 @@ def assign_capacity(idx, E, C, order=None):
     return counts, kept_counts, rank, kept
 
 
+def assign_capacity_shard(idx_shard, E, C, prior):
+    """The capacity step for one shard of a batch whose tokens are split by
+    position over ranks (shard r holds a contiguous range of positions).
+
+    prior[e] counts the assignments to expert e from all lower-position
+    shards.  In the whole batch's position-ordered queue of expert e, this
+    shard's i-th assignment sits at place prior[e] + i, so it is kept iff
+    that place is below C ("Drop-towards-the-End" applied to the whole
+    batch, "Take a Closer Look at the MoE LLM Routing").  Returns counts,
+    kept_counts, rank (local place) and kept as assign_capacity does.
+    """
+    counts, _, rank, _ = assign_capacity(idx_shard, E, None)
+    idx_shard = np.asarray(idx_shard, dtype=np.int64)
+    prior = np.asarray(prior, dtype=np.int64)
+    if C is None:
+        return counts, counts.copy(), rank, np.ones(rank.shape, dtype=bool)
+    room = np.maximum(0, C - prior)
+    kept = rank < room[idx_shard]
+    return counts, np.minimum(counts, room), rank, kept
+
+
 def silu(z):
     """SiLU(z) = z / (1 + exp(-z)) (the gate of SwiGLU)."""
     z = _f64(z)
@@ -306,3 +340,58 @@ def moe_forward_tokens(x_rows, logits_rows, sel_idx, kept, W1, W3, W2, act,
                          W2[e], act)
         y[rr] += gate[rr, jj][:, None] * out
     return y, gate
+
+
+def expert_choice_scores(logits):
+    """Token-to-expert affinity for expert-choice routing: the softmax of
+    each token's logits over all E experts (largest subtracted)."""
+    logits = _f64(logits)
+    z = np.exp(logits - logits.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def expert_choice_select(scores, C):
+    """Each expert's choice: sel[t, e] is True iff token t is among the
+    min(C, T) tokens with the largest scores[:, e], equal scores taken in
+    ascending position.  Returns sel [T, E] (bool) and, per expert, its
+    chosen tokens in ascending position (the order of its rows)."""
+    scores = _f64(scores)
+    T, E = scores.shape
+    n = min(int(C), T)
+    sel = np.zeros((T, E), dtype=bool)
+    for e in range(E):
+        # stable sort of the negated scores: descending score, ties by position
+        order = np.argsort(-scores[:, e], kind="stable")
+        sel[order[:n], e] = True
+    tokens = [np.nonzero(sel[:, e])[0] for e in range(E)]
+    return sel, tokens
+
+
+def moe_forward_expert_choice(x, Wg, bias, W1, W3, W2, k, cf, act, scores=None):
+    """The layer with expert-choice routing: affinity -> every expert takes
+    its top-C tokens -> expert FFN on them -> each token sums
+    affinity * output over the experts that took it (ascending expert).
+
+    cf must be > 0 (the experts' fixed intake is C = ceil(cf * T * k / E)).
+    scores: optional [T, E] affinities to select on instead of the oracle's
+    own (to replay another implementation's fp32 decision); the outputs are
+    then weighted by those given scores too.
+    """
+    x = _f64(x)
+    T = x.shape[0]
+    E = _f64(Wg).shape[1]
+    C = capacity(T, E, k, cf)
+    if C is None:
+        raise ValueError("expert-choice routing needs a finite capacity factor")
+    logits = router_logits(x, Wg, bias)
+    S = expert_choice_scores(logits) if scores is None else _f64(scores)
+    sel, tokens = expert_choice_select(S, C)
+    W2 = _f64(W2)
+    y = np.zeros((T, W2.shape[2]), dtype=np.float64)
+    for e in range(E):
+        tt = tokens[e]
+        if tt.size == 0:
+            continue
+        out = expert_ffn(x[tt], _f64(W1[e]), None if W3 is None else _f64(W3[e]), W2[e], act)
+        y[tt] += S[tt, e][:, None] * out
+    return dict(y=y, logits=logits, scores=S, C=C, sel=sel, tokens=tokens)

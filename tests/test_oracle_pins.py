@@ -475,3 +475,138 @@ def test_priority_drops_least_important_tokens():
         pd = gate[:, 0][np.nonzero((idx == e) & ~kept)[0]]
         if pk.size and pd.size:
             assert pd.max() <= pk.min()
+
+
+@pytest.mark.parametrize("T,E,k,cf,bounds", [
+    (200, 8, 2, 1.0, (0, 70, 130, 200)),
+    (96, 4, 1, 0.5, (0, 0, 50, 96)),       # an empty shard
+    (150, 6, 3, 0.8, (0, 1, 149, 150)),    # one-token shards
+    (64, 8, 2, 0.0, (0, 32, 64)),          # dropless
+])
+def test_sharded_capacity_concatenates_to_whole_batch(T, E, k, cf, bounds):
+    """Shards of a batch, each given the assignments of the lower-position
+    shards, keep exactly the assignments the whole batch keeps: checked
+    against the one-at-a-time queue on the whole batch."""
+    logits = RNG.standard_normal((T, E))
+    logits[:, 0] += 1.2  # a hot expert, so capacity binds
+    idx, _, _ = O.top_k(logits, k)
+    C = O.capacity(T, E, k, cf)
+    want = brute_capacity_queue(idx, E, C)[0]
+    prior = np.zeros(E, dtype=np.int64)
+    got = []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        counts, kept_counts, _, kept = O.assign_capacity_shard(idx[a:b], E, C, prior)
+        assert (kept_counts == kept.reshape(-1).astype(np.int64) @ np.eye(E, dtype=np.int64)[
+            idx[a:b].reshape(-1)]).all()
+        got.append(kept)
+        prior = prior + np.bincount(idx[a:b].reshape(-1), minlength=E)
+    assert (np.concatenate(got) == want).all()
+
+
+# ------------------------------------------------ expert-choice routing
+def test_golden_expert_choice_t5_e2(golden_dir):
+    g = {r[0]: r[1:] for r in _read_golden(os.path.join(golden_dir, "expert_choice_t5_e2.txt"))}
+    logits = np.array([[float(v) for v in g[f"logits_{t}"]] for t in range(5)])
+    k = int(g["k"][0])
+    S = O.expert_choice_scores(logits)
+    np.testing.assert_allclose(S[:, 0], [0.75, 0.5, 0.25, 0.9, 0.5], rtol=0, atol=1e-15)
+    for case in ("case_a", "case_b"):
+        cf, C = float(g[case][0]), int(g[case][1])
+        assert O.capacity(5, 2, k, cf) == C
+        sel, tokens = O.expert_choice_select(S, C)
+        assert tokens[0].tolist() == [int(v) for v in g[case + "_e0"]]
+        assert tokens[1].tolist() == [int(v) for v in g[case + "_e1"]]
+        np.testing.assert_allclose((S * sel).sum(1), [float(v) for v in g[case + "_weight"]],
+                                   rtol=0, atol=1e-15)
+
+
+def brute_expert_choice(scores, C):
+    """Selection by the defining property, with loops only: expert e takes
+    min(C, T) tokens, and every taken token beats every other token (larger
+    score, or an equal score at a lower position)."""
+    T, E = scores.shape
+    n = min(C, T)
+    sel = np.zeros((T, E), dtype=bool)
+    for e in range(E):
+        for t in range(T):
+            # tokens that beat t at expert e
+            better = 0
+            for u in range(T):
+                if scores[u, e] > scores[t, e] or (scores[u, e] == scores[t, e] and u < t):
+                    better += 1
+            sel[t, e] = better < n
+    return sel
+
+
+@pytest.mark.parametrize("T,E,C", [(12, 3, 4), (9, 4, 9), (10, 2, 15), (7, 5, 0), (16, 4, 5)])
+def test_expert_choice_selection_matches_definition(T, E, C):
+    # quantised scores make exact ties common
+    scores = np.round(RNG.random((T, E)) * 4) / 4
+    sel, tokens = O.expert_choice_select(scores, C)
+    assert (sel == brute_expert_choice(scores, C)).all()
+    assert (sel.sum(0) == min(C, T)).all()
+    for e in range(E):
+        assert tokens[e].tolist() == sorted(tokens[e].tolist())
+
+
+def test_expert_choice_uniform_router_takes_the_first_tokens():
+    """W_g = 0: every affinity is 1/E, so every expert takes tokens 0..C-1;
+    with identical experts y_t = FFN(x_t) there (sum of E weights 1/E) and
+    0 for the tokens no expert took."""
+    T, d, E, H, k, cf = 20, 6, 4, 10, 1, 1.0
+    x = RNG.standard_normal((T, d))
+    W1 = np.repeat(RNG.standard_normal((1, d, H)), E, 0)
+    W3 = np.repeat(RNG.standard_normal((1, d, H)), E, 0)
+    W2 = np.repeat(RNG.standard_normal((1, H, d)), E, 0)
+    r = O.moe_forward_expert_choice(x, np.zeros((d, E)), None, W1, W3, W2, k, cf, "swiglu")
+    C = r["C"]
+    assert C == 5
+    assert all(t.tolist() == list(range(C)) for t in r["tokens"])
+    dense = brute_ffn(x, W1[0], W3[0], W2[0], "swiglu")
+    np.testing.assert_allclose(r["y"][:C], dense[:C], rtol=1e-12, atol=1e-12)
+    assert (r["y"][C:] == 0).all()
+
+
+def test_expert_choice_single_expert_is_dense():
+    T, d, H = 9, 5, 7
+    x = RNG.standard_normal((T, d))
+    W1, W3, W2 = (RNG.standard_normal((1, d, H)), RNG.standard_normal((1, d, H)),
+                  RNG.standard_normal((1, H, d)))
+    r = O.moe_forward_expert_choice(x, RNG.standard_normal((d, 1)), None, W1, W3, W2, 1, 1.0,
+                                    "swiglu")
+    np.testing.assert_allclose(r["y"], brute_ffn(x, W1[0], W3[0], W2[0], "swiglu"),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_expert_choice_with_room_for_every_token_is_token_choice_top_e():
+    """C >= T: every expert takes every token, y = sum_e softmax_e * E_e(x),
+    which is the dropless token-choice layer with k = E."""
+    T, d, E, H = 11, 6, 3, 8
+    x, Wg, bias, W1, W3, W2 = rand_layer(T, d, E, H, "swiglu", bias=True)
+    r = O.moe_forward_expert_choice(x, Wg, bias, W1, W3, W2, E, 1.0, "swiglu")
+    assert r["C"] >= T and r["sel"].all()
+    ref = O.moe_forward(x, Wg, bias, W1, W3, W2, E, 0.0, "swiglu")
+    np.testing.assert_allclose(r["y"], ref["y"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_expert_choice_layer_matches_per_token_bruteforce(act):
+    T, d, E, H, k, cf = 14, 5, 4, 6, 2, 0.75
+    x, Wg, bias, W1, W3, W2 = rand_layer(T, d, E, H, act, bias=True)
+    r = O.moe_forward_expert_choice(x, Wg, bias, W1, W3, W2, k, cf, act)
+    logits = brute_matmul(x, Wg) + bias[None, :]
+    y = np.zeros((T, d))
+    C = math.ceil(cf * T * k / E)
+    S = np.zeros((T, E))
+    for t in range(T):
+        m = max(logits[t])
+        w = [math.exp(v - m) for v in logits[t]]
+        S[t] = [v / sum(w) for v in w]
+    sel = brute_expert_choice(S, C)
+    for t in range(T):
+        for e in range(E):
+            if sel[t, e]:
+                y[t] += S[t, e] * brute_ffn(x[t:t + 1], W1[e], None if W3 is None else W3[e],
+                                            W2[e], act)[0]
+    assert (r["sel"] == sel).all()
+    np.testing.assert_allclose(r["y"], y, rtol=1e-10, atol=1e-12)
