@@ -46,6 +46,12 @@ def parse_args(argv=None):
                     help="override E (profiling runs with fewer experts' weights)")
     ap.add_argument("--hidden", type=int, default=None,
                     help="override H (profiling the router/permute/combine kernels)")
+    ap.add_argument("--capacity-factor", type=float, default=None,
+                    help="override the workload's capacity factor")
+    ap.add_argument("--routing", choices=["token_choice", "expert_choice"],
+                    default="token_choice",
+                    help="expert_choice: every expert takes its top-C tokens "
+                         "(capacity factor 1.0 unless one is given)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -65,7 +71,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic(w, n_kept, tokens_with_kept):
+def algorithmic(w, n_kept, tokens_with_kept, routing="token_choice"):
     """FLOPs and HBM bytes of each stage for one forward (padding and dropped
     assignments are never counted)."""
     s = 2 if w.dtype == "bf16" else 4
@@ -88,6 +94,14 @@ def algorithmic(w, n_kept, tokens_with_kept):
         # read kept rows of o (fp32), pos and gate; write y
         "combine": n_kept * d * 4 + T * k * 8 + T * d * s,
     }
+    if routing == "expert_choice":
+        # route: read x and W_g, write the [T, E] affinities; select + gather:
+        # read the affinities, write pos [T, E] and the token lists, copy one
+        # x row per assignment; combine: kept rows of o, pos and affinities
+        # [T, E], write y
+        byts["route"] = T * d * s + d * E * s + T * E * 4
+        byts["permute"] = 2 * T * E * 4 + n_kept * 4 + 2 * n_kept * d * s
+        byts["combine"] = n_kept * d * 4 + T * E * 8 + T * d * s
     total_flop = flop["route"] + flop["ffn_up"] + flop["ffn_down"]
     return flop, byts, total_flop
 
@@ -197,12 +211,16 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
-def oracle_sample_seconds(w, cpu_inp, T_s):
+def oracle_sample_seconds(w, cpu_inp, T_s, routing="token_choice"):
     """Run the fp64 oracle as it stands on the first T_s tokens (routing,
     capacity over that sample batch, expert FFNs, combine); wall seconds."""
     import oracle
     x = cpu_inp["x"][:T_s]
     t0 = time.perf_counter()
+    if routing == "expert_choice":
+        oracle.moe_forward_expert_choice(x, cpu_inp["Wg"], cpu_inp["bias"], cpu_inp["W1"],
+                                         cpu_inp["W3"], cpu_inp["W2"], w.k, w.cf, w.act)
+        return time.perf_counter() - t0
     logits = oracle.router_logits(x, cpu_inp["Wg"], cpu_inp["bias"])
     idx, _, _ = oracle.top_k(logits, w.k)
     C = oracle.capacity(T_s, w.E, w.k, w.cf)
@@ -236,6 +254,10 @@ def main(argv=None):
         w = w.replace(E=a.experts)
     if a.hidden:
         w = w.replace(H=a.hidden)
+    if a.capacity_factor is not None:
+        w = w.replace(cf=a.capacity_factor)
+    elif a.routing == "expert_choice" and not w.cf > 0:
+        w = w.replace(cf=1.0)
     peaks, peak_src = load_peaks()
 
     if a.impl == "reference":
@@ -250,8 +272,13 @@ def main(argv=None):
     stream = torch.cuda.current_stream(dev)
 
     inp = make_inputs(w, dev)
-    layer = M.MoELayer(inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], w.k, w.cf, w.act,
-                       max_tokens=w.T)
+    ec = a.routing == "expert_choice"
+    if ec:
+        layer = M.ExpertChoiceLayer(inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], w.k,
+                                    w.cf, w.act)
+    else:
+        layer = M.MoELayer(inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], w.k, w.cf,
+                           w.act, max_tokens=w.T)
     x = inp["x"]
     y = torch.empty_like(x)
 
@@ -260,7 +287,7 @@ def main(argv=None):
     n_kept = int(st.kept)
     pos = layer.intermediates(w.T)["pos"]
     tokens_with_kept = int((pos >= 0).any(dim=1).sum().item())
-    flop, byts, total_flop = algorithmic(w, n_kept, tokens_with_kept)
+    flop, byts, total_flop = algorithmic(w, n_kept, tokens_with_kept, a.routing)
 
     for _ in range(a.warmup):
         layer(x, y=y)
@@ -303,7 +330,7 @@ def main(argv=None):
 
     # End to end: tokens in pinned host memory, copies inside the timed call.
     e2e = None
-    if not a.no_e2e:
+    if not a.no_e2e and not ec:
         x_host = x.cpu().pin_memory()
         y_host = torch.empty_like(x_host).pin_memory()
         x_dev, y_dev = torch.empty_like(x), torch.empty_like(x)
@@ -332,7 +359,7 @@ def main(argv=None):
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu_inp = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
         T_s = a.cpu_sample or default_cpu_sample(w)
-        secs = oracle_sample_seconds(w, cpu_inp, T_s)
+        secs = oracle_sample_seconds(w, cpu_inp, T_s, a.routing)
         cpu = {"value": T_s / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"first {T_s} tokens of the {w.name} batch (routing, capacity, expert "
                          f"FFNs, combine in fp64 NumPy), {secs:.1f} s"}
@@ -352,7 +379,8 @@ def main(argv=None):
     roof_peak = peaks["bf16_tflops_sustained"]
     achieved = flop["ffn_up"] / (up_ms / 1e3) / 1e12 if up_ms > 0 else None
     roofline = {
-        "kernel": "ffn_tc_kernel<SwiGLU> (grouped up projection)",
+        "kernel": "ffn_tc_kernel<%s> (grouped up projection)" % (
+            "SwiGLU" if w.act == "swiglu" else "GELU"),
         "bound": "tensor", "achieved": round(achieved, 2) if achieved else None,
         "peak": roof_peak, "unit": "TFLOP/s",
         "frac": round(achieved / roof_peak, 4) if achieved else None,
@@ -368,7 +396,8 @@ def main(argv=None):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded; random-init weights)",
             "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "H": w.H,
-                       "act": w.act, "capacity_factor": w.cf, "parallelism": f"replicas x{world}",
+                       "act": w.act, "capacity_factor": w.cf, "routing": a.routing,
+                       "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (expert weights "
                              f"{(3 if w.act == 'swiglu' else 2) * w.E * w.d * w.H * (2 if w.dtype == 'bf16' else 4) / 1e9:.2f} GB"
                              " stream from HBM every step)"},

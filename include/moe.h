@@ -144,6 +144,10 @@ int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double capacity_factor);
  * Returns -1 on invalid sizes. */
 int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double capacity_factor);
 
+/* The same bound for an explicit capacity C (C < 0: dropless), e.g. one
+ * shard of a batch under the whole batch's capacity (moe_permute_ex). */
+int64_t moe_rows_for_capacity(int32_t T, int32_t E, int32_t k, int32_t C);
+
 /* Scratch bytes moe_permute needs in `ws` (per-block counts and a counter). */
 size_t moe_permute_workspace_bytes(int32_t T, int32_t E);
 
@@ -195,15 +199,35 @@ moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d,
                        int32_t* kept_counts, int32_t* offsets,
                        void* ws, size_t ws_bytes, void* stream);
 
-/* moe_permute serving the expert queues in a given order: queue position i
- * is token order[i] (a permutation of 0..T-1, e.g. from moe_priority_order);
- * order == NULL is token position, i.e. moe_permute.  Rows inside an expert
- * block follow the queue order.  ws as for moe_permute. */
-moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order, int32_t T,
-                          int32_t d, int32_t E, int32_t k, double capacity_factor,
-                          moe_dtype dtype, void* xp, int64_t xp_rows, int32_t* pos,
-                          int32_t* counts, int32_t* kept_counts, int32_t* offsets,
+/* moe_permute with an explicit capacity, a queue order and earlier shards.
+ *   order: queue position i is token order[i] (a permutation of 0..T-1,
+ *     e.g. from moe_priority_order); NULL = token position.  Rows inside an
+ *     expert block follow the queue order.
+ *   prior: device int32 [E] or NULL -- assignments that earlier shards of
+ *     the same batch (tokens at lower positions, held by other ranks) routed
+ *     to each expert; this shard keeps at most max(0, capacity - prior[e])
+ *     at expert e, so a batch split over ranks drops exactly what the whole
+ *     batch would ("Drop-towards-the-End" over global position).
+ *   capacity: C (e.g. moe_capacity of the whole batch), or < 0 = dropless.
+ *   xp_rows >= rows for this T (moe_max_permuted_rows with the same C);
+ *   ws as for moe_permute. */
+moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order,
+                          const int32_t* prior, int32_t T, int32_t d, int32_t E, int32_t k,
+                          int32_t capacity, moe_dtype dtype, void* xp, int64_t xp_rows,
+                          int32_t* pos, int32_t* counts, int32_t* kept_counts, int32_t* offsets,
                           void* ws, size_t ws_bytes, void* stream);
+
+/* Per-expert assignment counts of idx [T, k] into counts [E] (device), for
+ * exchanging between ranks that hold shards of one batch (int32 sums:
+ * deterministic). */
+moe_status moe_expert_counts(const int32_t* idx, int32_t T, int32_t E, int32_t k, int32_t* counts,
+                             void* stream);
+
+/* prior[e] = sum of gathered[r][e] over ranks r < rank: the assignments the
+ * lower-position shards routed to expert e.  gathered: device int32
+ * [n_ranks][E] (the all-gathered moe_expert_counts); prior: device [E]. */
+moe_status moe_rank_prefix(const int32_t* gathered, int32_t n_ranks, int32_t E, int32_t rank,
+                           int32_t* prior, void* stream);
 
 /* Batch Priority Routing order ("Scaling Vision with Sparse Mixture of
  * Experts", "Priority Routing"): order[T] = the tokens sorted by descending
@@ -221,7 +245,7 @@ moe_status moe_priority_order(const float* gate, int32_t T, int32_t k, int32_t* 
  * plugin that its host framework forbids from allocating inside its execute
  * call.  Arguments and results are those of moe_permute, minus ws/ws_bytes.
  *   Scratch: a fixed array of MOE_PERMUTE_STATIC_MAX_INTS int32 (1 MiB) plus
- *   256 bytes, held by every GPU that loads the library until the process
+ *   512 bytes, held by every GPU that loads the library until the process
  *   exits.  A call with ceil(T / 256) * E > MOE_PERMUTE_STATIC_MAX_INTS
  *   (at E = 64: T > 1,048,576) returns MOE_ERR_ARG and enqueues nothing.
  *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
@@ -306,6 +330,91 @@ moe_status moe_forward_host(const void* x_host, void* y_host, void* x_dev, void*
  * themselves stay owned by the caller and must outlive those calls. */
 #define MOE_NUM_STAGE_EVENTS 6
 moe_status moe_set_stage_events(void* const* events);
+
+/* ------------------------------------------------- expert-choice routing
+ * "[Paper Club] Upcycling Large Language Models into Mixture of Experts",
+ * the Q&A on expert choice: the selection is reversed -- every expert takes
+ * a fixed number of tokens, so a token may be processed by no expert, by
+ * several, or by all.  Here the affinity of token t to expert e is the
+ * router probability S[t, e] = Softmax(x_t . W_g (+ bias))_e over all E
+ * experts ("How do Mixture of Expert Models Work?", "The Math Behind MoEs");
+ * expert e takes the n = min(C, T) tokens with the largest S[:, e]
+ * (C = moe_capacity(T, E, k, cf), k read as the average number of experts
+ * per token; equal affinities -> lower position first), and
+ *   y_t = sum over the experts e that took t, ascending e, of S[t, e] * E_e(x_t)
+ * with no renormalisation (a token no expert took gets y_t = 0).
+ * Expert e's rows in xp/h/o are [e * npad, e * npad + n), its tokens in
+ * ascending position; npad = n rounded up to 128. */
+
+/* n = min(T, moe_capacity(T, E, k, cf)); -1 when cf is not a finite
+ * positive number (expert choice has no dropless form) or sizes are invalid. */
+int32_t moe_expert_choice_tokens(int32_t T, int32_t E, int32_t k, double capacity_factor);
+
+/* scores [T, E] fp32 (device) = softmax over all E logits of every token.
+ * Sizes as moe_route (no k). */
+moe_status moe_expert_choice_route(const void* x, const void* Wg, const float* bias, int32_t T,
+                                   int32_t d, int32_t E, moe_dtype dtype, float* scores,
+                                   void* stream);
+
+/* Scratch bytes for moe_expert_choice_select (a transposed key copy, T*E*4). */
+size_t moe_expert_choice_select_workspace_bytes(int32_t T, int32_t E);
+
+/* Each expert's choice of n tokens (0 <= n <= T).  Outputs (device):
+ * tok [E, n] int32 (expert e's tokens, ascending position), pos [T, E]
+ * int32 (row in xp, or -1), kept_counts [E] (= n), offsets [E + 1]
+ * (= e * npad).  Deterministic: the selection and the row order follow
+ * from the scores alone. */
+moe_status moe_expert_choice_select(const float* scores, int32_t T, int32_t E, int32_t n,
+                                    int32_t* tok, int32_t* pos, int32_t* kept_counts,
+                                    int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
+
+/* xp row e * npad + r = x[tok[e, r]] for r < n (padding rows untouched);
+ * xp_rows >= E * npad. */
+moe_status moe_expert_choice_gather(const void* x, const int32_t* tok, int32_t T, int32_t d,
+                                    int32_t E, int32_t n, moe_dtype dtype, void* xp,
+                                    int64_t xp_rows, void* stream);
+
+/* y [T, d] (dtype) = sum over e with pos[t, e] >= 0, ascending e, of
+ * scores[t, e] * o[pos[t, e]] (o fp32 from moe_grouped_ffn), fp32
+ * accumulation, one rounding.  Every y row is written. */
+moe_status moe_expert_choice_combine(const float* o, const int32_t* pos, const float* scores,
+                                     int32_t T, int32_t d, int32_t E, moe_dtype dtype, void* y,
+                                     void* stream);
+
+/* Byte offsets inside the moe_forward_expert_choice workspace. */
+typedef struct {
+  size_t scores;       /* fp32  [T, E]  affinities                         */
+  size_t pos;          /* int32 [T, E]  row in xp/h/o, or -1               */
+  size_t tok;          /* int32 [E, n]  each expert's tokens               */
+  size_t kept_counts;  /* int32 [E]     (= n)                              */
+  size_t offsets;      /* int32 [E + 1] (= e * npad)                       */
+  size_t dev_error;    /* int32 [1]     device error word                  */
+  size_t scratch;      /* select scratch                                   */
+  size_t xp, h, o;     /* rows x d (dtype), rows x H (dtype), rows x d fp32 */
+  size_t total;
+  int64_t rows;        /* E * npad                                         */
+  int32_t n;           /* tokens per expert                                */
+} moe_ec_ws_layout;
+
+moe_status moe_expert_choice_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                    double capacity_factor, moe_dtype dtype, moe_act act,
+                                    moe_ec_ws_layout* layout);
+/* 0 on invalid sizes (including a capacity factor that is not finite and > 0). */
+size_t moe_expert_choice_workspace_bytes(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                         double capacity_factor, moe_dtype dtype, moe_act act);
+
+/* The whole layer with expert-choice routing: route (affinities) ->
+ * select -> gather -> grouped expert FFNs (as moe_grouped_ffn) -> combine,
+ * on one stream.  Arguments as moe_forward; k <= E (no kMaxK limit: a token
+ * may be taken by any number of experts).  stats (nullable): counts =
+ * kept_counts = n per expert; when given, the call waits for the stream and
+ * returns MOE_ERR_DEVICE if a kernel reported an error. */
+moe_status moe_forward_expert_choice(const void* x, const void* Wg, const float* bias,
+                                     const void* W1, const void* W3, const void* W2, int32_t T,
+                                     int32_t d, int32_t H, int32_t E, int32_t k,
+                                     double capacity_factor, moe_act act, moe_dtype dtype,
+                                     void* y, void* ws, size_t ws_bytes, moe_stats* stats,
+                                     void* stream);
 
 #ifdef __cplusplus
 }

@@ -52,27 +52,31 @@ namespace {
 
 constexpr int TM = 128;  // tile rows held by one CTA (UMMA M per CTA)
 constexpr int TN = 256;  // accumulator columns (UMMA N)
-constexpr int TK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int A_BYTES = TM * TK * 2;      // 16 KB
-constexpr int B_BOX_BYTES = 64 * TK * 2;  // one 64-column x 64-row box: 8 KB
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * TN;
 constexpr int CONTROL_BYTES = 1536;
 #ifndef MOE_PAIR_STAGES
-#define MOE_PAIR_STAGES 6  // ring depth of the CTA-pair kernel (7 fills 227 KB)
+#define MOE_PAIR_STAGES 6  // ring depth of the CTA-pair kernel with 64-wide K steps
 #endif
-// One CTA per tile (CG = 1): each CTA holds all 256 B columns.  A CTA pair
-// (CG = 2): each CTA holds half of them, so a stage is 32 KB and the ring
-// gets 6 stages in the same shared memory.
-template <int CG>
+// Shared-memory ring per K step of TKS elements (64 or 128):
+//   A: 128 rows, stored as TKS/64 chunks of [128 rows][64] (16 KB each);
+//   B: 4/CG chunks of 64 columns, each [TKS rows][64] (8 or 16 KB).
+// One CTA per tile (CG = 1) holds all 256 B columns; a CTA pair (CG = 2)
+// holds half of them per CTA.  The pair kernel with 128-wide steps has three
+// 64 KB stages; with 64-wide steps six 32 KB stages; one CTA, four 48 KB.
+template <int CG, int TKS>
 struct Cfg {
-  static constexpr int B_BOXES = 4 / CG;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BOXES * B_BOX_BYTES;
-  static constexpr int STAGES = CG == 1 ? 4 : MOE_PAIR_STAGES;
+  static constexpr int A_STAGE = TM * TKS * 2;
+  static constexpr int A_CHUNK = TM * 64 * 2;
+  static constexpr int B_CHUNK = 64 * TKS * 2;
+  static constexpr int B_CHUNKS = 4 / CG;
+  static constexpr int STAGE_BYTES = A_STAGE + B_CHUNKS * B_CHUNK;
+  static constexpr int STAGES = CG == 1 ? 4 : (TKS == 64 ? MOE_PAIR_STAGES : 3);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CONTROL_BYTES + 1024;
   static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
 };
 constexpr int MAX_STAGES = 8;
+constexpr int B_BOX_BYTES = 64 * 64 * 2;  // a 64 x 64 box (3-D fallback loads, TKS = 64)
 
 enum Epi { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_PLAIN_F32 = 2 };
 
@@ -130,13 +134,16 @@ __device__ __forceinline__ float gelu_f(float z) {
 // CTA's 128 accumulator rows into that CTA's tensor memory.  Stage-full and
 // accumulator-empty barriers live in the leader; stage-empty and
 // accumulator-full barriers in each CTA (the leader's commits reach both).
-template <int EPI, int CG>
+template <int EPI, int CG, int TKS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                   const __grid_constant__ CUtensorMap tmB1, const TcParams p) {
-  using C_ = Cfg<CG>;
+  using C_ = Cfg<CG, TKS>;
   constexpr int STAGES = C_::STAGES;
   constexpr int STAGE_BYTES = C_::STAGE_BYTES;
+  constexpr int A_STAGE = C_::A_STAGE;
+  constexpr int B_CHUNK = C_::B_CHUNK;
+  static_assert(TKS == 64 || CG == 2, "128-wide K steps only for CTA pairs");
   constexpr int TILE_M = TM * CG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -224,87 +231,79 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = c.tmem_base;
   const int total = c.total_tiles;
-  const int nk = (p.K + TK - 1) / TK;
+  const int nk = (p.K + TKS - 1) / TKS;
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t full0 = smem_u32(&c.full[0]);    // barriers of stage s are 8 bytes apart
+  const uint32_t empty0 = smem_u32(&c.empty[0]);
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int stage = 0;
+      int stage = 0, nissued = 0;
       uint32_t phase = 0;
-      int issued[STAGES];
-#pragma unroll
-      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
       bool ok = true, timed_out = false;
       for (int t = group; t < total && ok; t += ngroups) {
+        if (c.abort_flag) {
+          ok = false;
+          break;
+        }
         int e, m, n;
         decode_tile(c, t, e, m, n);
         const int row0 = c.off[e] + m * TILE_M + static_cast<int>(rank) * TM;
+        // First 64-column chunk of this CTA's B columns (4-D weight maps).
+        const int c0 = CG == 2 ? (EPI == EPI_SWIGLU ? n * 2 : n * 4 + 2 * static_cast<int>(rank))
+                               : (EPI == EPI_SWIGLU ? n * 2 : n * 4);
+        const CUtensorMap* mb = (CG == 2 && EPI == EPI_SWIGLU && !leader) ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&c.empty[stage]), phase ^ 1)) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
             ok = false;
             timed_out = true;
             break;
           }
-          if (c.abort_flag) {
-            ok = false;
-            break;
-          }
-          const uint32_t full_local = smem_u32(&c.full[stage]);
-          const uint32_t a_dst = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t b_dst = a_dst + A_BYTES;
-          if (CG == 1 && p.b_chunked) {
+          const uint32_t full_local = full0 + 8 * stage;
+          const uint32_t a_dst = smem_base + stage * STAGE_BYTES;
+          const uint32_t b_dst = a_dst + A_STAGE;
+          const int k0 = kb * TKS;
+          if (CG == 1) {
             mbar_arrive_expect_tx(full_local, STAGE_BYTES);
-            tma_load_2d(a_dst, &tmA, full_local, kb * TK, row0);
-            if (EPI == EPI_SWIGLU) {
-              const int c0 = n * (TN / 2) / 64;  // W1 then W3, two 64-column chunks each
-              tma_load_4d(b_dst, &tmB0, full_local, 0, kb * TK, c0, e);
-              tma_load_4d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_local, 0, kb * TK, c0, e);
-            } else {
-              tma_load_4d(b_dst, &tmB0, full_local, 0, kb * TK, n * TN / 64, e);
-            }
-          } else if (CG == 1) {
-            mbar_arrive_expect_tx(full_local, STAGE_BYTES);
-            tma_load_2d(a_dst, &tmA, full_local, kb * TK, row0);
-            if (EPI == EPI_SWIGLU) {
+            tma_load_2d(a_dst, &tmA, full_local, k0, row0);
+            if (p.b_chunked) {
+              tma_load_4d(b_dst, &tmB0, full_local, 0, k0, c0, e);
+              if (EPI == EPI_SWIGLU)  // W1 chunks, then the same chunks of W3
+                tma_load_4d(b_dst + 2 * B_CHUNK, &tmB1, full_local, 0, k0, c0, e);
+            } else if (EPI == EPI_SWIGLU) {
               const int n0 = n * (TN / 2);
-              tma_load_3d(b_dst + 0 * B_BOX_BYTES, &tmB0, full_local, n0, kb * TK, e);
-              tma_load_3d(b_dst + 1 * B_BOX_BYTES, &tmB0, full_local, n0 + 64, kb * TK, e);
-              tma_load_3d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_local, n0, kb * TK, e);
-              tma_load_3d(b_dst + 3 * B_BOX_BYTES, &tmB1, full_local, n0 + 64, kb * TK, e);
+              tma_load_3d(b_dst + 0 * B_BOX_BYTES, &tmB0, full_local, n0, k0, e);
+              tma_load_3d(b_dst + 1 * B_BOX_BYTES, &tmB0, full_local, n0 + 64, k0, e);
+              tma_load_3d(b_dst + 2 * B_BOX_BYTES, &tmB1, full_local, n0, k0, e);
+              tma_load_3d(b_dst + 3 * B_BOX_BYTES, &tmB1, full_local, n0 + 64, k0, e);
             } else {
               const int n0 = n * TN;
 #pragma unroll
               for (int q = 0; q < 4; ++q)
-                tma_load_3d(b_dst + q * B_BOX_BYTES, &tmB0, full_local, n0 + 64 * q, kb * TK, e);
+                tma_load_3d(b_dst + q * B_BOX_BYTES, &tmB0, full_local, n0 + 64 * q, k0, e);
             }
           } else {
             // Both CTAs' bytes complete on the leader's full barrier, which
             // the leader arms for the whole pair.
             const uint32_t full_leader = mapa_shared(full_local, 0);
             if (leader) mbar_arrive_expect_tx(full_local, CG * STAGE_BYTES);
-            tma_load_2d_pair(a_dst, &tmA, full_leader, kb * TK, row0);
+            if (TKS == 128)  // two 64-wide K chunks of A in one 3-D box
+              tma_load_3d_pair(a_dst, &tmA, full_leader, 0, row0, kb * 2);
+            else
+              tma_load_2d_pair(a_dst, &tmA, full_leader, k0, row0);
             if (p.b_chunked) {
-              // leader: W1 columns (gate half), peer: W3 columns (up half) for
-              // SwiGLU; otherwise the two halves of the 256 columns
-              const CUtensorMap* mb = (EPI == EPI_SWIGLU && !leader) ? &tmB1 : &tmB0;
-              const int c0 = EPI == EPI_SWIGLU ? n * (TN / 2) / 64
-                                               : (n * TN + static_cast<int>(rank) * (TN / 2)) / 64;
-              tma_load_4d_pair(b_dst, mb, full_leader, 0, kb * TK, c0, e);
-            } else if (EPI == EPI_SWIGLU) {
-              // leader: W1 columns (gate half); peer: W3 columns (up half)
-              const CUtensorMap* mb = leader ? &tmB0 : &tmB1;
-              const int n0 = n * (TN / 2);
-              tma_load_3d_pair(b_dst, mb, full_leader, n0, kb * TK, e);
-              tma_load_3d_pair(b_dst + B_BOX_BYTES, mb, full_leader, n0 + 64, kb * TK, e);
+              // SwiGLU: leader loads W1 columns (gate half), peer the same
+              // columns of W3 (up half); otherwise the two column halves.
+              tma_load_4d_pair(b_dst, mb, full_leader, 0, k0, c0, e);
             } else {
-              const int n0 = n * TN + static_cast<int>(rank) * (TN / 2);
-              tma_load_3d_pair(b_dst, &tmB0, full_leader, n0, kb * TK, e);
-              tma_load_3d_pair(b_dst + B_BOX_BYTES, &tmB0, full_leader, n0 + 64, kb * TK, e);
+              const int n0 = EPI == EPI_SWIGLU ? n * (TN / 2)
+                                               : n * TN + static_cast<int>(rank) * (TN / 2);
+              tma_load_3d_pair(b_dst, mb, full_leader, n0, k0, e);
+              tma_load_3d_pair(b_dst + B_BOX_BYTES, mb, full_leader, n0 + 64, k0, e);
             }
           }
-#pragma unroll
-          for (int s = 0; s < STAGES; ++s)
-            if (s == stage) ++issued[s];
+          ++nissued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -315,7 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // Tail: wait until the MMA has released every stage, so no
         // tcgen05.commit arrival is still in flight when the CTA exits.
         for (int i = 0; i < STAGES; ++i) {
-          if (!mbar_wait(smem_u32(&c.empty[stage]), phase ^ 1)) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
             timed_out = true;
             break;
           }
@@ -328,11 +327,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok || timed_out) {
         if (timed_out) atomicOr(p.err, kErrTimeoutProducer);
         c.abort_flag = 1;
-        // Let every issued copy land before the shared memory goes away.
+        // Let every issued copy land before the shared memory goes away:
+        // stage s was filled (nissued - 1 - s) / STAGES + 1 times.
         if (CG == 1 || leader) {
-          for (int s = 0; s < STAGES; ++s) {
-            if (issued[s] > 0 &&
-                !mbar_wait(smem_u32(&c.full[s]), static_cast<uint32_t>(issued[s] - 1) & 1u))
+          for (int s = 0; s < STAGES && s < nissued; ++s) {
+            const int fills = (nissued - 1 - s) / STAGES + 1;
+            if (!mbar_wait(full0 + 8 * s, static_cast<uint32_t>(fills - 1) & 1u))
               atomicOr(p.err, kErrTimeoutDrain);
           }
         } else {
@@ -346,45 +346,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------- MMA issuer
     if (lane == 0 && leader) {
       constexpr uint32_t idesc = idesc_bf16_f32(TILE_M, TN, false, true);
+      // Descriptors of stage 0; a stage and a 16-wide K step only move the
+      // 14-bit start-address field (addresses < 256 KB never carry out of it).
+      const uint64_t adesc0 = smem_desc_sw128(smem_base, 16, 1024);
+      const uint64_t bdesc0 = smem_desc_sw128(smem_base + A_STAGE, B_CHUNK, 1024);
+      const uint32_t tfull0 = smem_u32(&c.tfull[0]);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true, timed_out = false, issued_any = false;
       for (int t = group; t < total && ok; t += ngroups) {
+        if (c.abort_flag) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait(smem_u32(&c.tempty[acc]), acc_phase ^ 1)) {
           ok = false;
           timed_out = true;
           break;
         }
         tc_fence_after();
+        issued_any = true;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * TN);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&c.full[stage]), phase)) {
+          if (!mbar_wait(full0 + 8 * stage, phase)) {
             ok = false;
             timed_out = true;
             break;
           }
-          if (c.abort_flag) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t b_base = a_base + A_BYTES;
+          const uint64_t soff = static_cast<uint64_t>((stage * STAGE_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < TK / 16; ++kk) {
-            // A: K-major, advance 16 elements (32 bytes) inside the swizzled row.
-            const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
-            // B: N-major, 64-column boxes 8 KB apart; advance 16 K-rows (2 KB).
-            const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, B_BOX_BYTES, 1024);
+          for (int kk = 0; kk < TKS / 16; ++kk) {
+            // A: K-major; 16-element steps are 32 bytes inside a 128-byte
+            // swizzled row, then the next 64-wide chunk (16 KB on).
+            const uint64_t adesc =
+                adesc0 + soff + static_cast<uint64_t>(((kk >> 2) * C_::A_CHUNK + (kk & 3) * 32) >> 4);
+            // B: N-major, 64-column chunks B_CHUNK apart; 16 K-rows = 2 KB.
+            const uint64_t bdesc = bdesc0 + soff + static_cast<uint64_t>((kk * 2048) >> 4);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
             if (CG == 2)
-              tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, accum);
             else
-              tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+              tc_mma_bf16(d_tmem, adesc, bdesc, idesc, accum);
           }
-          issued_any = true;
-          const uint32_t empty_local = smem_u32(&c.empty[stage]);
+          const uint32_t empty_local = empty0 + 8 * stage;
           if (CG == 2) {
             tc_commit_pair(empty_local);
             tc_commit_pair(mapa_shared(empty_local, 1));
@@ -397,7 +404,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         if (!ok) break;
-        const uint32_t tfull_local = smem_u32(&c.tfull[acc]);
+        const uint32_t tfull_local = tfull0 + 8 * acc;
         if (CG == 2) {
           tc_commit_pair(tfull_local);
           tc_commit_pair(mapa_shared(tfull_local, 1));
@@ -584,23 +591,38 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint6
 // in one instruction, in the same shared-memory layout as separate 3-D boxes
 // (chunk-major, 8 KB per chunk).
 bool make_map_w4d(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t N,
-                  uint32_t chunks) {
+                  uint32_t chunks, uint32_t krows) {
   auto fn = encode_fn();
   if (!fn || N % 64 != 0) return false;
   cuuint64_t dims[4] = {64, K, N / 64, E};
   cuuint64_t strides[3] = {N * 2, 128, K * N * 2};
-  cuuint32_t box[4] = {64, 64, chunks, 1};
+  cuuint32_t box[4] = {64, krows, chunks, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, int CG>
+// 3-D view {64, rows, K/64} of a bf16 activation matrix [rows, K] (K % 64 ==
+// 0): a box {64, 128, 2} loads 128 rows x two 64-wide K chunks in one
+// instruction, chunk-major.
+bool make_map_a3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+  auto fn = encode_fn();
+  if (!fn || K % 64 != 0) return false;
+  cuuint64_t dims[3] = {64, rows, K / 64};
+  cuuint64_t strides[2] = {K * 2, 128};
+  cuuint32_t box[3] = {64, TM, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, int CG, int TKS>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const TcParams& p, int groups, cudaStream_t s) {
-  constexpr int smem = Cfg<CG>::SMEM_BYTES;
-  cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI, CG>,
+  constexpr int smem = Cfg<CG, TKS>::SMEM_BYTES;
+  cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI, CG, TKS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -615,7 +637,7 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<EPI, CG>, a, b0, b1, p);
+  return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<EPI, CG, TKS>, a, b0, b1, p);
 }
 
 // CTA pairs by default; MOE_TC_CTA_PAIR=0 selects one CTA per tile.
@@ -629,14 +651,16 @@ bool use_cta_pairs() {
 
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const TcParams& p, int num_sms, int64_t tiles_max, cudaStream_t s) {
+                        const TcParams& p, int num_sms, int64_t tiles_max, bool wide_k,
+                        cudaStream_t s) {
   if (use_cta_pairs()) {
     const int groups = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>(num_sms / 2, (tiles_max + 1) / 2)));
-    return launch_one<EPI, 2>(a, b0, b1, p, groups, s);
+    return wide_k ? launch_one<EPI, 2, 128>(a, b0, b1, p, groups, s)
+                  : launch_one<EPI, 2, 64>(a, b0, b1, p, groups, s);
   }
   const int groups = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms, tiles_max)));
-  return launch_one<EPI, 1>(a, b0, b1, p, groups, s);
+  return launch_one<EPI, 1, 64>(a, b0, b1, p, groups, s);
 }
 
 }  // namespace
@@ -646,17 +670,22 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   CUtensorMap mx, mw1, mw3, mh, mw2;
   const bool swiglu = a.act == MOE_SWIGLU;
   const bool pairs = use_cta_pairs();
-  if (!make_map_2d(&mx, a.xp, a.rows, a.d, TM) || !make_map_2d(&mh, a.h, a.rows, a.H, TM))
-    return MOE_ERR_CUDA;
-  // Weights: one 4-D load per K-step and CTA when the columns come in whole
-  // 64-wide chunks; per-chunk 3-D loads otherwise.
+  // Weights: one 4-D load per K step and CTA when the columns come in whole
+  // 64-wide chunks; per-chunk 3-D loads otherwise.  CTA pairs take 128-wide
+  // K steps (one 3-D activation load + one 4-D weight load per 64 KB stage)
+  // when K is also a multiple of 64.
   const bool up_chunked = a.H % 64 == 0, dn_chunked = a.d % 64 == 0;
+  const bool up_wide = pairs && up_chunked && a.d % 64 == 0;
+  const bool dn_wide = pairs && dn_chunked && a.H % 64 == 0;
   const uint32_t up_chunks = pairs ? 2 : (swiglu ? 2 : 4), dn_chunks = pairs ? 2 : 4;
-  bool ok = up_chunked ? make_map_w4d(&mw1, a.W1, a.E, a.d, a.H, up_chunks) &&
-                             (!swiglu || make_map_w4d(&mw3, a.W3, a.E, a.d, a.H, up_chunks))
-                       : make_map_3d(&mw1, a.W1, a.E, a.d, a.H) &&
-                             (!swiglu || make_map_3d(&mw3, a.W3, a.E, a.d, a.H));
-  ok = ok && (dn_chunked ? make_map_w4d(&mw2, a.W2, a.E, a.H, a.d, dn_chunks)
+  bool ok = (up_wide ? make_map_a3d(&mx, a.xp, a.rows, a.d) : make_map_2d(&mx, a.xp, a.rows, a.d, TM)) &&
+            (dn_wide ? make_map_a3d(&mh, a.h, a.rows, a.H) : make_map_2d(&mh, a.h, a.rows, a.H, TM));
+  const uint32_t up_kr = up_wide ? 128 : 64, dn_kr = dn_wide ? 128 : 64;
+  ok = ok && (up_chunked ? make_map_w4d(&mw1, a.W1, a.E, a.d, a.H, up_chunks, up_kr) &&
+                               (!swiglu || make_map_w4d(&mw3, a.W3, a.E, a.d, a.H, up_chunks, up_kr))
+                         : make_map_3d(&mw1, a.W1, a.E, a.d, a.H) &&
+                               (!swiglu || make_map_3d(&mw3, a.W3, a.E, a.d, a.H)));
+  ok = ok && (dn_chunked ? make_map_w4d(&mw2, a.W2, a.E, a.H, a.d, dn_chunks, dn_kr)
                          : make_map_3d(&mw2, a.W2, a.E, a.H, a.d));
   if (!ok) return MOE_ERR_CUDA;
   const int64_t mtiles_max = (a.rows + TM - 1) / TM;
@@ -674,8 +703,8 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.kept = a.kept_counts;
   up.err = a.dev_error;
   cudaError_t err =
-      swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, up, num_sms, mtiles_max * up.n_tiles, s)
-             : launch_gemm<EPI_GELU>(mx, mw1, mw1, up, num_sms, mtiles_max * up.n_tiles, s);
+      swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, up, num_sms, mtiles_max * up.n_tiles, up_wide, s)
+             : launch_gemm<EPI_GELU>(mx, mw1, mw1, up, num_sms, mtiles_max * up.n_tiles, up_wide, s);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (between && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -691,7 +720,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
-  err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, dn, num_sms, mtiles_max * dn.n_tiles, s);
+  err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, dn, num_sms, mtiles_max * dn.n_tiles, dn_wide, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -29,11 +29,6 @@ bool valid_route_sizes(int32_t T, int32_t d, int32_t E, int32_t k) {
 }
 bool valid_ffn_sizes(int32_t d, int32_t H) { return d > 0 && d % 8 == 0 && H > 0 && H % 8 == 0; }
 
-int capacity_or_max(int32_t T, int32_t E, int32_t k, double cf) {
-  const int32_t C = moe_capacity(T, E, k, cf);
-  return C < 0 ? INT32_MAX : C;
-}
-
 // Stage events set by moe_set_stage_events for this host thread.
 thread_local cudaEvent_t g_stage_events[MOE_NUM_STAGE_EVENTS] = {};
 thread_local bool g_stage_events_on = false;
@@ -146,14 +141,16 @@ MOE_API int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double cf) {
   return static_cast<int32_t>(c);
 }
 
-MOE_API int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double cf) {
+MOE_API int64_t moe_rows_for_capacity(int32_t T, int32_t E, int32_t k, int32_t C) {
   if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return -1;
   if (T == 0) return 0;
-  const int64_t tk = static_cast<int64_t>(T) * k;
-  const int32_t C = moe_capacity(T, E, k, cf);
-  int64_t rows = tk + static_cast<int64_t>(E) * (kRowAlign - 1);
+  int64_t rows = static_cast<int64_t>(T) * k + static_cast<int64_t>(E) * (kRowAlign - 1);
   if (C >= 0) rows = std::min<int64_t>(rows, static_cast<int64_t>(E) * pad_rows(C));
   return pad_rows(std::max<int64_t>(rows, kRowAlign));
+}
+
+MOE_API int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double cf) {
+  return moe_rows_for_capacity(T, E, k, moe_capacity(T, E, k, cf));
 }
 
 MOE_API size_t moe_permute_workspace_bytes(int32_t T, int32_t E) {
@@ -199,17 +196,18 @@ MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, i
 }
 
 MOE_API moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order,
-                                  int32_t T, int32_t d, int32_t E, int32_t k, double cf,
-                                  moe_dtype dt, void* xp, int64_t xp_rows, int32_t* pos,
-                                  int32_t* counts, int32_t* kept_counts, int32_t* offsets,
-                                  void* ws, size_t ws_bytes, void* stream) {
+                                  const int32_t* prior, int32_t T, int32_t d, int32_t E,
+                                  int32_t k, int32_t capacity, moe_dtype dt, void* xp,
+                                  int64_t xp_rows, int32_t* pos, int32_t* counts,
+                                  int32_t* kept_counts, int32_t* offsets, void* ws,
+                                  size_t ws_bytes, void* stream) {
   if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
   if (!counts || !kept_counts || !offsets) return MOE_ERR_ARG;
   if (T > 0) {
     if (!x || !idx || !xp || !pos || !ws || !aligned16(x) || !aligned16(xp) ||
         !aligned16(ws))
       return MOE_ERR_ARG;
-    if (xp_rows < moe_max_permuted_rows(T, E, k, cf)) return MOE_ERR_ARG;
+    if (xp_rows < moe_rows_for_capacity(T, E, k, capacity)) return MOE_ERR_ARG;
     if (ws_bytes < permute_scratch_bytes(T, E)) return MOE_ERR_ARG;
   }
   DeviceInfo di;
@@ -219,8 +217,9 @@ MOE_API moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32
   int32_t* block_base = static_cast<int32_t*>(ws);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(
       static_cast<uint8_t*>(ws) + align_up(nblk * static_cast<size_t>(E) * 4));
-  PermuteArgs a{x, idx, T, d, E, k, capacity_or_max(T, E, k, cf), xp, pos, counts, kept_counts,
-                offsets, block_base, ticket, order};
+  PermuteArgs a{x,      idx,         T,       d,          E,     k,
+                capacity < 0 ? INT32_MAX : capacity, xp, pos, counts, kept_counts, offsets,
+                block_base, ticket, order, prior};
   return launch_permute(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
                                                                                  : MOE_ERR_CUDA;
 }
@@ -229,8 +228,34 @@ MOE_API moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int
                                int32_t k, double cf, moe_dtype dt, void* xp, int64_t xp_rows,
                                int32_t* pos, int32_t* counts, int32_t* kept_counts,
                                int32_t* offsets, void* ws, size_t ws_bytes, void* stream) {
-  return moe_permute_ex(x, idx, nullptr, T, d, E, k, cf, dt, xp, xp_rows, pos, counts,
-                        kept_counts, offsets, ws, ws_bytes, stream);
+  return moe_permute_ex(x, idx, nullptr, nullptr, T, d, E, k, moe_capacity(T, E, k, cf), dt, xp,
+                        xp_rows, pos, counts, kept_counts, offsets, ws, ws_bytes, stream);
+}
+
+MOE_API moe_status moe_expert_counts(const int32_t* idx, int32_t T, int32_t E, int32_t k,
+                                     int32_t* counts, void* stream) {
+  if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E || !counts) return MOE_ERR_ARG;
+  if (T > 0 && !idx) return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_expert_counts(idx, T, E, k, counts, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_rank_prefix(const int32_t* gathered, int32_t n_ranks, int32_t E,
+                                   int32_t rank, int32_t* prior, void* stream) {
+  if (n_ranks < 1 || rank < 0 || rank >= n_ranks || E < 1 || E > kMaxE || !gathered || !prior)
+    return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_rank_prefix(gathered, n_ranks, E, rank, prior, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 MOE_API size_t moe_priority_workspace_bytes(int32_t T) {
@@ -336,8 +361,9 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
     if (st != MOE_OK) return st;
     order = reinterpret_cast<const int32_t*>(w + L.order);
   }
-  st = moe_permute_ex(x, idx, order, T, d, E, k, cf, dt, w + L.xp, L.rows, pos, counts, kept,
-                      offsets, w + L.scratch, permute_scratch_bytes(T, E), s);
+  st = moe_permute_ex(x, idx, order, nullptr, T, d, E, k, moe_capacity(T, E, k, cf), dt, w + L.xp,
+                      L.rows, pos, counts, kept, offsets, w + L.scratch,
+                      permute_scratch_bytes(T, E), s);
   if (st == MOE_OK) st = record_stage(2, s);
   if (st != MOE_OK) return st;
   st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,
@@ -524,4 +550,188 @@ MOE_API moe_status moe_forward_host(const void* x_host, void* y_host, void* x_de
   st = read_device_error(Lc, ws, s, &derr);
   if (st != MOE_OK) return st;
   return derr ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+// ============================================================ expert choice
+namespace {
+
+bool ec_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, double cf, moe_dtype dt,
+               moe_act act, moe_ec_ws_layout* L) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || k < 1 || k > E ||
+      !valid_ffn_sizes(d, H) || !valid_dtype(dt) || !valid_act(act))
+    return false;
+  const int32_t n = moe_expert_choice_tokens(T, E, k, cf);
+  if (n < 0) return false;
+  const int64_t npad = pad_rows(n);
+  const int64_t rows = static_cast<int64_t>(E) * npad;
+  const size_t es = elt_size(dt);
+  const size_t te = static_cast<size_t>(T) * E;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  memset(L, 0, sizeof(*L));
+  L->scores = take(te * 4);
+  L->pos = take(te * 4);
+  L->tok = take(static_cast<size_t>(E) * n * 4);
+  L->kept_counts = take(kMaxE * 4);
+  L->offsets = take((kMaxE + 1) * 4);
+  L->dev_error = take(4);
+  L->scratch = take(ec_select_scratch_bytes(T, E));
+  L->xp = take(static_cast<size_t>(rows) * d * es);
+  L->h = take(static_cast<size_t>(rows) * H * es);
+  L->o = take(static_cast<size_t>(rows) * d * 4);
+  L->total = off;
+  L->rows = rows;
+  L->n = n;
+  return true;
+}
+
+}  // namespace
+
+MOE_API int32_t moe_expert_choice_tokens(int32_t T, int32_t E, int32_t k, double cf) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+  const int32_t C = moe_capacity(T, E, k, cf);
+  return C < 0 ? -1 : std::min(C, T);
+}
+
+MOE_API moe_status moe_expert_choice_route(const void* x, const void* Wg, const float* bias,
+                                           int32_t T, int32_t d, int32_t E, moe_dtype dt,
+                                           float* scores, void* stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || !valid_dtype(dt)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wg || !scores || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  RouteArgs a{x, Wg, bias, T, d, E, 1, nullptr, nullptr, nullptr, MOE_GATE_TOPK_SOFTMAX, 1.0f,
+              scores};
+  return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API size_t moe_expert_choice_select_workspace_bytes(int32_t T, int32_t E) {
+  if (T < 0 || E < 1 || E > kMaxE) return 0;
+  return ec_select_scratch_bytes(T, E);
+}
+
+MOE_API moe_status moe_expert_choice_select(const float* scores, int32_t T, int32_t E, int32_t n,
+                                            int32_t* tok, int32_t* pos, int32_t* kept_counts,
+                                            int32_t* offsets, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  if (T < 0 || E < 1 || E > kMaxE || n < 0 || n > T) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!scores || !pos || !kept_counts || !offsets || !ws || !aligned16(ws) ||
+      ws_bytes < ec_select_scratch_bytes(T, E) || (n > 0 && !tok))
+    return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_ec_select(scores, T, E, n, static_cast<int>(pad_rows(n)), ws, tok, pos,
+                          kept_counts, offsets, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_expert_choice_gather(const void* x, const int32_t* tok, int32_t T,
+                                            int32_t d, int32_t E, int32_t n, moe_dtype dt,
+                                            void* xp, int64_t xp_rows, void* stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || n < 0 || n > T || !valid_dtype(dt))
+    return MOE_ERR_ARG;
+  if (n == 0) return MOE_OK;
+  if (!x || !tok || !xp || !aligned16(x) || !aligned16(xp) ||
+      xp_rows < static_cast<int64_t>(E) * pad_rows(n))
+    return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_ec_gather(x, tok, E, n, static_cast<int>(pad_rows(n)), d, dt, xp,
+                          static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_expert_choice_combine(const float* o, const int32_t* pos,
+                                             const float* scores, int32_t T, int32_t d,
+                                             int32_t E, moe_dtype dt, void* y, void* stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || !valid_dtype(dt)) return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!o || !pos || !scores || !y || !aligned16(o) || !aligned16(y)) return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_ec_combine(o, pos, scores, T, d, E, dt, y, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_expert_choice_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                            double cf, moe_dtype dt, moe_act act,
+                                            moe_ec_ws_layout* layout) {
+  if (!layout) return MOE_ERR_ARG;
+  return ec_layout(T, d, H, E, k, cf, dt, act, layout) ? MOE_OK : MOE_ERR_ARG;
+}
+
+MOE_API size_t moe_expert_choice_workspace_bytes(int32_t T, int32_t d, int32_t H, int32_t E,
+                                                 int32_t k, double cf, moe_dtype dt,
+                                                 moe_act act) {
+  moe_ec_ws_layout L;
+  return ec_layout(T, d, H, E, k, cf, dt, act, &L) ? L.total : 0;
+}
+
+MOE_API moe_status moe_forward_expert_choice(const void* x, const void* Wg, const float* bias,
+                                             const void* W1, const void* W3, const void* W2,
+                                             int32_t T, int32_t d, int32_t H, int32_t E,
+                                             int32_t k, double cf, moe_act act, moe_dtype dt,
+                                             void* y, void* ws, size_t ws_bytes,
+                                             moe_stats* stats, void* stream) {
+  moe_ec_ws_layout L;
+  if (!ec_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
+  if (T > 0 && (!y || !ws || ws_bytes < L.total || !aligned16(ws))) return MOE_ERR_ARG;
+  if (stats) memset(stats, 0, sizeof(*stats));
+  if (T == 0) {
+    if (stats) stats->capacity = moe_capacity(T, E, k, cf);
+    return MOE_OK;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  float* scores = reinterpret_cast<float*>(w + L.scores);
+  int32_t* pos = reinterpret_cast<int32_t*>(w + L.pos);
+  int32_t* tok = reinterpret_cast<int32_t*>(w + L.tok);
+  int32_t* kept = reinterpret_cast<int32_t*>(w + L.kept_counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* err = reinterpret_cast<int32_t*>(w + L.dev_error);
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  moe_status st = record_stage(0, s);
+  if (st == MOE_OK) st = moe_expert_choice_route(x, Wg, bias, T, d, E, dt, scores, s);
+  if (st == MOE_OK) st = record_stage(1, s);
+  if (st == MOE_OK)
+    st = moe_expert_choice_select(scores, T, E, L.n, tok, pos, kept, offsets, w + L.scratch,
+                                  ec_select_scratch_bytes(T, E), s);
+  if (st == MOE_OK) st = moe_expert_choice_gather(x, tok, T, d, E, L.n, dt, w + L.xp, L.rows, s);
+  if (st == MOE_OK) st = record_stage(2, s);
+  if (st == MOE_OK && L.rows > 0)
+    st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,
+                         reinterpret_cast<float*>(w + L.o), err, s);
+  else if (st == MOE_OK)
+    st = record_stage(3, s);
+  if (st == MOE_OK) st = record_stage(4, s);
+  if (st == MOE_OK)
+    st = moe_expert_choice_combine(reinterpret_cast<float*>(w + L.o), pos, scores, T, d, E, dt, y,
+                                   s);
+  if (st == MOE_OK) st = record_stage(5, s);
+  if (st != MOE_OK || !stats) return st;
+  for (int e = 0; e < E; ++e) stats->counts[e] = stats->kept_counts[e] = L.n;
+  stats->assignments = static_cast<int64_t>(E) * L.n;
+  stats->kept = stats->assignments;
+  stats->capacity = moe_capacity(T, E, k, cf);
+  if (cudaMemcpyAsync(&stats->device_error, err, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return stats->device_error ? MOE_ERR_DEVICE : MOE_OK;
 }

@@ -292,6 +292,7 @@ struct RouteArgs {
   float* margin;
   int gating;        // moe_gating
   float gate_scale;  // multiplies every gate
+  float* scores = nullptr;  // non-null: write softmax over all E to [T, E] instead of TopK
 };
 cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms);
 
@@ -308,7 +309,12 @@ struct PermuteArgs {
   int32_t* block_base;  // [nblk * E] scratch
   unsigned int* ticket; // scratch counter
   const int32_t* order = nullptr;  // queue order (token at position i), or null
+  const int32_t* prior = nullptr;  // per-expert assignments of earlier shards, or null
 };
+cudaError_t launch_expert_counts(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                                 cudaStream_t s);
+cudaError_t launch_rank_prefix(const int32_t* gathered, int n_ranks, int E, int rank,
+                               int32_t* prior, cudaStream_t s);
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s);
 
@@ -316,6 +322,17 @@ size_t priority_scratch_bytes(int T);
 // Stable argsort of the tokens by descending slot-0 gate into order[T].
 cudaError_t launch_priority_order(const float* gate, int T, int k, int32_t* order, void* scratch,
                                   cudaStream_t s);
+
+// Expert-choice routing (expert_choice.cu).  n = tokens each expert takes,
+// npad = n rounded up to the 128-row block.
+size_t ec_select_scratch_bytes(int T, int E);
+cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad, void* scratch,
+                             int32_t* tok, int32_t* pos, int32_t* kept_counts, int32_t* offsets,
+                             cudaStream_t s);
+cudaError_t launch_ec_gather(const void* x, const int32_t* tok, int E, int n, int npad, int d,
+                             moe_dtype dtype, void* xp, cudaStream_t s);
+cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,
+                              int d, int E, moe_dtype dtype, void* y, cudaStream_t s);
 
 struct FfnArgs {
   const void* xp;

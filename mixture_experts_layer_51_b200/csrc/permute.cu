@@ -52,10 +52,14 @@ __device__ __forceinline__ int token_at(const int32_t* __restrict__ order, int i
   return (order && i < T) ? order[i] : i;
 }
 
+// `prior` (nullable): per expert, assignments that earlier shards of the
+// batch (lower positions, other ranks) already queued; this shard may keep
+// cap[e] = max(0, C - prior[e]) more.
 __global__ void __launch_bounds__(kPermBlock)
     permute_count_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ order, int T,
-                         int E, int k, int C, int nblk, int32_t* __restrict__ block_base,
-                         unsigned int* __restrict__ ticket, int32_t* __restrict__ counts,
+                         int E, int k, int C, const int32_t* __restrict__ prior, int nblk,
+                         int32_t* __restrict__ block_base, unsigned int* __restrict__ ticket,
+                         int32_t* __restrict__ cap, int32_t* __restrict__ counts,
                          int32_t* __restrict__ kept_counts, int32_t* __restrict__ offsets) {
   __shared__ int wcnt[kWarpsPerBlock][kMaxE];
   __shared__ int padded[kMaxE];
@@ -99,7 +103,10 @@ __global__ void __launch_bounds__(kPermBlock)
       block_base[(int64_t)b * E + tid] = run;
       run += v;
     }
-    const int kept = run < C ? run : C;
+    int ce = C;
+    if (prior && C != INT32_MAX) ce = max(0, C - prior[tid]);
+    cap[tid] = ce;
+    const int kept = run < ce ? run : ce;
     counts[tid] = run;
     kept_counts[tid] = kept;
     padded[tid] = (kept + kRowAlign - 1) / kRowAlign * kRowAlign;
@@ -124,7 +131,7 @@ template <int UNROLL>
 __global__ void __launch_bounds__(kPermBlock)
     permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
                            const int32_t* __restrict__ order, int T,
-                           int dvec, int slice_vec, int E, int k, int C,
+                           int dvec, int slice_vec, int E, int k, const int32_t* __restrict__ cap,
                            const int32_t* __restrict__ block_base,
                            const int32_t* __restrict__ offsets, int32_t* __restrict__ pos,
                            uint4* __restrict__ xp) {
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kPermBlock)
     }
     for (int j = 0; j < k; ++j) {
       int p = -1;
-      if (t < T && ej[j] >= 0 && ej[j] < E && rj[j] < C) p = offsets[ej[j]] + rj[j];
+      if (t < T && ej[j] >= 0 && ej[j] < E && rj[j] < cap[ej[j]]) p = offsets[ej[j]] + rj[j];
       if (t < T && blockIdx.y == 0) pos[(int64_t)t * k + j] = p;
       spos[lane * k + j] = p;
     }
@@ -222,7 +229,51 @@ size_t permute_scratch_bytes(int T, int E) {
   const size_t nblk = (static_cast<size_t>(T) + kPermBlock - 1) / kPermBlock;
   size_t b = nblk * static_cast<size_t>(E) * sizeof(int32_t);
   b = (b + 255) / 256 * 256;
-  return b + 256;  // + ticket counter
+  return b + 512;  // + ticket counter (256 B) + per-expert capacities (256 B)
+}
+
+namespace {
+__global__ void __launch_bounds__(kPermBlock)
+    expert_count_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                        int32_t* __restrict__ counts) {
+  __shared__ int wcnt[kMaxE];
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid < kMaxE) wcnt[tid] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kPermBlock + tid;
+  const uint64_t mask = t < T ? expert_mask(idx, t, T, k, E) : 0ull;
+  for (int e = 0; e < E; ++e) {
+    const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
+    if (lane == 0 && b) atomicAdd(&wcnt[e], __popc(b));
+  }
+  __syncthreads();
+  // Integer counts: the order the additions land in does not matter.
+  if (tid < E && wcnt[tid]) atomicAdd(&counts[tid], wcnt[tid]);
+}
+
+__global__ void rank_prefix_kernel(const int32_t* __restrict__ gathered, int n_ranks, int E,
+                                   int rank, int32_t* __restrict__ prior) {
+  const int e = threadIdx.x;
+  if (e >= E) return;
+  int s = 0;
+  for (int r = 0; r < rank && r < n_ranks; ++r) s += gathered[(int64_t)r * E + e];
+  prior[e] = s;
+}
+}  // namespace
+
+cudaError_t launch_expert_counts(const int32_t* idx, int T, int E, int k, int32_t* counts,
+                                 cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s);
+  if (err != cudaSuccess || T == 0) return err;
+  expert_count_kernel<<<(T + kPermBlock - 1) / kPermBlock, kPermBlock, 0, s>>>(idx, T, E, k,
+                                                                               counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rank_prefix(const int32_t* gathered, int n_ranks, int E, int rank,
+                               int32_t* prior, cudaStream_t s) {
+  rank_prefix_kernel<<<1, kMaxE, 0, s>>>(gathered, n_ranks, E, rank, prior);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s) {
@@ -239,9 +290,10 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
   const int dvec = a.d * elt / 16;
   cudaError_t err = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned int), s);
   if (err != cudaSuccess) return err;
-  permute_count_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.order, a.T, a.E, a.k, a.capacity, nblk,
-                                                   a.block_base, a.ticket, a.counts,
-                                                   a.kept_counts, a.offsets);
+  int32_t* cap = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a.ticket) + 256);
+  permute_count_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.order, a.T, a.E, a.k, a.capacity,
+                                                   a.prior, nblk, a.block_base, a.ticket, cap,
+                                                   a.counts, a.kept_counts, a.offsets);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   // Enough row slices for ~4 CTAs per SM; each slice a multiple of 32 vectors.
@@ -252,7 +304,7 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
   slice_vec = (slice_vec + 31) / 32 * 32;
   nslice = (dvec + slice_vec - 1) / slice_vec;
   permute_scatter_kernel<4><<<dim3(nchunk, nslice), kPermBlock, 0, s>>>(
-      static_cast<const uint4*>(a.x), a.idx, a.order, a.T, dvec, slice_vec, a.E, a.k, a.capacity,
+      static_cast<const uint4*>(a.x), a.idx, a.order, a.T, dvec, slice_vec, a.E, a.k, cap,
       a.block_base, a.offsets, a.pos, static_cast<uint4*>(a.xp));
   return cudaGetLastError();
 }

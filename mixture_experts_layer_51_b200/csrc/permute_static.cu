@@ -11,8 +11,8 @@
 // cudaMalloc, cudaFree or any allocating routine.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the
-// library holds it (MOE_PERMUTE_STATIC_MAX_INTS int32 plus a 256-byte
-// counter slot) until the process exits.  In host code its name is only a
+// library holds it (MOE_PERMUTE_STATIC_MAX_INTS int32 plus a 512-byte
+// slot for a counter and per-expert capacities) until the process exits.  In host code its name is only a
 // host-side stand-in, so its device address is looked up with
 // cudaGetSymbolAddress once per device (on the first call made with that
 // device current) and that address is what the kernels receive.
@@ -23,7 +23,7 @@
 
 namespace {
 
-constexpr int kCounterInts = 64;  // 256 bytes: the completion counter's slot
+constexpr int kCounterInts = 128;  // 512 bytes: the completion counter and per-expert capacities
 
 static __device__ __align__(256) int32_t g_permute_scratch[MOE_PERMUTE_STATIC_MAX_INTS + kCounterInts];
 

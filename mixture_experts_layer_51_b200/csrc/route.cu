@@ -147,7 +147,8 @@ __global__ void __launch_bounds__(kRouteThreads)
     route_bf16_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wg,
                       const float* __restrict__ bias, int T, int d, int E, int k,
                       int32_t* __restrict__ idx, float* __restrict__ gate,
-                      float* __restrict__ margin, int gating, float gate_scale) {
+                      float* __restrict__ margin, int gating, float gate_scale,
+                      float* __restrict__ scores) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int WS = wg_stride(NT);
   constexpr int XS = x_stride(BK);
@@ -256,15 +257,39 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
   }
   __syncthreads();
+  auto logit = [&](int r, int e) {
+    float v = lg[r * LS + e];
+#pragma unroll
+    for (int g = 1; g < KG; ++g) v += lg[(g * BM + r) * LS + e];
+    return bias ? v + bias[e] : v;
+  };
+  if (scores) {
+    // Expert-choice affinities: the softmax over all E logits of every
+    // token, written as rows of [T, E].  One thread per token finds the
+    // maximum and the denominator; then the whole CTA writes the BM x E
+    // tile in index order (coalesced), each value recomputed from the same
+    // logit and maximum, so it equals the term that entered the sum.
+    float* rowstat = lg + KG * BM * LS;  // [BM][2]: max, 1/sum
+    if (tid < BM) {
+      float m = -INFINITY;
+      for (int e = 0; e < E; ++e) m = fmaxf(m, logit(tid, e));
+      float sum = 0.f;
+      for (int e = 0; e < E; ++e) sum += expf(logit(tid, e) - m);
+      rowstat[2 * tid] = m;
+      rowstat[2 * tid + 1] = 1.f / sum;
+    }
+    __syncthreads();
+    const int nrow = min(BM, T - t0);
+    for (int i = tid; i < nrow * E; i += kRouteThreads) {
+      const int r = i / E, e = i - r * E;
+      scores[(int64_t)t0 * E + i] = expf(logit(r, e) - rowstat[2 * r]) * rowstat[2 * r + 1];
+    }
+    return;
+  }
   if (tid < BM) {
     const int t = t0 + tid;
     if (t < T) {
-      auto get = [&](int e) {
-        float v = lg[tid * LS + e];
-#pragma unroll
-        for (int g = 1; g < KG; ++g) v += lg[(g * BM + tid) * LS + e];
-        return bias ? v + bias[e] : v;
-      };
+      auto get = [&](int e) { return logit(tid, e); };
       topk_softmax_store<KM>(get, E, k, t, idx, gate, margin, gating, gate_scale);
     }
   }
@@ -276,7 +301,8 @@ __global__ void __launch_bounds__(256)
     route_fp32_kernel(const float* __restrict__ x, const float* __restrict__ Wg,
                       const float* __restrict__ bias, int T, int d, int E, int k,
                       int32_t* __restrict__ idx, float* __restrict__ gate,
-                      float* __restrict__ margin, int gating, float gate_scale) {
+                      float* __restrict__ margin, int gating, float gate_scale,
+                      float* __restrict__ scores) {
   __shared__ float lg[8][kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
@@ -305,23 +331,32 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncwarp();
-  if (lane == 0) {
-    auto get = [&](int e) { return bias ? lg[warp][e] + bias[e] : lg[warp][e]; };
-    topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
+  auto get = [&](int e) { return bias ? lg[warp][e] + bias[e] : lg[warp][e]; };
+  if (scores) {
+    // Expert-choice affinities (softmax over all E), same order of
+    // operations in every lane.
+    float m = -INFINITY;
+    for (int e = 0; e < E; ++e) m = fmaxf(m, get(e));
+    float sum = 0.f;
+    for (int e = 0; e < E; ++e) sum += expf(get(e) - m);
+    const float inv = 1.f / sum;
+    for (int e = lane; e < E; e += 32) scores[(int64_t)t * E + e] = expf(get(e) - m) * inv;
+    return;
   }
+  if (lane == 0) topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
 }
 
 template <int NT, int BM, int BK, int STAGES, int KM>
 cudaError_t launch_route_cfg(const RouteArgs& a, cudaStream_t s) {
   constexpr int smem = STAGES * stage_bytes(NT, BM, BK);
-  static_assert(BM * (NT * 8 + 1) * 4 * (4 / (BM / 16)) <= smem, "epilogue buffer");
+  static_assert(BM * (NT * 8 + 1) * 4 * (4 / (BM / 16)) + BM * 8 <= smem, "epilogue buffer");
   cudaError_t err = cudaFuncSetAttribute(route_bf16_kernel<NT, BM, BK, STAGES, KM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   const int grid = (a.T + BM - 1) / BM;
   route_bf16_kernel<NT, BM, BK, STAGES, KM><<<grid, kRouteThreads, smem, s>>>(
       static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T,
-      a.d, a.E, a.k, a.idx, a.gate, a.margin, a.gating, a.gate_scale);
+      a.d, a.E, a.k, a.idx, a.gate, a.margin, a.gating, a.gate_scale, a.scores);
   return cudaGetLastError();
 }
 
@@ -357,11 +392,12 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
     route_fp32_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(static_cast<const float*>(a.x),
                                                     static_cast<const float*>(a.Wg), a.bias, a.T,
                                                     a.d, a.E, a.k, a.idx, a.gate, a.margin,
-                                                    a.gating, a.gate_scale);
+                                                    a.gating, a.gate_scale, a.scores);
     return cudaGetLastError();
   }
-  // KM = slots of the running top list (k + 1, rounded up to 3, 5 or 9).
-  if (a.k <= 2) return launch_route_km<3>(a, s);
+  // KM = slots of the running top list (k + 1, rounded up to 3, 5 or 9);
+  // the affinity output uses no list.
+  if (a.scores || a.k <= 2) return launch_route_km<3>(a, s);
   if (a.k <= 4) return launch_route_km<5>(a, s);
   return launch_route_km<kMaxK + 1>(a, s);
 }

@@ -29,7 +29,11 @@ EXPORTED = (
     "moe_route", "moe_permute", "moe_grouped_ffn", "moe_unpermute_combine",
     "moe_forward", "moe_forward_host", "moe_set_stage_events", "moe_permute_static",
     "moe_route_ex", "moe_forward_ex", "moe_permute_ex", "moe_priority_order",
-    "moe_priority_workspace_bytes",
+    "moe_priority_workspace_bytes", "moe_rows_for_capacity", "moe_expert_counts",
+    "moe_rank_prefix", "moe_expert_choice_tokens", "moe_expert_choice_route",
+    "moe_expert_choice_select_workspace_bytes", "moe_expert_choice_select",
+    "moe_expert_choice_gather", "moe_expert_choice_combine", "moe_expert_choice_layout",
+    "moe_expert_choice_workspace_bytes", "moe_forward_expert_choice",
 )
 MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
 MOE_PRIORITY_POSITION, MOE_PRIORITY_GATE = 0, 1
@@ -82,6 +86,12 @@ class moe_ws_layout(ctypes.Structure):
         "scratch", "xp", "h", "o", "total")] + [("rows", ctypes.c_int64),
                                                  ("order", ctypes.c_size_t),
                                                  ("prio_scratch", ctypes.c_size_t)]
+
+
+class moe_ec_ws_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "scores", "pos", "tok", "kept_counts", "offsets", "dev_error", "scratch", "xp", "h", "o",
+        "total")] + [("rows", ctypes.c_int64), ("n", ctypes.c_int32)]
 
 
 _lib_handle = None
@@ -144,8 +154,37 @@ def lib():
                                  ctypes.c_int, ctypes.c_int, ctypes.POINTER(moe_options), _P, _P,
                                  _SZ, ctypes.POINTER(moe_stats), _P]
     L.moe_permute_ex.restype = ctypes.c_int
-    L.moe_permute_ex.argtypes = [_P, _P, _P, _I32, _I32, _I32, _I32, _D, ctypes.c_int, _P, _I64,
-                                 _P, _P, _P, _P, _P, _SZ, _P]
+    L.moe_permute_ex.argtypes = [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, ctypes.c_int, _P,
+                                 _I64, _P, _P, _P, _P, _P, _SZ, _P]
+    L.moe_rows_for_capacity.restype = _I64
+    L.moe_rows_for_capacity.argtypes = [_I32, _I32, _I32, _I32]
+    L.moe_expert_counts.restype = ctypes.c_int
+    L.moe_expert_counts.argtypes = [_P, _I32, _I32, _I32, _P, _P]
+    L.moe_rank_prefix.restype = ctypes.c_int
+    L.moe_rank_prefix.argtypes = [_P, _I32, _I32, _I32, _P, _P]
+    L.moe_expert_choice_tokens.restype = _I32
+    L.moe_expert_choice_tokens.argtypes = [_I32, _I32, _I32, _D]
+    L.moe_expert_choice_route.restype = ctypes.c_int
+    L.moe_expert_choice_route.argtypes = [_P, _P, _P, _I32, _I32, _I32, ctypes.c_int, _P, _P]
+    L.moe_expert_choice_select_workspace_bytes.restype = _SZ
+    L.moe_expert_choice_select_workspace_bytes.argtypes = [_I32, _I32]
+    L.moe_expert_choice_select.restype = ctypes.c_int
+    L.moe_expert_choice_select.argtypes = [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]
+    L.moe_expert_choice_gather.restype = ctypes.c_int
+    L.moe_expert_choice_gather.argtypes = [_P, _P, _I32, _I32, _I32, _I32, ctypes.c_int, _P, _I64,
+                                           _P]
+    L.moe_expert_choice_combine.restype = ctypes.c_int
+    L.moe_expert_choice_combine.argtypes = [_P, _P, _P, _I32, _I32, _I32, ctypes.c_int, _P, _P]
+    L.moe_expert_choice_layout.restype = ctypes.c_int
+    L.moe_expert_choice_layout.argtypes = [_I32, _I32, _I32, _I32, _I32, _D, ctypes.c_int,
+                                           ctypes.c_int, ctypes.POINTER(moe_ec_ws_layout)]
+    L.moe_expert_choice_workspace_bytes.restype = _SZ
+    L.moe_expert_choice_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, _I32, _D,
+                                                    ctypes.c_int, ctypes.c_int]
+    L.moe_forward_expert_choice.restype = ctypes.c_int
+    L.moe_forward_expert_choice.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                            _D, ctypes.c_int, ctypes.c_int, _P, _P, _SZ,
+                                            ctypes.POINTER(moe_stats), _P]
     L.moe_priority_workspace_bytes.restype = _SZ
     L.moe_priority_workspace_bytes.argtypes = [_I32]
     L.moe_priority_order.restype = ctypes.c_int
@@ -270,12 +309,40 @@ def moe_priority_order(gate, order=None, ws=None, stream=None):
     return order
 
 
+def moe_rows_for_capacity(T, E, k, capacity):
+    return lib().moe_rows_for_capacity(T, E, k, -1 if capacity is None else int(capacity))
+
+
+def moe_expert_counts(idx, E, counts=None, stream=None):
+    """Per-expert assignment counts of idx [T, k] (int32 [E])."""
+    T, k = idx.shape
+    dev = idx.device
+    counts = counts if counts is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    _check(lib().moe_expert_counts(_ptr(idx), T, E, k, _ptr(counts), _stream(dev, stream)),
+           "moe_expert_counts")
+    return counts
+
+
+def moe_rank_prefix(gathered, rank, prior=None, stream=None):
+    """prior[e] = sum of gathered[r, e] over r < rank (int32 [E])."""
+    n, E = gathered.shape
+    dev = gathered.device
+    prior = prior if prior is not None else torch.empty(E, dtype=torch.int32, device=dev)
+    _check(lib().moe_rank_prefix(_ptr(gathered), n, E, rank, _ptr(prior), _stream(dev, stream)),
+           "moe_rank_prefix")
+    return prior
+
+
 def moe_permute(x, idx, E, capacity_factor, xp=None, pos=None, counts=None, kept_counts=None,
-                offsets=None, ws=None, stream=None, order=None):
+                offsets=None, ws=None, stream=None, order=None, prior=None, capacity=None):
+    """Counting-sort permutation.  capacity (int, or None = from
+    capacity_factor over this T) and prior (int32 [E] of earlier shards'
+    assignments) serve a batch sharded over ranks."""
     T, d = x.shape
     k = idx.shape[1]
     dev = x.device
-    rows = moe_max_permuted_rows(T, E, k, capacity_factor)
+    C = moe_capacity(T, E, k, capacity_factor) if capacity is None else int(capacity)
+    rows = moe_rows_for_capacity(T, E, k, C)
     xp = xp if xp is not None else torch.empty((max(rows, 0), d), dtype=x.dtype, device=dev)
     pos = pos if pos is not None else torch.empty((T, k), dtype=torch.int32, device=dev)
     counts = counts if counts is not None else torch.empty(E, dtype=torch.int32, device=dev)
@@ -283,8 +350,8 @@ def moe_permute(x, idx, E, capacity_factor, xp=None, pos=None, counts=None, kept
     offsets = offsets if offsets is not None else torch.empty(E + 1, dtype=torch.int32, device=dev)
     wsb = moe_permute_workspace_bytes(T, E)
     ws = ws if ws is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
-    _check(lib().moe_permute_ex(_ptr(x), _ptr(idx), _ptr(order), T, d, E, k,
-                                _cf(capacity_factor), _dtype_code(x), _ptr(xp), xp.shape[0],
+    _check(lib().moe_permute_ex(_ptr(x), _ptr(idx), _ptr(order), _ptr(prior), T, d, E, k,
+                                C, _dtype_code(x), _ptr(xp), xp.shape[0],
                                 _ptr(pos), _ptr(counts), _ptr(kept_counts), _ptr(offsets),
                                 _ptr(ws), ws.numel(), _stream(dev, stream)), "moe_permute_ex")
     return dict(xp=xp, pos=pos, counts=counts, kept_counts=kept_counts, offsets=offsets)
@@ -432,3 +499,125 @@ class MoELayer:
                            self.act, y=y, ws=self.workspace(x.shape[0]), stats=stats,
                            stream=stream, gating=self.gating, gate_scale=self.gate_scale,
                            priority=self.priority)
+
+
+# ------------------------------------------------ expert-choice routing
+def moe_expert_choice_tokens(T, E, k, capacity_factor):
+    """Tokens each expert takes: min(T, C); -1 if the capacity factor is not
+    a finite positive number."""
+    return lib().moe_expert_choice_tokens(T, E, k, _cf(capacity_factor))
+
+
+def moe_expert_choice_route(x, Wg, bias, scores=None, stream=None):
+    """Affinities [T, E] fp32: softmax over all E logits of every token."""
+    T, d = x.shape
+    E = Wg.shape[1]
+    dev = x.device
+    scores = scores if scores is not None else torch.empty((T, E), dtype=torch.float32, device=dev)
+    _check(lib().moe_expert_choice_route(_ptr(x), _ptr(Wg), _ptr(bias), T, d, E, _dtype_code(x),
+                                         _ptr(scores), _stream(dev, stream)),
+           "moe_expert_choice_route")
+    return scores
+
+
+def moe_expert_choice_select(scores, n, stream=None):
+    """Each expert's n tokens: tok [E, n], pos [T, E], kept_counts, offsets."""
+    T, E = scores.shape
+    dev = scores.device
+    tok = torch.empty((E, max(n, 0)), dtype=torch.int32, device=dev)
+    pos = torch.empty((T, E), dtype=torch.int32, device=dev)
+    kept_counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    wsb = lib().moe_expert_choice_select_workspace_bytes(T, E)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    _check(lib().moe_expert_choice_select(_ptr(scores), T, E, n, _ptr(tok), _ptr(pos),
+                                          _ptr(kept_counts), _ptr(offsets), _ptr(ws), ws.numel(),
+                                          _stream(dev, stream)), "moe_expert_choice_select")
+    return dict(tok=tok, pos=pos, kept_counts=kept_counts, offsets=offsets)
+
+
+def moe_expert_choice_gather(x, tok, xp=None, stream=None):
+    T, d = x.shape
+    E, n = tok.shape
+    npad = (n + MOE_ROW_ALIGN - 1) // MOE_ROW_ALIGN * MOE_ROW_ALIGN
+    xp = xp if xp is not None else torch.empty((E * npad, d), dtype=x.dtype, device=x.device)
+    _check(lib().moe_expert_choice_gather(_ptr(x), _ptr(tok), T, d, E, n, _dtype_code(x),
+                                          _ptr(xp), xp.shape[0], _stream(x.device, stream)),
+           "moe_expert_choice_gather")
+    return xp
+
+
+def moe_expert_choice_combine(o, pos, scores, dtype, y=None, stream=None):
+    T, E = pos.shape
+    d = o.shape[1]
+    y = y if y is not None else torch.empty((T, d), dtype=dtype, device=o.device)
+    code = MOE_BF16 if dtype == torch.bfloat16 else MOE_FP32
+    _check(lib().moe_expert_choice_combine(_ptr(o), _ptr(pos), _ptr(scores), T, d, E, code,
+                                           _ptr(y), _stream(o.device, stream)),
+           "moe_expert_choice_combine")
+    return y
+
+
+def moe_expert_choice_layout(T, d, H, E, k, capacity_factor, dtype, act):
+    code = MOE_BF16 if dtype in (torch.bfloat16, "bf16") else MOE_FP32
+    L = moe_ec_ws_layout()
+    _check(lib().moe_expert_choice_layout(T, d, H, E, k, _cf(capacity_factor), code,
+                                          _act_code(act), ctypes.byref(L)),
+           "moe_expert_choice_layout")
+    return L
+
+
+class ExpertChoiceLayer:
+    """An MoE layer with expert-choice routing: every expert takes the
+    min(T, ceil(cf*T*k/E)) tokens with the highest softmax affinity to it.
+    Holds its workspace; __call__ runs moe_forward_expert_choice."""
+
+    def __init__(self, Wg, bias, W1, W3, W2, k, capacity_factor, act="swiglu"):
+        self.Wg, self.bias, self.W1, self.W3, self.W2 = Wg, bias, W1, W3, W2
+        self.k, self.cf, self.act = k, capacity_factor, act
+        self.E, self.d, self.H = W1.shape
+        self.dtype = W1.dtype
+        self.device = W1.device
+        self._ws = None
+        self._ws_T = -1
+
+    def layout(self, T):
+        return moe_expert_choice_layout(T, self.d, self.H, self.E, self.k, self.cf, self.dtype,
+                                        self.act)
+
+    def workspace(self, T):
+        if self._ws_T != T:
+            need = self.layout(T).total
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+            self._ws_T = T
+        return self._ws
+
+    def intermediates(self, T):
+        """Views of scores, pos, tok, kept_counts, offsets, dev_error, xp."""
+        L = self.layout(T)
+        ws = self._ws
+
+        def view(off, count, dt):
+            nbytes = count * torch.empty((), dtype=dt).element_size()
+            return ws[off:off + nbytes].view(dt)
+        return dict(
+            scores=view(L.scores, T * self.E, torch.float32).view(T, self.E),
+            pos=view(L.pos, T * self.E, torch.int32).view(T, self.E),
+            tok=view(L.tok, self.E * L.n, torch.int32).view(self.E, L.n),
+            kept_counts=view(L.kept_counts, self.E, torch.int32),
+            offsets=view(L.offsets, self.E + 1, torch.int32),
+            dev_error=view(L.dev_error, 1, torch.int32),
+            xp=view(L.xp, L.rows * self.d, self.dtype).view(L.rows, self.d),
+            n=L.n, rows=L.rows)
+
+    def __call__(self, x, y=None, stats=False, stream=None):
+        T, d = x.shape
+        ws = self.workspace(T)
+        y = y if y is not None else torch.empty((T, d), dtype=x.dtype, device=x.device)
+        st = moe_stats() if stats else None
+        _check(lib().moe_forward_expert_choice(
+            _ptr(x), _ptr(self.Wg), _ptr(self.bias), _ptr(self.W1), _ptr(self.W3), _ptr(self.W2),
+            T, d, self.H, self.E, self.k, _cf(self.cf), _act_code(self.act), _dtype_code(x),
+            _ptr(y), _ptr(ws), ws.numel(), ctypes.byref(st) if st is not None else None,
+            _stream(x.device, stream)), "moe_forward_expert_choice")
+        return (y, st) if stats else y

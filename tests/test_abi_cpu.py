@@ -149,3 +149,70 @@ def test_invalid_options_are_rejected(lib):
     bad.reserved[3] = 1
     assert lib.moe_route_ex(fake, fake, None, 16, 64, 8, 2, M.MOE_BF16, ctypes.byref(bad),
                             fake, fake, None, None) == M.MOE_ERR_ARG
+
+
+@pytest.mark.parametrize("T,E,k,cf,bounds", [(1000, 8, 2, 1.0, (0, 400, 1000)),
+                                              (600, 32, 2, 1.0, (0, 1, 300, 600)),
+                                              (513, 64, 8, 0.5, (0, 100, 513))])
+def test_rows_for_capacity_bounds_every_shard(lib, T, E, k, cf, bounds):
+    """A shard under the whole batch's capacity never needs more rows than
+    moe_rows_for_capacity(shard T, E, k, C) (kept counts from the oracle's
+    shard rule, on a skewed routing)."""
+    import numpy as np
+    C = M.moe_capacity(T, E, k, cf)
+    assert M.moe_rows_for_capacity(T, E, k, C) == M.moe_max_permuted_rows(T, E, k, cf)
+    idx = np.tile(np.arange(k), (T, 1))
+    idx[::3] = (idx[::3] + 1) % E
+    prior = np.zeros(E, dtype=np.int64)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        _, kc, _, _ = oracle.assign_capacity_shard(idx[a:b], E, C, prior)
+        need = int(sum(-(-int(c) // 128) * 128 for c in kc))
+        assert need <= M.moe_rows_for_capacity(b - a, E, k, C)
+        prior = prior + np.bincount(idx[a:b].reshape(-1), minlength=E)
+
+
+def test_shard_entry_points_validate_arguments(lib):
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.moe_expert_counts(fake, 16, 65, 2, fake, None) == M.MOE_ERR_ARG   # E > 64
+    assert lib.moe_expert_counts(fake, 16, 8, 9, fake, None) == M.MOE_ERR_ARG    # k > E
+    assert lib.moe_expert_counts(None, 16, 8, 2, fake, None) == M.MOE_ERR_ARG    # no idx
+    assert lib.moe_rank_prefix(fake, 2, 8, 2, fake, None) == M.MOE_ERR_ARG       # rank >= n
+    assert lib.moe_rank_prefix(fake, 0, 8, 0, fake, None) == M.MOE_ERR_ARG       # no ranks
+    assert lib.moe_rank_prefix(None, 2, 8, 0, fake, None) == M.MOE_ERR_ARG
+    # xp smaller than the shard's bound under the given capacity
+    rows = M.moe_rows_for_capacity(64, 8, 2, 10)
+    assert lib.moe_permute_ex(fake, fake, None, fake, 64, 64, 8, 2, 10, M.MOE_BF16, fake,
+                              rows - 128, fake, fake, fake, fake, fake, 1 << 20,
+                              None) == M.MOE_ERR_ARG
+
+
+def test_expert_choice_sizes_and_validation(lib):
+    import math
+    assert M.moe_expert_choice_tokens(16384, 64, 8, 1.0) == 2048
+    assert M.moe_expert_choice_tokens(100, 4, 2, 8.0) == 100        # capped at T
+    assert M.moe_expert_choice_tokens(100, 4, 2, 0.0) == -1         # no dropless form
+    assert M.moe_expert_choice_tokens(100, 4, 2, math.inf) == -1
+    assert M.moe_expert_choice_tokens(100, 4, 5, 1.0) == -1         # k > E
+    L = M.moe_expert_choice_layout(700, 256, 384, 64, 8, 1.0, "bf16", "swiglu")
+    assert L.n == 88 and L.rows == 64 * 128
+    offs = [L.scores, L.pos, L.tok, L.kept_counts, L.offsets, L.dev_error, L.scratch, L.xp, L.h,
+            L.o]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert L.total >= L.o + L.rows * 256 * 4
+    assert lib.moe_expert_choice_workspace_bytes(700, 256, 384, 64, 8, 1.0, M.MOE_BF16,
+                                                 M.MOE_SWIGLU) == L.total
+    assert lib.moe_expert_choice_workspace_bytes(700, 256, 384, 64, 8, 0.0, M.MOE_BF16,
+                                                 M.MOE_SWIGLU) == 0
+    fake = ctypes.c_void_p(0x10000)
+    # n > T, E > 64, misaligned x, xp too small, workspace too small
+    assert lib.moe_expert_choice_select(fake, 10, 4, 11, fake, fake, fake, fake, fake, 1 << 20,
+                                        None) == M.MOE_ERR_ARG
+    assert lib.moe_expert_choice_route(fake, fake, None, 10, 64, 65, M.MOE_BF16, fake,
+                                       None) == M.MOE_ERR_ARG
+    assert lib.moe_expert_choice_gather(ctypes.c_void_p(0x10004), fake, 10, 64, 4, 3, M.MOE_BF16,
+                                        fake, 512, None) == M.MOE_ERR_ARG
+    assert lib.moe_expert_choice_gather(fake, fake, 10, 64, 4, 3, M.MOE_BF16, fake, 384,
+                                        None) == M.MOE_ERR_ARG
+    assert lib.moe_forward_expert_choice(fake, fake, None, fake, fake, fake, 64, 64, 64, 8, 2,
+                                         1.0, M.MOE_SWIGLU, M.MOE_BF16, fake, fake, 16, None,
+                                         None) == M.MOE_ERR_ARG

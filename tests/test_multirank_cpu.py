@@ -72,3 +72,55 @@ def test_reference_arm_nonzero_rank_exits_cleanly():
                        text=True, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def _shard_worker(rank, world, port, bounds, results):
+    """One rank of a position-sharded batch: its counts go through the
+    package's all-gather; the capacity rule is the oracle's."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+
+    import oracle
+    from mixture_experts_layer_51_b200.sharded import gather_expert_counts
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        T, E, k, cf = 240, 8, 2, 1.0
+        rng = np.random.default_rng(7)
+        logits = rng.standard_normal((T, E))
+        logits[:, 1] += 1.3
+        idx, _, _ = oracle.top_k(logits, k)
+        a, b = bounds[rank], bounds[rank + 1]
+        counts = torch.as_tensor(np.bincount(idx[a:b].reshape(-1), minlength=E), dtype=torch.int32)
+        gathered = gather_expert_counts(counts)
+        prior = gathered[:rank].sum(0).numpy()
+        _, _, _, kept = oracle.assign_capacity_shard(idx[a:b], E, oracle.capacity(T, E, k, cf),
+                                                     prior)
+        results[rank] = (gathered.numpy().tolist(), kept.tolist())
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_sharded_capacity_exchange_gloo():
+    """Two ranks holding positions [0, 100) and [100, 240) of one batch keep,
+    after exchanging per-expert counts, exactly what the whole batch keeps."""
+    import numpy as np
+
+    import oracle
+    world, bounds = 2, (0, 100, 240)
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_shard_worker, args=(world, port, bounds, results), nprocs=world,
+                       join=True, start_method="spawn")
+    rng = np.random.default_rng(7)
+    logits = rng.standard_normal((240, 8))
+    logits[:, 1] += 1.3
+    idx, _, _ = oracle.top_k(logits, 2)
+    _, _, _, want = oracle.assign_capacity(idx, 8, oracle.capacity(240, 8, 2, 1.0))
+    assert not want.all()  # capacity binds, so the exchange matters
+    g0, kept0 = results[0]
+    g1, kept1 = results[1]
+    assert g0 == g1 == [np.bincount(idx[a:b].reshape(-1), minlength=8).tolist()
+                        for a, b in zip(bounds[:-1], bounds[1:])]
+    assert (np.concatenate([np.array(kept0), np.array(kept1)]) == want).all()
