@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 
 DEFAULT_WORKLOAD = "mixtral_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse_args(argv=None):
@@ -96,19 +97,19 @@ def algorithmic(w, n_kept, tokens_with_kept, routing="token_choice"):
     }
     if routing == "expert_choice":
         # route: read x and W_g, write the [T, E] affinities; select + gather:
-        # read the affinities, write pos [T, E] and the token lists, copy one
-        # x row per assignment; combine: kept rows of o, pos and affinities
-        # [T, E], write y
+        # read the affinities, write pos [T, E] and the token lists, read each
+        # chosen token's x row once and write one row per assignment; combine:
+        # kept rows of o, pos and affinities [T, E], write y
         byts["route"] = T * d * s + d * E * s + T * E * 4
-        byts["permute"] = 2 * T * E * 4 + n_kept * 4 + 2 * n_kept * d * s
+        byts["permute"] = 2 * T * E * 4 + n_kept * 4 + tokens_with_kept * d * s + n_kept * d * s
         byts["combine"] = n_kept * d * 4 + T * E * 8 + T * d * s
     total_flop = flop["route"] + flop["ffn_up"] + flop["ffn_down"]
     return flop, byts, total_flop
 
 
-def traffic_for(kernel_file, kernel):
+def traffic_for(kernel_file, kernel, w):
     """Per-launch DRAM bytes from the committed ncu summary, if it was taken
-    on the current source of the kernel; else None."""
+    on the current source of the kernel and on this workload; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -116,6 +117,9 @@ def traffic_for(kernel_file, kernel):
         src = os.path.join(ROOT, "mixture_experts_layer_51_b200", "csrc", kernel_file)
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         if rec.get("source_sha") != sha:
+            return None
+        cfg = rec.get("config", {})
+        if cfg != {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "H": w.H}:
             return None
         return float(rec["dram_bytes_per_launch"])
     except Exception:
@@ -376,17 +380,23 @@ def main(argv=None):
         if s in ("route", "permute", "combine") and rec["gbs"]:
             rec["frac_hbm"] = round(rec["gbs"] / hbm, 4)
         stages[s] = rec
-    roof_peak = peaks["bf16_tflops_sustained"]
+    act_name = "SwiGLU" if w.act == "swiglu" else "GELU"
     achieved = flop["ffn_up"] / (up_ms / 1e3) / 1e12 if up_ms > 0 else None
-    roofline = {
-        "kernel": "ffn_tc_kernel<%s> (grouped up projection)" % (
-            "SwiGLU" if w.act == "swiglu" else "GELU"),
-        "bound": "tensor", "achieved": round(achieved, 2) if achieved else None,
-        "peak": roof_peak, "unit": "TFLOP/s",
-        "frac": round(achieved / roof_peak, 4) if achieved else None,
-        "traffic": traffic_for("ffn_tc.cu", "ffn_up"),
-        "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)",
-    }
+    if w.dtype == "bf16":
+        roof_peak = peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": f"ffn_tc_kernel<{act_name}> (grouped up projection)",
+                    "bound": "tensor",
+                    "traffic": traffic_for("ffn_tc.cu", "ffn_up", w),
+                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)"}
+    else:
+        # fp32 FMA on the SIMT pipes: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
+        roof_peak = FP32_SIMT_TFLOPS
+        roofline = {"kernel": f"ffn_simt_kernel<{act_name}> (grouped up projection)",
+                    "bound": "alu", "traffic": None,
+                    "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz"}
+    roofline.update({"achieved": round(achieved, 2) if achieved else None, "peak": roof_peak,
+                     "unit": "TFLOP/s",
+                     "frac": round(achieved / roof_peak, 4) if achieved else None})
 
     if rank == 0:
         line = {
