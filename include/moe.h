@@ -321,6 +321,37 @@ moe_status moe_forward_host(const void* x_host, void* y_host, void* x_dev, void*
                             moe_act act, moe_dtype dtype, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* Streaming host pipeline: consecutive batches with tokens in HOST memory,
+ * each copied in, run and copied out on its own slot, so the copies of one
+ * batch overlap the forward of another (copy engines in both directions run
+ * beside the compute stream).  The handle owns two copy streams, events and
+ * a small pinned host array for the device error words; it allocates no
+ * device memory.  depth = number of slots (1 .. MOE_PIPELINE_MAX_DEPTH).
+ *
+ * moe_pipeline_submit enqueues, and returns without waiting:
+ *   copy x_host -> x_dev (copy stream; after the slot's previous forward has
+ *   finished reading x_dev), moe_forward on `stream` (after that copy and
+ *   after the slot's previous copy-out has read y_dev), copy y_dev -> y_host
+ *   (second copy stream); opt as moe_forward_ex (NULL = defaults).
+ *   x_dev, y_dev and ws belong to the slot until
+ *   moe_pipeline_wait(slot) returns; x_host must stay unchanged and y_host
+ *   unread until then.  Every submit on one handle must use the same stream.
+ * moe_pipeline_wait blocks the host until the slot's y_host is written and
+ *   returns MOE_ERR_DEVICE if a kernel of that forward reported an error.
+ * Use one handle from one host thread at a time. */
+#define MOE_PIPELINE_MAX_DEPTH 4
+typedef struct moe_pipeline moe_pipeline;
+moe_status moe_pipeline_create(int32_t depth, moe_pipeline** out);
+moe_status moe_pipeline_submit(moe_pipeline* p, int32_t slot, const void* x_host, void* y_host,
+                               void* x_dev, void* y_dev, const void* Wg, const float* bias,
+                               const void* W1, const void* W3, const void* W2, int32_t T,
+                               int32_t d, int32_t H, int32_t E, int32_t k,
+                               double capacity_factor, moe_act act, moe_dtype dtype,
+                               const moe_options* opt, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_pipeline_wait(moe_pipeline* p, int32_t slot);
+/* Waits for every slot, then releases the handle (NULL is a no-op). */
+moe_status moe_pipeline_destroy(moe_pipeline* p);
+
 /* Stage timing.  `events` points to MOE_NUM_STAGE_EVENTS cudaEvent_t
  * handles (passed as void*) created by the caller, or is NULL to stop.  The
  * next moe_forward / moe_forward_host calls on the calling host thread
@@ -368,11 +399,13 @@ moe_status moe_expert_choice_select(const float* scores, int32_t T, int32_t E, i
                                     int32_t* tok, int32_t* pos, int32_t* kept_counts,
                                     int32_t* offsets, void* ws, size_t ws_bytes, void* stream);
 
-/* xp row e * npad + r = x[tok[e, r]] for r < n (padding rows untouched);
- * xp_rows >= E * npad. */
-moe_status moe_expert_choice_gather(const void* x, const int32_t* tok, int32_t T, int32_t d,
-                                    int32_t E, int32_t n, moe_dtype dtype, void* xp,
-                                    int64_t xp_rows, void* stream);
+/* xp row pos[t, e] = x[t] for every pos[t, e] >= 0 (pos from
+ * moe_expert_choice_select: row e * npad + r holds expert e's r-th token;
+ * padding rows untouched).  Each x row is read once and written once per
+ * expert that took it.  xp_rows >= E * npad. */
+moe_status moe_expert_choice_permute(const void* x, const int32_t* pos, int32_t T, int32_t d,
+                                     int32_t E, int32_t n, moe_dtype dtype, void* xp,
+                                     int64_t xp_rows, void* stream);
 
 /* y [T, d] (dtype) = sum over e with pos[t, e] >= 0, ascending e, of
  * scores[t, e] * o[pos[t, e]] (o fp32 from moe_grouped_ffn), fp32
@@ -404,7 +437,7 @@ size_t moe_expert_choice_workspace_bytes(int32_t T, int32_t d, int32_t H, int32_
                                          double capacity_factor, moe_dtype dtype, moe_act act);
 
 /* The whole layer with expert-choice routing: route (affinities) ->
- * select -> gather -> grouped expert FFNs (as moe_grouped_ffn) -> combine,
+ * select -> permute -> grouped expert FFNs (as moe_grouped_ffn) -> combine,
  * on one stream.  Arguments as moe_forward; k <= E (no kMaxK limit: a token
  * may be taken by any number of experts).  stats (nullable): counts =
  * kept_counts = n per expert; when given, the call waits for the stream and

@@ -11,13 +11,16 @@
 // C = ceil(cf * T * k / E); equal affinities go to the lower position.
 //
 // Kernels here:
-//   ec_select_kernel   one CTA per expert: radix select of the n-th largest
-//                      affinity in its column (4 passes of 8 bits over
-//                      order-preserving 32-bit keys), then one ordered pass
-//                      that marks the chosen tokens and ranks them in
-//                      position order (block-wide ballot scans) -- writes
-//                      the expert's token list and pos[t, e].
-//   ec_gather_kernel   xp row (e, r) = x[token r of expert e] (16-byte copies).
+//   ec_select_kernel   a cluster of CTAs per expert: radix select of the n-th
+//                      largest affinity in its column (4 passes of 8 bits
+//                      over order-preserving 32-bit keys, histograms merged
+//                      through distributed shared memory), then one ordered
+//                      pass that marks the chosen tokens and ranks them in
+//                      position order (CTA-wide ballot scans, slice offsets
+//                      from the cluster) -- writes the expert's token list
+//                      and pos[t, e].
+// The chosen x rows are copied by the token-major row copy of the
+// permutation (read once, written once per expert that took the token).
 //   ec_combine_kernel  one warp per token: y_t = sum over the experts that
 //                      took t, ascending e, of affinity * o row, fp32, one
 //                      rounding.  A gather (no atomics): deterministic.
@@ -28,7 +31,15 @@
 namespace moe {
 namespace {
 
-constexpr int kSelThreads = 1024;
+// Selection: a cluster of kSelCta CTAs per expert, CTA r owning the r-th
+// contiguous slice of token positions.  Every pass builds per-CTA digit
+// histograms (warp-aggregated shared-memory atomics: integer counts, so the
+// order they land in does not matter), then every CTA reads all kSelCta
+// histograms of its cluster through distributed shared memory and sums them
+// in rank order, so all CTAs find the same bucket.  The last pass exchanges
+// per-slice counts the same way to give each slice its starting ranks.
+constexpr int kSelCta = 8;       // CTAs per expert (one cluster)
+constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 
 // Ascending order of these keys is descending order of the float (the
@@ -49,7 +60,7 @@ __device__ __forceinline__ int cta_exclusive_scan(bool flag, int* wsum, int* tot
   if (lane == 0) wsum[warp] = __popc(b);
   __syncthreads();
   int before = 0, all = 0;
-#pragma unroll 4
+#pragma unroll
   for (int w = 0; w < kSelWarps; ++w) {
     const int c = wsum[w];
     before += (w < warp) ? c : 0;
@@ -59,94 +70,168 @@ __device__ __forceinline__ int cta_exclusive_scan(bool flag, int* wsum, int* tot
   return before + __popc(b & ((1u << lane) - 1u));
 }
 
+// Adds 1 to hist[bin] for every lane with bin < 256; lanes with the same
+// bin are combined first, so a popular bin takes one atomic per warp.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
+  const unsigned peers = __match_any_sync(0xffffffffu, bin);
+  const int lane = threadIdx.x & 31;
+  if (bin < 256u && lane == __ffs(peers) - 1)
+    atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+}
+
 __global__ void __launch_bounds__(kSelThreads)
     ec_select_kernel(const float* __restrict__ scores, int T, int E, int n, int npad,
                      uint32_t* __restrict__ keys_t, int32_t* __restrict__ tok,
                      int32_t* __restrict__ pos, int32_t* __restrict__ kept_counts,
                      int32_t* __restrict__ offsets) {
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[2][256];  // alternate passes, so one cluster barrier per pass
+  __shared__ uint32_t tot[256];      // cluster-wide histogram of the current pass
+  __shared__ int slice_cnt[2];       // this slice's keys below the cut and equal to it
   __shared__ int wsum_a[kSelWarps], wsum_b[kSelWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
-  const int e = blockIdx.x;
+  const int e = blockIdx.x / kSelCta;
+  const uint32_t r = cluster_ctarank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (T + kSelCta - 1) / kSelCta;
+  const int t_begin = min(T, static_cast<int>(r) * per), t_end = min(T, t_begin + per);
   uint32_t* keys = keys_t + (int64_t)e * T;
 
-  for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+  for (int i = tid; i < 512; i += kSelThreads) (&hist[0][0])[i] = 0;
   __syncthreads();
-  // The column of affinities as keys (a strided read of [T, E]; the
+  // The slice of the affinity column as keys (a strided read of [T, E]; the
   // transposed copy makes the later passes contiguous) and the histogram of
-  // the top byte.
-  for (int t = tid; t < T; t += kSelThreads) {
-    const uint32_t key = desc_key(scores[(int64_t)t * E + e]);
-    keys[t] = key;
-    atomicAdd(&hist[key >> 24], 1u);
+  // the top byte.  All lanes run the same trip count for the warp votes.
+  for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
+    const int t = b0 + tid;
+    uint32_t bin = 256u;
+    if (t < t_end) {
+      const uint32_t key = desc_key(scores[(int64_t)t * E + e]);
+      keys[t] = key;
+      bin = key >> 24;
+    }
+    hist_add(hist[0], bin);
   }
-  __syncthreads();
 
-  uint32_t prefix = 0;  // the n-th smallest key, one byte per pass
-  int need = n;         // how many of the keys matching prefix are still wanted
-  if (n > 0) {
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      if (pass > 0) {
-        for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
-        __syncthreads();
-        for (int t = tid; t < T; t += kSelThreads) {
+  uint32_t prefix = 0;  // the n-th smallest key of the column, one byte per pass
+  int need = n;         // how many keys equal to the final prefix are taken
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    uint32_t* h = hist[pass & 1];
+    if (pass > 0) {
+      for (int i = tid; i < 256; i += kSelThreads) h[i] = 0;
+      __syncthreads();
+      for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
+        const int t = b0 + tid;
+        uint32_t bin = 256u;
+        if (t < t_end) {
           const uint32_t key = keys[t];
-          if ((key >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+          if ((key >> (shift + 8)) == (prefix >> (shift + 8))) bin = (key >> shift) & 255u;
         }
-        __syncthreads();
+        hist_add(h, bin);
       }
-      if (warp == 0) {
-        // Lane l owns buckets 8l .. 8l+7; find the bucket holding the
-        // need-th key (1-based) in ascending order.
-        int c[8], sum = 0;
+    }
+    // Every CTA's histogram of this pass is complete before any is read;
+    // the other buffer is rewritten only after the next barrier.
+    cluster_sync();
+    if (tid < 256) {
+      const uint32_t local = smem_u32(&h[tid]);
+      uint32_t sum = 0;
+      for (uint32_t q = 0; q < kSelCta; ++q) sum += ld_shared_cluster_u32(mapa_shared(local, q));
+      tot[tid] = sum;
+    }
+    __syncthreads();
+    if (warp == 0 && n > 0) {
+      // Lane l owns buckets 8l .. 8l+7; find the bucket holding the
+      // need-th key (1-based) in ascending order.
+      int c[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = static_cast<int>(tot[lane * 8 + j]);
+        sum += c[j];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      int before = incl - sum;
+      if (before < need && need <= incl) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          c[j] = static_cast<int>(hist[lane * 8 + j]);
-          sum += c[j];
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int u = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += u;
-        }
-        int before = incl - sum;
-        if (before < need && need <= incl) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (need <= before + c[j]) {
-              s_prefix = prefix | (static_cast<uint32_t>(lane * 8 + j) << shift);
-              s_need = need - before;
-              break;
-            }
-            before += c[j];
+          if (need <= before + c[j]) {
+            s_prefix = prefix | (static_cast<uint32_t>(lane * 8 + j) << shift);
+            s_need = need - before;
+            break;
           }
+          before += c[j];
         }
       }
-      __syncthreads();
+    }
+    __syncthreads();
+    if (n > 0) {
       prefix = s_prefix;
       need = s_need;
-      __syncthreads();
     }
   }
 
   // Chosen: key < prefix, or key == prefix among the first `need` such
-  // tokens in position order.  Rows follow position order.
+  // tokens in position order.  First every slice counts both kinds; the
+  // counts of the lower slices give this slice's starting ranks.
+  int lt_n = 0, eq_n = 0;
+  for (int t = t_begin + tid; t < t_end; t += kSelThreads) {
+    const uint32_t key = keys[t];
+    lt_n += (n > 0 && key < prefix);
+    eq_n += (n > 0 && key == prefix);
+  }
+  {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lt_n += __shfl_xor_sync(0xffffffffu, lt_n, o);
+      eq_n += __shfl_xor_sync(0xffffffffu, eq_n, o);
+    }
+    if (lane == 0) {
+      wsum_a[warp] = lt_n;
+      wsum_b[warp] = eq_n;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int a = 0, b = 0;
+      for (int w = 0; w < kSelWarps; ++w) {
+        a += wsum_a[w];
+        b += wsum_b[w];
+      }
+      slice_cnt[0] = a;
+      slice_cnt[1] = b;
+    }
+  }
+  cluster_sync();
+  int eq_before = 0, row_before = 0;
+  for (uint32_t q = 0; q < r; ++q) {
+    const int lt_q =
+        static_cast<int>(ld_shared_cluster_u32(mapa_shared(smem_u32(&slice_cnt[0]), q)));
+    const int eq_q =
+        static_cast<int>(ld_shared_cluster_u32(mapa_shared(smem_u32(&slice_cnt[1]), q)));
+    const int take_q = max(0, min(eq_q, need - eq_before));
+    row_before += lt_q + take_q;
+    eq_before += eq_q;
+  }
+  // No CTA may leave (or reuse its shared memory) while others read it.
+  cluster_sync();
+
   const int32_t row0 = e * npad;
-  int carry_eq = 0, carry_sel = 0;
-  for (int base = 0; base < T; base += kSelThreads) {
-    const int t = base + tid;
-    const uint32_t key = t < T ? keys[t] : 0xffffffffu;
-    const bool eq = n > 0 && t < T && key == prefix;
-    const bool lt = n > 0 && t < T && key < prefix;
+  int carry_eq = eq_before, carry_sel = row_before;
+  for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
+    const int t = b0 + tid;
+    const uint32_t key = t < t_end ? keys[t] : 0xffffffffu;
+    const bool eq = n > 0 && t < t_end && key == prefix;
+    const bool lt = n > 0 && t < t_end && key < prefix;
     int tot_eq, tot_sel;
     const int eq_rank = carry_eq + cta_exclusive_scan(eq, wsum_a, &tot_eq);
     const bool chosen = lt || (eq && eq_rank < need);
     const int row = carry_sel + cta_exclusive_scan(chosen, wsum_b, &tot_sel);
-    if (t < T) {
+    if (t < t_end) {
       pos[(int64_t)t * E + e] = chosen ? row0 + row : -1;
       if (chosen) tok[(int64_t)e * n + row] = t;
     }
@@ -154,33 +239,9 @@ __global__ void __launch_bounds__(kSelThreads)
     carry_sel += tot_sel;
     __syncthreads();  // wsum_a / wsum_b are rewritten by the next chunk
   }
-  if (tid == 0) kept_counts[e] = n;
-  if (e == 0)
+  if (r == 0 && tid == 0) kept_counts[e] = n;
+  if (blockIdx.x == 0)
     for (int i = tid; i <= E; i += kSelThreads) offsets[i] = i * npad;
-}
-
-constexpr int kGatherWarps = 8;
-
-// One warp per xp row; 16-byte vectors, four loads in flight per lane.
-__global__ void __launch_bounds__(kGatherWarps * 32)
-    ec_gather_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ tok, int n, int npad,
-                     int dvec, uint4* __restrict__ xp) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kGatherWarps + warp;
-  const int e = blockIdx.y;
-  if (r >= n) return;
-  const int t = tok[(int64_t)e * n + r];
-  const uint4* src = x + (int64_t)t * dvec;
-  uint4* dst = xp + ((int64_t)e * npad + r) * dvec;
-  for (int v0 = lane; v0 < dvec; v0 += 32 * 4) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (v0 + u * 32 < dvec) v[u] = __ldcs(src + v0 + u * 32);
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (v0 + u * 32 < dvec) dst[v0 + u * 32] = v[u];
-  }
 }
 
 constexpr int kEcCombineWarps = 8;
@@ -263,20 +324,19 @@ size_t ec_select_scratch_bytes(int T, int E) {
 cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad, void* scratch,
                              int32_t* tok, int32_t* pos, int32_t* kept_counts, int32_t* offsets,
                              cudaStream_t s) {
-  ec_select_kernel<<<E, kSelThreads, 0, s>>>(scores, T, E, n, npad,
-                                             static_cast<uint32_t*>(scratch), tok, pos,
-                                             kept_counts, offsets);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_ec_gather(const void* x, const int32_t* tok, int E, int n, int npad, int d,
-                             moe_dtype dtype, void* xp, cudaStream_t s) {
-  if (n == 0) return cudaSuccess;
-  const int dvec = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
-  const dim3 grid((n + kGatherWarps - 1) / kGatherWarps, E);
-  ec_gather_kernel<<<grid, kGatherWarps * 32, 0, s>>>(static_cast<const uint4*>(x), tok, n, npad,
-                                                      dvec, static_cast<uint4*>(xp));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(E * kSelCta);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSelCta;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ec_select_kernel, scores, T, E, n, npad,
+                            static_cast<uint32_t*>(scratch), tok, pos, kept_counts, offsets);
 }
 
 cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,

@@ -55,6 +55,10 @@ constexpr int TN = 256;  // accumulator columns (UMMA N)
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * TN;
 constexpr int CONTROL_BYTES = 1536;
+// Epilogue output staging: per epilogue warp two 4 KB boxes (32 rows x
+// 128 bytes, 128-byte swizzled) that TMA stores drain to global memory.
+constexpr int OUT_BOX_BYTES = 32 * 128;
+constexpr int OUT_STAGE_BYTES = 4 * 2 * OUT_BOX_BYTES;
 #ifndef MOE_PAIR_STAGES
 #define MOE_PAIR_STAGES 6  // ring depth of the CTA-pair kernel with 64-wide K steps
 #endif
@@ -72,7 +76,7 @@ struct Cfg {
   static constexpr int B_CHUNKS = 4 / CG;
   static constexpr int STAGE_BYTES = A_STAGE + B_CHUNKS * B_CHUNK;
   static constexpr int STAGES = CG == 1 ? 4 : (TKS == 64 ? MOE_PAIR_STAGES : 3);
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + CONTROL_BYTES + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_STAGE_BYTES + CONTROL_BYTES + 1024;
   static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
 };
 constexpr int MAX_STAGES = 8;
@@ -137,7 +141,8 @@ __device__ __forceinline__ float gelu_f(float z) {
 template <int EPI, int CG, int TKS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                  const __grid_constant__ CUtensorMap tmB1, const TcParams p) {
+                  const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut,
+                  const TcParams p) {
   using C_ = Cfg<CG, TKS>;
   constexpr int STAGES = C_::STAGES;
   constexpr int STAGE_BYTES = C_::STAGE_BYTES;
@@ -148,7 +153,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  Control& c = *reinterpret_cast<Control*>(smem + STAGES * STAGE_BYTES);
+  Control& c = *reinterpret_cast<Control*>(smem + STAGES * STAGE_BYTES + OUT_STAGE_BYTES);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
@@ -179,6 +184,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     if (EPI == EPI_SWIGLU) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
     if (CG == 2) {
@@ -429,8 +435,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue
+    // Each warp drains its 32 TMEM lanes (tile rows) in batches of 32-column
+    // loads, applies the activation, writes 128-byte rows into a swizzled
+    // 32-row staging box and lets one TMA store per box carry it to global
+    // memory (whole lines, asynchronous; two boxes per warp alternate).  The
+    // accumulator is released as soon as its last batch is in registers.
+    // Rows of a box past the expert's kept rows are padding rows of the same
+    // expert block (never read as results); a CTA whose 128-row block starts
+    // past the kept rows stores nothing.
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
-    const int row = quad * 32 + lane;
+    const uint32_t obuf0 = smem_base + STAGES * STAGE_BYTES + quad * 2 * OUT_BOX_BYTES;
+    uint8_t* const obuf0_p = smem + STAGES * STAGE_BYTES + quad * 2 * OUT_BOX_BYTES;
+    int nbox = 0;
+    // The outputs (h, o) are far larger than L2 and are not read again by
+    // this kernel: their lines go first, so the weight and activation tiles
+    // that other CTAs still read stay resident.
+    const uint64_t out_policy = make_policy_evict_first();
+    // Stages this lane's 8 x 16 bytes as row `lane` of the next box and
+    // issues its store at (col0, row0).
+    auto store_box = [&](const uint4 (&v)[8], int col0, int row0) {
+      const int b = nbox & 1;
+      if (nbox >= 2 && lane == 0) bulk_wait_read<1>();  // the box two stores ago is read
+      __syncwarp();
+      uint8_t* rowp = obuf0_p + b * OUT_BOX_BYTES + lane * 128;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(rowp + ((q ^ (lane & 7)) * 16)) = v[q];
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d_hint(&tmOut, obuf0 + b * OUT_BOX_BYTES, col0, row0, out_policy);
+        bulk_commit();
+      }
+      ++nbox;
+    };
+    auto release = [&](int a) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 2)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&c.tempty[a]), 0));
+        else
+          mbar_arrive(smem_u32(&c.tempty[a]));
+      }
+    };
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = group; t < total; t += ngroups) {
@@ -445,90 +492,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * TN);
-      const int row_in_expert = m * TILE_M + static_cast<int>(rank) * TM + row;
-      const bool row_ok = row_in_expert < c.kept[e];
-      const int64_t grow = static_cast<int64_t>(c.off[e]) + row_in_expert;
+      const int blk_row = m * TILE_M + static_cast<int>(rank) * TM;
+      const bool blk_ok = blk_row < c.kept[e];
+      const int row0 = c.off[e] + blk_row + quad * 32;
       if (EPI == EPI_SWIGLU) {
         const int n0 = n * (TN / 2);
-        __nv_bfloat16* dst_row = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float g[32], u[32];
-          tc_ld_32cols(tbase + cc * 32, g);
-          tc_ld_32cols(tbase + TN / 2 + cc * 32, u);
-          tc_wait_ld();
-          if (row_ok) {
+        for (int c0 = 0; c0 < 4; c0 += 2) {
+          float g[2][32], u[2][32];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int col = n0 + cc * 32 + v * 8;
-              if (col < p.n_out) {
-                uint4 pk;
-                pk.x = pack_bf16x2(silu_f(g[v * 8 + 0]) * u[v * 8 + 0],
-                                   silu_f(g[v * 8 + 1]) * u[v * 8 + 1]);
-                pk.y = pack_bf16x2(silu_f(g[v * 8 + 2]) * u[v * 8 + 2],
-                                   silu_f(g[v * 8 + 3]) * u[v * 8 + 3]);
-                pk.z = pack_bf16x2(silu_f(g[v * 8 + 4]) * u[v * 8 + 4],
-                                   silu_f(g[v * 8 + 5]) * u[v * 8 + 5]);
-                pk.w = pack_bf16x2(silu_f(g[v * 8 + 6]) * u[v * 8 + 6],
-                                   silu_f(g[v * 8 + 7]) * u[v * 8 + 7]);
-                *reinterpret_cast<uint4*>(dst_row + col) = pk;
-              }
+          for (int b = 0; b < 2; ++b) {
+            tc_ld_32cols(tbase + (c0 + b) * 32, g[b]);
+            tc_ld_32cols(tbase + TN / 2 + (c0 + b) * 32, u[b]);
+          }
+          tc_wait_ld();
+          if (c0 + 2 == 4) release(acc);
+          const int col0 = n0 + c0 * 32;
+          if (blk_ok && col0 < p.n_out) {
+            uint4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float* gg = g[q >> 2] + (q & 3) * 8;
+              const float* uu = u[q >> 2] + (q & 3) * 8;
+              v[q].x = pack_bf16x2(silu_f(gg[0]) * uu[0], silu_f(gg[1]) * uu[1]);
+              v[q].y = pack_bf16x2(silu_f(gg[2]) * uu[2], silu_f(gg[3]) * uu[3]);
+              v[q].z = pack_bf16x2(silu_f(gg[4]) * uu[4], silu_f(gg[5]) * uu[5]);
+              v[q].w = pack_bf16x2(silu_f(gg[6]) * uu[6], silu_f(gg[7]) * uu[7]);
             }
+            store_box(v, col0, row0);
           }
         }
       } else if (EPI == EPI_GELU) {
         const int n0 = n * TN;
-        __nv_bfloat16* dst_row = static_cast<__nv_bfloat16*>(p.out) + grow * p.ld_out;
 #pragma unroll 1
-        for (int cc = 0; cc < TN / 32; ++cc) {
-          float g[32];
-          tc_ld_32cols(tbase + cc * 32, g);
-          tc_wait_ld();
-          if (row_ok) {
+        for (int c0 = 0; c0 < TN / 32; c0 += 4) {
+          float g[4][32];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int col = n0 + cc * 32 + v * 8;
-              if (col < p.n_out) {
-                uint4 pk;
-                pk.x = pack_bf16x2(gelu_f(g[v * 8 + 0]), gelu_f(g[v * 8 + 1]));
-                pk.y = pack_bf16x2(gelu_f(g[v * 8 + 2]), gelu_f(g[v * 8 + 3]));
-                pk.z = pack_bf16x2(gelu_f(g[v * 8 + 4]), gelu_f(g[v * 8 + 5]));
-                pk.w = pack_bf16x2(gelu_f(g[v * 8 + 6]), gelu_f(g[v * 8 + 7]));
-                *reinterpret_cast<uint4*>(dst_row + col) = pk;
+          for (int b = 0; b < 4; ++b) tc_ld_32cols(tbase + (c0 + b) * 32, g[b]);
+          tc_wait_ld();
+          if (c0 + 4 == TN / 32) release(acc);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int col0 = n0 + c0 * 32 + h * 64;
+            if (blk_ok && col0 < p.n_out) {
+              uint4 v[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float* gg = g[2 * h + (q >> 2)] + (q & 3) * 8;
+                v[q].x = pack_bf16x2(gelu_f(gg[0]), gelu_f(gg[1]));
+                v[q].y = pack_bf16x2(gelu_f(gg[2]), gelu_f(gg[3]));
+                v[q].z = pack_bf16x2(gelu_f(gg[4]), gelu_f(gg[5]));
+                v[q].w = pack_bf16x2(gelu_f(gg[6]), gelu_f(gg[7]));
               }
+              store_box(v, col0, row0);
             }
           }
         }
       } else {
         const int n0 = n * TN;
-        float* dst_row = static_cast<float*>(p.out) + grow * p.ld_out;
 #pragma unroll 1
-        for (int cc = 0; cc < TN / 32; ++cc) {
-          float g[32];
-          tc_ld_32cols(tbase + cc * 32, g);
-          tc_wait_ld();
-          if (row_ok) {
+        for (int c0 = 0; c0 < TN / 32; c0 += 4) {
+          float g[4][32];
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const int col = n0 + cc * 32 + v * 4;
-              if (col < p.n_out)
-                *reinterpret_cast<float4*>(dst_row + col) =
-                    make_float4(g[v * 4 + 0], g[v * 4 + 1], g[v * 4 + 2], g[v * 4 + 3]);
+          for (int b = 0; b < 4; ++b) tc_ld_32cols(tbase + (c0 + b) * 32, g[b]);
+          tc_wait_ld();
+          if (c0 + 4 == TN / 32) release(acc);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int col0 = n0 + (c0 + b) * 32;
+            if (blk_ok && col0 < p.n_out) {
+              uint4 v[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                v[q] = make_uint4(__float_as_uint(g[b][4 * q + 0]), __float_as_uint(g[b][4 * q + 1]),
+                                  __float_as_uint(g[b][4 * q + 2]), __float_as_uint(g[b][4 * q + 3]));
+              store_box(v, col0, row0);
             }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (CG == 2)
-          mbar_arrive_cluster(mapa_shared(smem_u32(&c.tempty[acc]), 0));
-        else
-          mbar_arrive(smem_u32(&c.tempty[acc]));
-      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    // Every store has completed (and read its staging box) before the CTA
+    // can finish.
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
   }
 
   // ---------------------------------------------------------- teardown
@@ -618,9 +667,24 @@ bool make_map_a3d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D output matrix [rows, cols] (bf16 or fp32) for the epilogue's TMA
+// stores: box = 128 bytes of a row x 32 rows, 128-byte swizzle.
+bool make_map_out(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols, bool f32) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * es};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), 32};
+  cuuint32_t el[2] = {1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+            dims, strides, box, el, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPI, int CG, int TKS>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                       const TcParams& p, int groups, cudaStream_t s) {
+                       const CUtensorMap& out, const TcParams& p, int groups, cudaStream_t s) {
   constexpr int smem = Cfg<CG, TKS>::SMEM_BYTES;
   cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI, CG, TKS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -637,7 +701,7 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<EPI, CG, TKS>, a, b0, b1, p);
+  return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<EPI, CG, TKS>, a, b0, b1, out, p);
 }
 
 // CTA pairs by default; MOE_TC_CTA_PAIR=0 selects one CTA per tile.
@@ -651,23 +715,23 @@ bool use_cta_pairs() {
 
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const TcParams& p, int num_sms, int64_t tiles_max, bool wide_k,
-                        cudaStream_t s) {
+                        const CUtensorMap& out, const TcParams& p, int num_sms, int64_t tiles_max,
+                        bool wide_k, cudaStream_t s) {
   if (use_cta_pairs()) {
     const int groups = static_cast<int>(std::max<int64_t>(
         1, std::min<int64_t>(num_sms / 2, (tiles_max + 1) / 2)));
-    return wide_k ? launch_one<EPI, 2, 128>(a, b0, b1, p, groups, s)
-                  : launch_one<EPI, 2, 64>(a, b0, b1, p, groups, s);
+    return wide_k ? launch_one<EPI, 2, 128>(a, b0, b1, out, p, groups, s)
+                  : launch_one<EPI, 2, 64>(a, b0, b1, out, p, groups, s);
   }
   const int groups = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms, tiles_max)));
-  return launch_one<EPI, 1, 64>(a, b0, b1, p, groups, s);
+  return launch_one<EPI, 1, 64>(a, b0, b1, out, p, groups, s);
 }
 
 }  // namespace
 
 moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEvent_t between) {
   if (a.rows <= 0) return MOE_OK;
-  CUtensorMap mx, mw1, mw3, mh, mw2;
+  CUtensorMap mx, mw1, mw3, mh, mw2, mh_out, mo_out;
   const bool swiglu = a.act == MOE_SWIGLU;
   const bool pairs = use_cta_pairs();
   // Weights: one 4-D load per K step and CTA when the columns come in whole
@@ -687,6 +751,8 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
                                (!swiglu || make_map_3d(&mw3, a.W3, a.E, a.d, a.H)));
   ok = ok && (dn_chunked ? make_map_w4d(&mw2, a.W2, a.E, a.H, a.d, dn_chunks, dn_kr)
                          : make_map_3d(&mw2, a.W2, a.E, a.H, a.d));
+  ok = ok && make_map_out(&mh_out, a.h, a.rows, a.H, false) &&
+       make_map_out(&mo_out, a.o, a.rows, a.d, true);
   if (!ok) return MOE_ERR_CUDA;
   const int64_t mtiles_max = (a.rows + TM - 1) / TM;
 
@@ -703,8 +769,10 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.kept = a.kept_counts;
   up.err = a.dev_error;
   cudaError_t err =
-      swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, up, num_sms, mtiles_max * up.n_tiles, up_wide, s)
-             : launch_gemm<EPI_GELU>(mx, mw1, mw1, up, num_sms, mtiles_max * up.n_tiles, up_wide, s);
+      swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, mh_out, up, num_sms,
+                                       mtiles_max * up.n_tiles, up_wide, s)
+             : launch_gemm<EPI_GELU>(mx, mw1, mw1, mh_out, up, num_sms, mtiles_max * up.n_tiles,
+                                     up_wide, s);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   if (between && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -720,7 +788,8 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
-  err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, dn, num_sms, mtiles_max * dn.n_tiles, dn_wide, s);
+  err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, mo_out, dn, num_sms, mtiles_max * dn.n_tiles,
+                                   dn_wide, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

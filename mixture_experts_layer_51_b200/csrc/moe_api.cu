@@ -4,6 +4,7 @@
 
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -469,10 +470,16 @@ moe_status host_pipe(int dev, HostPipe** out) {
 // the copy of chunk c+1 in and of chunk c-1 out overlap the forward of chunk
 // c.  Tokens are independent without a capacity, so y is unchanged; with a
 // capacity the batch stays whole (capacity is counted over the batch).
+// MOE_HOST_CHUNKS (1 .. 8) overrides the upper bound, for measurements.
 int host_chunks(int32_t T, double cf) {
   if (moe_capacity(T, 1, 1, cf) >= 0) return 1;
+  static const int most = [] {
+    const char* v = getenv("MOE_HOST_CHUNKS");
+    const int n = v ? atoi(v) : 0;
+    return (n >= 1 && n <= kMaxHostChunks) ? n : 4;
+  }();
   int n = T / 1024;
-  return n < 1 ? 1 : (n > 4 ? 4 : n);
+  return n < 1 ? 1 : (n > most ? most : n);
 }
 
 }  // namespace
@@ -550,6 +557,126 @@ MOE_API moe_status moe_forward_host(const void* x_host, void* y_host, void* x_de
   st = read_device_error(Lc, ws, s, &derr);
   if (st != MOE_OK) return st;
   return derr ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+// ======================================================= streaming pipeline
+struct moe_pipeline {
+  int depth = 0;
+  int device = -1;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  struct Slot {
+    cudaEvent_t in = nullptr;        // x copied in
+    cudaEvent_t fwd_done = nullptr;  // forward finished (x_dev, ws free to rewrite)
+    cudaEvent_t out_done = nullptr;  // y copied out (and the error word)
+    bool used = false;
+  } slot[MOE_PIPELINE_MAX_DEPTH];
+  int32_t* err_host = nullptr;       // pinned, one word per slot
+};
+
+namespace {
+void pipeline_release(moe_pipeline* p) {
+  for (auto& sl : p->slot) {
+    if (sl.in) cudaEventDestroy(sl.in);
+    if (sl.fwd_done) cudaEventDestroy(sl.fwd_done);
+    if (sl.out_done) cudaEventDestroy(sl.out_done);
+  }
+  if (p->h2d) cudaStreamDestroy(p->h2d);
+  if (p->d2h) cudaStreamDestroy(p->d2h);
+  if (p->err_host) cudaFreeHost(p->err_host);
+  delete p;
+}
+}  // namespace
+
+MOE_API moe_status moe_pipeline_create(int32_t depth, moe_pipeline** out) {
+  if (!out || depth < 1 || depth > MOE_PIPELINE_MAX_DEPTH) return MOE_ERR_ARG;
+  *out = nullptr;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  moe_pipeline* p = new moe_pipeline();
+  p->depth = depth;
+  p->device = di.device;
+  const unsigned f = cudaEventDisableTiming;
+  bool ok = cudaStreamCreateWithFlags(&p->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p->d2h, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaHostAlloc(reinterpret_cast<void**>(&p->err_host), sizeof(int32_t) * depth,
+                          cudaHostAllocDefault) == cudaSuccess;
+  for (int i = 0; ok && i < depth; ++i)
+    ok = cudaEventCreateWithFlags(&p->slot[i].in, f) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p->slot[i].fwd_done, f) == cudaSuccess &&
+         cudaEventCreateWithFlags(&p->slot[i].out_done, f) == cudaSuccess;
+  if (!ok) {
+    pipeline_release(p);
+    return MOE_ERR_CUDA;
+  }
+  for (int i = 0; i < depth; ++i) p->err_host[i] = 0;
+  *out = p;
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_pipeline_submit(moe_pipeline* p, int32_t slot, const void* x_host,
+                                       void* y_host, void* x_dev, void* y_dev, const void* Wg,
+                                       const float* bias, const void* W1, const void* W3,
+                                       const void* W2, int32_t T, int32_t d, int32_t H,
+                                       int32_t E, int32_t k, double cf, moe_act act,
+                                       moe_dtype dt, const moe_options* opt, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  if (!p || slot < 0 || slot >= p->depth) return MOE_ERR_ARG;
+  moe_ws_layout L;
+  int gating, priority;
+  float gate_scale;
+  if (!compute_layout(T, d, H, E, k, cf, dt, act, &L) ||
+      !read_options(opt, &gating, &gate_scale, &priority))
+    return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !y_host || !x_dev || !y_dev || !ws || ws_bytes < L.total || !aligned16(ws))
+    return MOE_ERR_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev != p->device) return MOE_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto& sl = p->slot[slot];
+  const size_t bytes = static_cast<size_t>(T) * d * elt_size(dt);
+  // The slot's previous forward must be done with x_dev and ws, and its
+  // previous copy-out done with y_dev, before they are rewritten.
+  if (sl.used && (cudaStreamWaitEvent(p->h2d, sl.fwd_done, 0) != cudaSuccess ||
+                  cudaStreamWaitEvent(s, sl.out_done, 0) != cudaSuccess))
+    return MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, p->h2d) != cudaSuccess ||
+      cudaEventRecord(sl.in, p->h2d) != cudaSuccess ||
+      cudaStreamWaitEvent(s, sl.in, 0) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  moe_status st =
+      forward_enqueue(x_dev, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, y_dev, ws, ws_bytes,
+                      L, s, true, opt);
+  if (st != MOE_OK) return st;
+  if (cudaEventRecord(sl.fwd_done, s) != cudaSuccess ||
+      cudaStreamWaitEvent(p->d2h, sl.fwd_done, 0) != cudaSuccess ||
+      cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, p->d2h) != cudaSuccess ||
+      cudaMemcpyAsync(p->err_host + slot, static_cast<uint8_t*>(ws) + L.dev_error,
+                      sizeof(int32_t), cudaMemcpyDeviceToHost, p->d2h) != cudaSuccess ||
+      cudaEventRecord(sl.out_done, p->d2h) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  sl.used = true;
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_pipeline_wait(moe_pipeline* p, int32_t slot) {
+  if (!p || slot < 0 || slot >= p->depth) return MOE_ERR_ARG;
+  auto& sl = p->slot[slot];
+  if (!sl.used) return MOE_OK;
+  if (cudaEventSynchronize(sl.out_done) != cudaSuccess) return MOE_ERR_CUDA;
+  return p->err_host[slot] ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+MOE_API moe_status moe_pipeline_destroy(moe_pipeline* p) {
+  if (!p) return MOE_OK;
+  moe_status st = MOE_OK;
+  for (int i = 0; i < p->depth; ++i)
+    if (p->slot[i].used && cudaEventSynchronize(p->slot[i].out_done) != cudaSuccess)
+      st = MOE_ERR_CUDA;
+  pipeline_release(p);
+  return st;
 }
 
 // ============================================================ expert choice
@@ -636,20 +763,20 @@ MOE_API moe_status moe_expert_choice_select(const float* scores, int32_t T, int3
              : MOE_ERR_CUDA;
 }
 
-MOE_API moe_status moe_expert_choice_gather(const void* x, const int32_t* tok, int32_t T,
-                                            int32_t d, int32_t E, int32_t n, moe_dtype dt,
-                                            void* xp, int64_t xp_rows, void* stream) {
+MOE_API moe_status moe_expert_choice_permute(const void* x, const int32_t* pos, int32_t T,
+                                             int32_t d, int32_t E, int32_t n, moe_dtype dt,
+                                             void* xp, int64_t xp_rows, void* stream) {
   if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || n < 0 || n > T || !valid_dtype(dt))
     return MOE_ERR_ARG;
   if (n == 0) return MOE_OK;
-  if (!x || !tok || !xp || !aligned16(x) || !aligned16(xp) ||
+  if (!x || !pos || !xp || !aligned16(x) || !aligned16(xp) ||
       xp_rows < static_cast<int64_t>(E) * pad_rows(n))
     return MOE_ERR_ARG;
   DeviceInfo di;
   moe_status st = device_info(&di);
   if (st != MOE_OK) return st;
-  return launch_ec_gather(x, tok, E, n, static_cast<int>(pad_rows(n)), d, dt, xp,
-                          static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_row_copy(x, pos, T, E, d, dt, xp, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
@@ -712,7 +839,7 @@ MOE_API moe_status moe_forward_expert_choice(const void* x, const void* Wg, cons
   if (st == MOE_OK)
     st = moe_expert_choice_select(scores, T, E, L.n, tok, pos, kept, offsets, w + L.scratch,
                                   ec_select_scratch_bytes(T, E), s);
-  if (st == MOE_OK) st = moe_expert_choice_gather(x, tok, T, d, E, L.n, dt, w + L.xp, L.rows, s);
+  if (st == MOE_OK) st = moe_expert_choice_permute(x, pos, T, d, E, L.n, dt, w + L.xp, L.rows, s);
   if (st == MOE_OK) st = record_stage(2, s);
   if (st == MOE_OK && L.rows > 0)
     st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,

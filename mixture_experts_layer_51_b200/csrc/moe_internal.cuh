@@ -20,8 +20,6 @@ constexpr int kMaxK = MOE_MAX_TOPK;
 constexpr int kRowAlign = MOE_ROW_ALIGN;
 // Tokens per block of the permutation's first (counting) pass.
 constexpr int kPermBlock = 256;
-// Tokens per chunk (one warp) of the permutation's scatter pass.
-constexpr int kPermChunk = 32;
 // Bounded waits: a kernel that waits longer than this on an on-chip barrier
 // gives up, reports through its error word and exits.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
@@ -97,6 +95,43 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
+}
+// TMA store of a 2-D box from this CTA's shared memory (bulk-group
+// completion: commit, then wait for the reads of the shared-memory source).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+// Same, with an L2 eviction-priority policy (from make_policy_evict_first).
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* m, uint32_t src, int32_t c0,
+                                                  int32_t c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], "
+      "%4;" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+// L2 policy: lines written with it are the first candidates for eviction.
+__device__ __forceinline__ uint64_t make_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N committed bulk groups still read their source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N committed bulk groups are still incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar,
                                             int32_t c0, int32_t c1, int32_t c2) {
@@ -187,6 +222,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
+}
+// 32-bit load from a shared::cluster address (another CTA's shared memory).
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
 // Arrive on an mbarrier that may live in another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
@@ -317,6 +358,9 @@ cudaError_t launch_rank_prefix(const int32_t* gathered, int n_ranks, int E, int 
                                int32_t* prior, cudaStream_t s);
 size_t permute_scratch_bytes(int T, int E);
 cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s);
+// xp[pos[t, j]] = x[t] for every pos[t, j] >= 0 (pos is [T, npos], npos <= kMaxE).
+cudaError_t launch_row_copy(const void* x, const int32_t* pos, int T, int npos, int d,
+                            moe_dtype dtype, void* xp, cudaStream_t s);
 
 size_t priority_scratch_bytes(int T);
 // Stable argsort of the tokens by descending slot-0 gate into order[T].
@@ -329,8 +373,6 @@ size_t ec_select_scratch_bytes(int T, int E);
 cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad, void* scratch,
                              int32_t* tok, int32_t* pos, int32_t* kept_counts, int32_t* offsets,
                              cudaStream_t s);
-cudaError_t launch_ec_gather(const void* x, const int32_t* tok, int E, int n, int npad, int d,
-                             moe_dtype dtype, void* xp, cudaStream_t s);
 cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,
                               int d, int E, moe_dtype dtype, void* y, cudaStream_t s);
 

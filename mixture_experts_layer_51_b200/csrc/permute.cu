@@ -15,9 +15,13 @@
 //     the last block to finish (atomic ticket) turns them into exclusive
 //     per-expert bases, the counts, kept counts (min(count, C)) and the
 //     128-row aligned block offsets.
-//   pass 2 (scatter): per 32-token chunk, rank = block base + counts of the
-//     preceding chunks in the block + ballot prefix inside the chunk; then
-//     the chunk's rows are copied to xp with 16-byte loads and stores.
+//   pass 2 (rank): per 256-token block, rank = block base + counts of the
+//     preceding warps in the block + ballot prefix inside the warp, giving
+//     pos[t, j] (row in xp, or -1 when dropped);
+//   pass 3 (copy): token-major, one warp per token reads its x row once and
+//     writes it to each of its rows (16-byte vectors, eight in flight per
+//     lane).  Splitting the ranks out of the copy keeps their dependent
+//     ballots off the copy's critical path.
 // Every rank is computed from counts in queue order: no atomics decide
 // placement, so the output is deterministic.  The queue order is token
 // position, or -- Batch Priority Routing -- a given permutation `order`
@@ -31,7 +35,7 @@
 namespace moe {
 namespace {
 
-constexpr int kWarpsPerBlock = kPermBlock / 32;  // 8 chunks per block
+constexpr int kWarpsPerBlock = kPermBlock / 32;  // 8 warps per block
 
 // Bit e set when token t selected expert e.  Ids outside [0, E) (possible
 // only when a caller passes its own idx) select nothing and are never kept.
@@ -123,102 +127,86 @@ __global__ void __launch_bounds__(kPermBlock)
   }
 }
 
-// Grid: (chunks of 32 tokens) x (slices of the row).  Every CTA of a chunk
-// recomputes the chunk's ranks (a few ballots); the slice-0 CTA writes pos;
-// each CTA copies its slice [v_begin, v_end) of the 16-byte vectors of every
-// kept row, so a small batch still spreads its copy over all SMs.
-template <int UNROLL>
+// Ranks: one thread per queue position of a 256-token block.  Each warp
+// counts, per expert, its lanes' assignments with one ballot per expert; the
+// ranks inside the warp come from the same ballots (lanes below), the
+// warps below come from the shared counts, and the blocks below from the
+// scanned block_base.  Everything follows from counts in queue order, so
+// positions are deterministic.
 __global__ void __launch_bounds__(kPermBlock)
-    permute_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
-                           const int32_t* __restrict__ order, int T,
-                           int dvec, int slice_vec, int E, int k, const int32_t* __restrict__ cap,
-                           const int32_t* __restrict__ block_base,
-                           const int32_t* __restrict__ offsets, int32_t* __restrict__ pos,
-                           uint4* __restrict__ xp) {
+    permute_rank_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ order, int T,
+                        int E, int k, const int32_t* __restrict__ cap,
+                        const int32_t* __restrict__ block_base,
+                        const int32_t* __restrict__ offsets, int32_t* __restrict__ pos) {
   __shared__ int wcnt[kWarpsPerBlock][kMaxE];
-  __shared__ int base[kMaxE];
-  __shared__ int spos[kPermChunk * kMaxK];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x;
-  const int blk = chunk / kWarpsPerBlock;
-  const int cw = chunk % kWarpsPerBlock;
+  const int blk = blockIdx.x;
+  const int i = blk * kPermBlock + tid;
+  const int t = i < T ? token_at(order, i, T) : T;  // T: no token
+  int ej[kMaxK];
+  uint64_t mask = 0;
+  for (int j = 0; j < k; ++j) {
+    ej[j] = (t < T) ? idx[(int64_t)t * k + j] : -1;
+    if (ej[j] >= 0 && ej[j] < E) mask |= 1ull << ej[j];
+  }
+  int rj[kMaxK];
+  for (int j = 0; j < k; ++j) rj[j] = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int e = 0; e < E; ++e) {
+    const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
+    if (lane == 0) wcnt[warp][e] = __popc(b);
+    if ((mask >> e) & 1ull) {
+      const int r = __popc(b & lt);
+      for (int j = 0; j < k; ++j)
+        if (ej[j] == e) rj[j] = r;
+    }
+  }
+  __syncthreads();
+  if (t >= T) return;
+  for (int j = 0; j < k; ++j) {
+    const int e = ej[j];
+    int p = -1;
+    if (e >= 0 && e < E) {
+      int r = block_base[(int64_t)blk * E + e] + rj[j];
+      for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+      if (r < cap[e]) p = offsets[e] + r;
+    }
+    pos[(int64_t)t * k + j] = p;
+  }
+}
 
-  // Counts of the chunks that precede this one inside its 256-token block.
-  if (warp < cw) {
-    const int i = (blk * kWarpsPerBlock + warp) * kPermChunk + lane;
-    const uint64_t mask = i < T ? expert_mask(idx, token_at(order, i, T), T, k, E) : 0ull;
-    for (int e = 0; e < E; ++e) {
-      const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
-      if (lane == 0) wcnt[warp][e] = __popc(b);
-    }
-  }
-  __syncthreads();
-  if (tid < E) {
-    int s = block_base[(int64_t)blk * E + tid];
-    for (int w = 0; w < cw; ++w) s += wcnt[w][tid];
-    base[tid] = s;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int i = chunk * kPermChunk + lane;
-    const int t = i < T ? token_at(order, i, T) : T;  // T: no token
-    int ej[kMaxK];
-    uint64_t mask = 0;
-    for (int j = 0; j < k; ++j) {
-      ej[j] = (t < T) ? idx[(int64_t)t * k + j] : -1;
-      if (ej[j] >= 0 && ej[j] < E) mask |= 1ull << ej[j];
-    }
-    int rj[kMaxK];
-    for (int j = 0; j < k; ++j) rj[j] = 0;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int e = 0; e < E; ++e) {
-      const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
-      if ((mask >> e) & 1ull) {
-        const int r = base[e] + __popc(b & lt);
-        for (int j = 0; j < k; ++j)
-          if (ej[j] == e) rj[j] = r;
-      }
-    }
-    for (int j = 0; j < k; ++j) {
-      int p = -1;
-      if (t < T && ej[j] >= 0 && ej[j] < E && rj[j] < cap[ej[j]]) p = offsets[ej[j]] + rj[j];
-      if (t < T && blockIdx.y == 0) pos[(int64_t)t * k + j] = p;
-      spos[lane * k + j] = p;
-    }
-  }
-  __syncthreads();
+constexpr int kCopyWarps = 8;
 
-  // Copy each kept token row to its k destinations.
-  for (int i = warp; i < kPermChunk; i += kWarpsPerBlock) {
-    const int q = chunk * kPermChunk + i;
-    if (q >= T) break;
-    const int t = token_at(order, q, T);
-    int p[kMaxK];
-    bool any = false;
-    for (int j = 0; j < k; ++j) {
-      p[j] = spos[i * k + j];
-      any |= p[j] >= 0;
-    }
-    if (!any) continue;
-    const uint4* src = x + (int64_t)t * dvec;
-    const int v_begin = blockIdx.y * slice_vec;
-    const int v_end = min(dvec, v_begin + slice_vec);
-    for (int v0 = v_begin + lane; v0 < v_end; v0 += 32 * UNROLL) {
-      uint4 buf[UNROLL];
+// Token-major row copy: one warp per token reads its x row once (16-byte
+// vectors, eight in flight per lane) and writes it to every destination row
+// pos[t, 0..npos-1] that is >= 0.
+__global__ void __launch_bounds__(kCopyWarps * 32)
+    row_copy_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ pos, int T,
+                    int npos, int dvec, uint4* __restrict__ xp) {
+  __shared__ int dst[kCopyWarps][kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kCopyWarps + warp;
+  if (t >= T) return;
+  int nd = 0;
+  for (int e0 = 0; e0 < npos; e0 += 32) {
+    const int p = e0 + lane < npos ? pos[(int64_t)t * npos + e0 + lane] : -1;
+    const unsigned b = __ballot_sync(0xffffffffu, p >= 0);
+    if (p >= 0) dst[warp][nd + __popc(b & ((1u << lane) - 1u))] = p;
+    nd += __popc(b);
+  }
+  __syncwarp();
+  if (nd == 0) return;
+  const uint4* src = x + (int64_t)t * dvec;
+  for (int v0 = lane; v0 < dvec; v0 += 32 * 8) {
+    uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        const int v = v0 + u * 32;
-        if (v < v_end) buf[u] = __ldg(src + v);
-      }
-      for (int j = 0; j < k; ++j) {
-        if (p[j] < 0) continue;
-        uint4* dst = xp + (int64_t)p[j] * dvec;
+    for (int u = 0; u < 8; ++u)
+      if (v0 + u * 32 < dvec) v[u] = __ldcs(src + v0 + u * 32);
+    for (int j = 0; j < nd; ++j) {
+      uint4* out = xp + (int64_t)dst[warp][j] * dvec;
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-          const int v = v0 + u * 32;
-          if (v < v_end) dst[v] = buf[u];
-        }
-      }
+      for (int u = 0; u < 8; ++u)
+        if (v0 + u * 32 < dvec) out[v0 + u * 32] = v[u];
     }
   }
 }
@@ -285,9 +273,6 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
     return err;
   }
   const int nblk = (a.T + kPermBlock - 1) / kPermBlock;
-  const int nchunk = (a.T + kPermChunk - 1) / kPermChunk;
-  const int elt = dtype == MOE_BF16 ? 2 : 4;
-  const int dvec = a.d * elt / 16;
   cudaError_t err = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned int), s);
   if (err != cudaSuccess) return err;
   int32_t* cap = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a.ticket) + 256);
@@ -296,16 +281,19 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
                                                    a.counts, a.kept_counts, a.offsets);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  // Enough row slices for ~4 CTAs per SM; each slice a multiple of 32 vectors.
-  constexpr int kTargetCtas = 4 * 148;
-  int nslice = (kTargetCtas + nchunk - 1) / nchunk;
-  nslice = std::max(1, std::min(nslice, (dvec + 31) / 32));
-  int slice_vec = (dvec + nslice - 1) / nslice;
-  slice_vec = (slice_vec + 31) / 32 * 32;
-  nslice = (dvec + slice_vec - 1) / slice_vec;
-  permute_scatter_kernel<4><<<dim3(nchunk, nslice), kPermBlock, 0, s>>>(
-      static_cast<const uint4*>(a.x), a.idx, a.order, a.T, dvec, slice_vec, a.E, a.k, cap,
-      a.block_base, a.offsets, a.pos, static_cast<uint4*>(a.xp));
+  permute_rank_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.order, a.T, a.E, a.k, cap,
+                                                  a.block_base, a.offsets, a.pos);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_row_copy(a.x, a.pos, a.T, a.k, a.d, dtype, a.xp, s);
+}
+
+cudaError_t launch_row_copy(const void* x, const int32_t* pos, int T, int npos, int d,
+                            moe_dtype dtype, void* xp, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int dvec = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
+  row_copy_kernel<<<(T + kCopyWarps - 1) / kCopyWarps, kCopyWarps * 32, 0, s>>>(
+      static_cast<const uint4*>(x), pos, T, npos, dvec, static_cast<uint4*>(xp));
   return cudaGetLastError();
 }
 

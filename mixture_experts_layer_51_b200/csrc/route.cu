@@ -18,6 +18,7 @@
 
 #include <float.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include "moe_internal.cuh"
 
@@ -98,6 +99,24 @@ __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t,
   }
 }
 
+// Inserts (v, ei) into a list sorted by descending value (ei < 0: nothing
+// to insert).  An unfilled slot (index < 0) always takes the value, so -inf
+// logits are still ranked in expert order; a strict comparison leaves an
+// equal earlier (lower-index) entry in front.
+template <int KM>
+__device__ __forceinline__ void insert_sorted(float (&tv)[KM], int (&ti)[KM], float v, int ei) {
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    const bool take = ei >= 0 && (v > tv[j] || ti[j] < 0);
+    const float tvj = tv[j];
+    const int tij = ti[j];
+    tv[j] = take ? v : tvj;
+    ti[j] = take ? ei : tij;
+    v = take ? tvj : v;
+    ei = take ? tij : ei;
+  }
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                "r"(src_bytes)
@@ -138,11 +157,22 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// bf16 router.  NT = ceil(E / 8) column tiles of 8 experts; BM tokens per
-// CTA.  The 4 warps split the work as (BM/16) token tiles x KG K-groups:
-// inside each 64-wide K stage, K-group g takes the 16-wide steps g, g+KG, ...
-// The KG partial sums of a token tile are added in a fixed order at the end.
-template <int NT, int BM, int BK, int STAGES, int KM>
+// bf16 router.  NT = ceil(E / 8) column tiles of 8 experts; a cluster of CL
+// CTAs shares one tile of BM = 64 tokens and splits the hidden dimension d:
+// CTA q multiplies its contiguous range of 128-wide K chunks.  Inside a CTA
+// the 4 warps each own 16 tokens.  x and the matching W_g rows stream
+// through a cp.async ring in shared memory.  After the K loop every CTA
+// leaves its partial logits [BM][E] in shared memory, and CTA q sums, for
+// its BM/CL tokens, the CL partials read through distributed shared memory
+// in rank order (a fixed order: deterministic), adds the bias, and selects.
+//
+// Selection: the P = 128 / (BM/CL) threads of a token each keep the sorted
+// top-(k+1) list of a contiguous range of experts (a compare-and-swap
+// chain), then merge lists in a butterfly over the P threads: each round
+// inserts the higher-index half's entries into the lower half's list, so
+// equal logits keep the lower expert first and every thread ends with the
+// same list -- the stable descending order.
+template <int NT, int BM, int BK, int STAGES, int CL, int KM>
 __global__ void __launch_bounds__(kRouteThreads)
     route_bf16_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wg,
                       const float* __restrict__ bias, int T, int d, int E, int k,
@@ -154,19 +184,24 @@ __global__ void __launch_bounds__(kRouteThreads)
   constexpr int XS = x_stride(BK);
   constexpr int SB = stage_bytes(NT, BM, BK);
   constexpr int CPR = BK / 8;        // 16-byte chunks per x row per stage
-  constexpr int MT = BM / 16;        // token tiles per CTA
-  constexpr int KG = 4 / MT;         // K groups
+  static_assert(BM == 64, "four warps of 16 tokens");
+  constexpr int TPC = BM / CL;       // tokens each CTA selects for
+  constexpr int P = kRouteThreads / TPC;  // threads per token in the selection
+  constexpr int LS = NT * 8 + 1;     // logit row stride (floats), conflict-free
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int mt = warp % MT, kg = warp / MT;
-  const int t0 = blockIdx.x * BM;
-  const int nk = (d + BK - 1) / BK;
+  const uint32_t q = CL > 1 ? cluster_ctarank() : 0u;
+  const int t0 = static_cast<int>(blockIdx.x / CL) * BM;
+  const int nk_all = (d + BK - 1) / BK;
+  const int kc_begin = static_cast<int>(q) * nk_all / CL;
+  const int kc_end = (static_cast<int>(q) + 1) * nk_all / CL;
+  const int nk = kc_end - kc_begin;
   const bool vec_wg = (E % 8) == 0;
 
-  auto x_tile = [&](int s) { return smem + s * SB; };
-  auto w_tile = [&](int s) { return smem + s * SB + BM * XS * 2; };
+  auto x_tile = [&](int st) { return smem + st * SB; };
+  auto w_tile = [&](int st) { return smem + st * SB + BM * XS * 2; };
 
-  auto load_stage = [&](int s, int kc) {
+  auto load_stage = [&](int st, int kc) {
     const int k0 = kc * BK;
     // x: BM rows x CPR chunks of 16 bytes (each row segment contiguous).
     for (int i = tid; i < BM * CPR; i += kRouteThreads) {
@@ -174,7 +209,7 @@ __global__ void __launch_bounds__(kRouteThreads)
       const int t = t0 + r, col = k0 + c * 8;
       const bool ok = (t < T) && (col < d);
       const __nv_bfloat16* src = ok ? x + (int64_t)t * d + col : x;
-      cp_async16(smem_u32(x_tile(s) + (r * XS + c * 8) * 2), src, ok ? 16 : 0);
+      cp_async16(smem_u32(x_tile(st) + (r * XS + c * 8) * 2), src, ok ? 16 : 0);
     }
     // W_g rows k0 .. k0+BK-1, columns 0 .. NT*8-1 (zero beyond E and d).
     if (vec_wg) {
@@ -184,10 +219,10 @@ __global__ void __launch_bounds__(kRouteThreads)
         const int row = k0 + r;
         const bool ok = (row < d) && (c < cpr);
         const __nv_bfloat16* src = ok ? Wg + (int64_t)row * E + c * 8 : Wg;
-        cp_async16(smem_u32(w_tile(s) + (r * WS + c * 8) * 2), src, ok ? 16 : 0);
+        cp_async16(smem_u32(w_tile(st) + (r * WS + c * 8) * 2), src, ok ? 16 : 0);
       }
     } else {
-      __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(w_tile(s));
+      __nv_bfloat16* wt = reinterpret_cast<__nv_bfloat16*>(w_tile(st));
       for (int i = tid; i < BK * NT * 8; i += kRouteThreads) {
         const int r = i / (NT * 8), c = i % (NT * 8);
         const int row = k0 + r;
@@ -203,21 +238,21 @@ __global__ void __launch_bounds__(kRouteThreads)
     for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
 
 #pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (s < nk) load_stage(s, s);
+  for (int st = 0; st < STAGES - 1; ++st) {
+    if (st < nk) load_stage(st, kc_begin + st);
     cp_async_commit();
   }
 
-  for (int kc = 0; kc < nk; ++kc) {
+  for (int kk_c = 0; kk_c < nk; ++kk_c) {
     cp_async_wait<STAGES - 2>();
     __syncthreads();
-    const int s = kc % STAGES;
-    const uint32_t xa = smem_u32(x_tile(s));
-    const uint32_t wa = smem_u32(w_tile(s));
+    const int st = kk_c % STAGES;
+    const uint32_t xa = smem_u32(x_tile(st));
+    const uint32_t wa = smem_u32(w_tile(st));
 #pragma unroll
-    for (int kk = kg; kk < BK / 16; kk += KG) {
+    for (int kk = 0; kk < BK / 16; ++kk) {
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(xa + ((mt * 16 + (lane & 15)) * XS + kk * 16 + (lane >> 4) * 8) * 2, a0, a1, a2,
+      ldsm_x4(xa + ((warp * 16 + (lane & 15)) * XS + kk * 16 + (lane >> 4) * 8) * 2, a0, a1, a2,
               a3);
 #pragma unroll
       for (int n = 0; n + 1 < NT; n += 2) {
@@ -233,20 +268,17 @@ __global__ void __launch_bounds__(kRouteThreads)
         mma_bf16_16816(acc[NT - 1], a0, a1, a2, a3, b0, b1);
       }
     }
-    const int nxt = kc + STAGES - 1;
-    if (nxt < nk) load_stage(nxt % STAGES, nxt);
+    const int nxt = kk_c + STAGES - 1;
+    if (nxt < nk) load_stage(nxt % STAGES, kc_begin + nxt);
     cp_async_commit();
   }
   cp_async_wait<0>();
   __syncthreads();
 
-  // Partial logits to shared memory: [KG][BM][NT*8 + 1] fp32 (reuses the ring),
-  // then each token's KG partials are added in group order.
-  float* lg = reinterpret_cast<float*>(smem);
-  constexpr int LS = NT * 8 + 1;
+  // This CTA's partial logits [BM][LS] (reusing the ring).
+  float* part = reinterpret_cast<float*>(smem);
   {
-    float* part = lg + kg * BM * LS;
-    const int r = mt * 16 + (lane >> 2);
+    const int r = warp * 16 + (lane >> 2);
     const int c = (lane & 3) * 2;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
@@ -256,41 +288,114 @@ __global__ void __launch_bounds__(kRouteThreads)
       part[(r + 8) * LS + n * 8 + c + 1] = acc[n][3];
     }
   }
-  __syncthreads();
-  auto logit = [&](int r, int e) {
-    float v = lg[r * LS + e];
+  if (CL > 1) cluster_sync(); else __syncthreads();
+
+  // Logits of this CTA's TPC tokens: the CL partials summed in rank order.
+  float* fin = part + BM * LS;              // [TPC][LS]
+  for (int i = tid; i < TPC * E; i += kRouteThreads) {
+    const int rr = i / E, e = i - rr * E;
+    const int r = static_cast<int>(q) * TPC + rr;
+    float v;
+    if (CL > 1) {
+      const uint32_t a = smem_u32(&part[r * LS + e]);
+      v = 0.f;
 #pragma unroll
-    for (int g = 1; g < KG; ++g) v += lg[(g * BM + r) * LS + e];
-    return bias ? v + bias[e] : v;
-  };
+      for (int c = 0; c < CL; ++c) v += __uint_as_float(ld_shared_cluster_u32(mapa_shared(a, c)));
+    } else {
+      v = part[r * LS + e];
+    }
+    fin[rr * LS + e] = bias ? v + bias[e] : v;
+  }
+  // Every CTA has read the partials it needs before any CTA moves on.
+  if (CL > 1) cluster_sync(); else __syncthreads();
+
+  const int rr = tid / P, p = tid % P;
+  const int t = t0 + static_cast<int>(q) * TPC + rr;
+  const float* lrow = fin + rr * LS;
   if (scores) {
-    // Expert-choice affinities: the softmax over all E logits of every
-    // token, written as rows of [T, E].  One thread per token finds the
-    // maximum and the denominator; then the whole CTA writes the BM x E
-    // tile in index order (coalesced), each value recomputed from the same
-    // logit and maximum, so it equals the term that entered the sum.
-    float* rowstat = lg + KG * BM * LS;  // [BM][2]: max, 1/sum
-    if (tid < BM) {
-      float m = -INFINITY;
-      for (int e = 0; e < E; ++e) m = fmaxf(m, logit(tid, e));
-      float sum = 0.f;
-      for (int e = 0; e < E; ++e) sum += expf(logit(tid, e) - m);
-      rowstat[2 * tid] = m;
-      rowstat[2 * tid + 1] = 1.f / sum;
-    }
-    __syncthreads();
-    const int nrow = min(BM, T - t0);
-    for (int i = tid; i < nrow * E; i += kRouteThreads) {
-      const int r = i / E, e = i - r * E;
-      scores[(int64_t)t0 * E + i] = expf(logit(r, e) - rowstat[2 * r]) * rowstat[2 * r + 1];
-    }
+    // Expert-choice affinities: softmax over all E logits.  The P threads
+    // of a token combine their maxima and sums with a fixed butterfly.
+    float m = -INFINITY;
+    for (int e = p; e < E; e += P) m = fmaxf(m, lrow[e]);
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+    for (int e = p; e < E; e += P) sum += expf(lrow[e] - m);
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.f / sum;
+    if (t < T)
+      for (int e = p; e < E; e += P) scores[(int64_t)t * E + e] = expf(lrow[e] - m) * inv;
     return;
   }
-  if (tid < BM) {
-    const int t = t0 + tid;
-    if (t < T) {
-      auto get = [&](int e) { return logit(tid, e); };
-      topk_softmax_store<KM>(get, E, k, t, idx, gate, margin, gating, gate_scale);
+  // This thread's experts [e_lo, e_hi), then the butterfly merge.
+  float tv[KM];
+  int ti[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    tv[j] = -INFINITY;
+    ti[j] = -1;
+  }
+  {
+    const int per = (E + P - 1) / P;
+    const int e_lo = min(E, p * per), e_hi = min(E, e_lo + per);
+    for (int e = e_lo; e < e_hi; ++e) insert_sorted<KM>(tv, ti, lrow[e], e);
+  }
+#pragma unroll
+  for (int o = 1; o < P; o <<= 1) {
+    float pv[KM];
+    int pi[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      pv[j] = __shfl_xor_sync(0xffffffffu, tv[j], o);
+      pi[j] = __shfl_xor_sync(0xffffffffu, ti[j], o);
+    }
+    if (p & o) {
+      // The partner holds the lower experts: its list goes first.
+#pragma unroll
+      for (int j = 0; j < KM; ++j) {
+        const float v = tv[j];
+        const int ei = ti[j];
+        tv[j] = pv[j];
+        ti[j] = pi[j];
+        pv[j] = v;
+        pi[j] = ei;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j) insert_sorted<KM>(tv, ti, pv[j], pi[j]);
+  }
+  const float m = tv[0];  // the largest logit
+  float denom = 0.f;
+  if (gating == MOE_GATE_SOFTMAX_TOPK) {
+    // Switch order: the softmax denominator over all E logits.
+    for (int e = p; e < E; e += P) denom += expf(lrow[e] - m);
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+  } else {
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (j < k) denom += expf(tv[j] - m);
+  }
+  if (t < T) {
+    const float inv = gate_scale / denom;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (j < k && j % P == p) {
+        idx[(int64_t)t * k + j] = ti[j];
+        gate[(int64_t)t * k + j] = expf(tv[j] - m) * inv;
+      }
+    }
+    if (margin) {
+      // slot k-1 minus slot k (every gap computed, one kept: no dynamic
+      // index into the list)
+      float mg = INFINITY;
+#pragma unroll
+      for (int j = 1; j < KM; ++j) {
+        const float gap = tv[j - 1] - tv[j];
+        mg = (j == k && k < E) ? gap : mg;
+      }
+      if (p == 0) margin[t] = mg;
     }
   }
 }
@@ -346,28 +451,57 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
 }
 
-template <int NT, int BM, int BK, int STAGES, int KM>
+template <int NT, int BM, int BK, int STAGES, int CL, int KM>
 cudaError_t launch_route_cfg(const RouteArgs& a, cudaStream_t s) {
   constexpr int smem = STAGES * stage_bytes(NT, BM, BK);
-  static_assert(BM * (NT * 8 + 1) * 4 * (4 / (BM / 16)) + BM * 8 <= smem, "epilogue buffer");
-  cudaError_t err = cudaFuncSetAttribute(route_bf16_kernel<NT, BM, BK, STAGES, KM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr int TPC = BM / CL;
+  static_assert((BM + TPC) * (NT * 8 + 1) * 4 <= smem, "epilogue buffers");
+  auto kern = route_bf16_kernel<NT, BM, BK, STAGES, CL, KM>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  const int grid = (a.T + BM - 1) / BM;
-  route_bf16_kernel<NT, BM, BK, STAGES, KM><<<grid, kRouteThreads, smem, s>>>(
-      static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T,
-      a.d, a.E, a.k, a.idx, a.gate, a.margin, a.gating, a.gate_scale, a.scores);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(((a.T + BM - 1) / BM) * CL);
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(a.x),
+                            static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T, a.d, a.E, a.k,
+                            a.idx, a.gate, a.margin, a.gating, a.gate_scale, a.scores);
 }
 
-// Configurations chosen by a sweep on B200 (8192 x 4096, E = 8 and
-// 16384 x 2048, E = 64): 64-token tiles with 128-wide K stages were fastest,
-// because each stage re-streams a W_g chunk from L2 and larger token tiles
-// amortise it; fewer, longer-lived CTAs beat finer tiles here.
+// CTAs per token tile: the largest of 1, 2, 4 that keeps the grid within
+// about two CTAs per SM and gives every CTA at least four 128-wide K chunks
+// (a sweep on the B200: the 8192 x 4096 router is fastest with pairs, the
+// 16384 x 2048 one with single CTAs).  MOE_ROUTE_CL (1, 2 or 4) overrides
+// the choice, for measurements.
+int route_cluster_size(int T, int d) {
+  static const int forced = [] {
+    const char* v = getenv("MOE_ROUTE_CL");
+    return v ? atoi(v) : 0;
+  }();
+  if (forced == 1 || forced == 2 || forced == 4) return forced;
+  const int tiles = (T + 63) / 64;
+  const int chunks = (d + 127) / 128;
+  int cl = 1;
+  while (cl < 4 && tiles * cl * 2 <= 2 * 148 && chunks >= 8 * cl) cl *= 2;
+  return cl;
+}
+
 template <int NT, int KM>
 cudaError_t launch_route_nt(const RouteArgs& a, cudaStream_t s) {
-  if (NT <= 2) return launch_route_cfg<NT, 64, 128, 4, KM>(a, s);
-  return launch_route_cfg<NT, 64, 128, 3, KM>(a, s);
+  constexpr int ST = NT <= 2 ? 4 : 3;
+  switch (route_cluster_size(a.T, a.d)) {
+    case 4: return launch_route_cfg<NT, 64, 128, ST, 4, KM>(a, s);
+    case 2: return launch_route_cfg<NT, 64, 128, ST, 2, KM>(a, s);
+    default: return launch_route_cfg<NT, 64, 128, ST, 1, KM>(a, s);
+  }
 }
 
 template <int KM>
@@ -384,6 +518,14 @@ cudaError_t launch_route_km(const RouteArgs& a, cudaStream_t s) {
   }
 }
 
+// KM = length of the running top lists (k + 1, rounded up to 3, 5 or 9);
+// the affinity output uses none.
+cudaError_t launch_route_bf16(const RouteArgs& a, cudaStream_t s) {
+  if (a.scores || a.k <= 2) return launch_route_km<3>(a, s);
+  if (a.k <= 4) return launch_route_km<5>(a, s);
+  return launch_route_km<kMaxK + 1>(a, s);
+}
+
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int /*num_sms*/) {
@@ -395,11 +537,7 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
                                                     a.gating, a.gate_scale, a.scores);
     return cudaGetLastError();
   }
-  // KM = slots of the running top list (k + 1, rounded up to 3, 5 or 9);
-  // the affinity output uses no list.
-  if (a.scores || a.k <= 2) return launch_route_km<3>(a, s);
-  if (a.k <= 4) return launch_route_km<5>(a, s);
-  return launch_route_km<kMaxK + 1>(a, s);
+  return launch_route_bf16(a, s);
 }
 
 }  // namespace moe

@@ -32,9 +32,11 @@ EXPORTED = (
     "moe_priority_workspace_bytes", "moe_rows_for_capacity", "moe_expert_counts",
     "moe_rank_prefix", "moe_expert_choice_tokens", "moe_expert_choice_route",
     "moe_expert_choice_select_workspace_bytes", "moe_expert_choice_select",
-    "moe_expert_choice_gather", "moe_expert_choice_combine", "moe_expert_choice_layout",
-    "moe_expert_choice_workspace_bytes", "moe_forward_expert_choice",
+    "moe_expert_choice_permute", "moe_expert_choice_combine", "moe_expert_choice_layout",
+    "moe_expert_choice_workspace_bytes", "moe_forward_expert_choice", "moe_pipeline_create",
+    "moe_pipeline_submit", "moe_pipeline_wait", "moe_pipeline_destroy",
 )
+MOE_PIPELINE_MAX_DEPTH = 4
 MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
 MOE_PRIORITY_POSITION, MOE_PRIORITY_GATE = 0, 1
 MOE_PERMUTE_STATIC_MAX_INTS = 1 << 18
@@ -170,9 +172,9 @@ def lib():
     L.moe_expert_choice_select_workspace_bytes.argtypes = [_I32, _I32]
     L.moe_expert_choice_select.restype = ctypes.c_int
     L.moe_expert_choice_select.argtypes = [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]
-    L.moe_expert_choice_gather.restype = ctypes.c_int
-    L.moe_expert_choice_gather.argtypes = [_P, _P, _I32, _I32, _I32, _I32, ctypes.c_int, _P, _I64,
-                                           _P]
+    L.moe_expert_choice_permute.restype = ctypes.c_int
+    L.moe_expert_choice_permute.argtypes = [_P, _P, _I32, _I32, _I32, _I32, ctypes.c_int, _P,
+                                            _I64, _P]
     L.moe_expert_choice_combine.restype = ctypes.c_int
     L.moe_expert_choice_combine.argtypes = [_P, _P, _P, _I32, _I32, _I32, ctypes.c_int, _P, _P]
     L.moe_expert_choice_layout.restype = ctypes.c_int
@@ -181,6 +183,16 @@ def lib():
     L.moe_expert_choice_workspace_bytes.restype = _SZ
     L.moe_expert_choice_workspace_bytes.argtypes = [_I32, _I32, _I32, _I32, _I32, _D,
                                                     ctypes.c_int, ctypes.c_int]
+    L.moe_pipeline_create.restype = ctypes.c_int
+    L.moe_pipeline_create.argtypes = [_I32, ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_pipeline_submit.restype = ctypes.c_int
+    L.moe_pipeline_submit.argtypes = [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
+                                      _I32, _I32, _I32, _D, ctypes.c_int, ctypes.c_int,
+                                      ctypes.POINTER(moe_options), _P, _SZ, _P]
+    L.moe_pipeline_wait.restype = ctypes.c_int
+    L.moe_pipeline_wait.argtypes = [_P, _I32]
+    L.moe_pipeline_destroy.restype = ctypes.c_int
+    L.moe_pipeline_destroy.argtypes = [_P]
     L.moe_forward_expert_choice.restype = ctypes.c_int
     L.moe_forward_expert_choice.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                             _D, ctypes.c_int, ctypes.c_int, _P, _P, _SZ,
@@ -444,6 +456,53 @@ def moe_forward_host(x_host, Wg, bias, W1, W3, W2, k, capacity_factor, act, y_ho
     return y_host
 
 
+class Pipeline:
+    """Streaming forwards of host-resident batches (moe_pipeline_*): slot i
+    owns a device input, output and workspace; submit() enqueues copy-in,
+    forward and copy-out and returns at once, wait() blocks until the slot's
+    host output is written.  Copies of one batch overlap the forward of
+    another."""
+
+    def __init__(self, layer, T, depth=2, stream=None):
+        self.layer, self.T, self.depth = layer, T, depth
+        dev, d = layer.device, layer.d
+        self.stream = stream
+        self.x_dev = [torch.empty((T, d), dtype=layer.dtype, device=dev) for _ in range(depth)]
+        self.y_dev = [torch.empty((T, d), dtype=layer.dtype, device=dev) for _ in range(depth)]
+        need = moe_workspace_bytes(T, d, layer.H, layer.E, layer.k, layer.cf, layer.dtype,
+                                   layer.act)
+        self.ws = [torch.empty(need, dtype=torch.uint8, device=dev) for _ in range(depth)]
+        h = ctypes.c_void_p()
+        _check(lib().moe_pipeline_create(depth, ctypes.byref(h)), "moe_pipeline_create")
+        self._h = h
+
+    def submit(self, slot, x_host, y_host):
+        L = self.layer
+        T, d = x_host.shape
+        assert T == self.T and d == L.d
+        _check(lib().moe_pipeline_submit(
+            self._h, slot, _ptr(x_host), _ptr(y_host), _ptr(self.x_dev[slot]),
+            _ptr(self.y_dev[slot]), _ptr(L.Wg), _ptr(L.bias), _ptr(L.W1), _ptr(L.W3),
+            _ptr(L.W2), T, d, L.H, L.E, L.k, _cf(L.cf), _act_code(L.act), _dtype_code(x_host),
+            ctypes.byref(_options(L.gating, L.gate_scale, L.priority)), _ptr(self.ws[slot]),
+            self.ws[slot].numel(), _stream(L.device, self.stream)),
+            "moe_pipeline_submit")
+
+    def wait(self, slot):
+        _check(lib().moe_pipeline_wait(self._h, slot), "moe_pipeline_wait")
+
+    def close(self):
+        if self._h:
+            _check(lib().moe_pipeline_destroy(self._h), "moe_pipeline_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 def moe_set_stage_events(events):
     """Record ``events`` (six torch.cuda.Event, created with timing enabled)
     between the stages of the next forwards on this thread; None stops."""
@@ -536,14 +595,15 @@ def moe_expert_choice_select(scores, n, stream=None):
     return dict(tok=tok, pos=pos, kept_counts=kept_counts, offsets=offsets)
 
 
-def moe_expert_choice_gather(x, tok, xp=None, stream=None):
+def moe_expert_choice_permute(x, pos, n, xp=None, stream=None):
+    """xp rows from pos [T, E] (moe_expert_choice_select): row pos[t, e] = x[t]."""
     T, d = x.shape
-    E, n = tok.shape
+    E = pos.shape[1]
     npad = (n + MOE_ROW_ALIGN - 1) // MOE_ROW_ALIGN * MOE_ROW_ALIGN
     xp = xp if xp is not None else torch.empty((E * npad, d), dtype=x.dtype, device=x.device)
-    _check(lib().moe_expert_choice_gather(_ptr(x), _ptr(tok), T, d, E, n, _dtype_code(x),
-                                          _ptr(xp), xp.shape[0], _stream(x.device, stream)),
-           "moe_expert_choice_gather")
+    _check(lib().moe_expert_choice_permute(_ptr(x), _ptr(pos), T, d, E, n, _dtype_code(x),
+                                           _ptr(xp), xp.shape[0], _stream(x.device, stream)),
+           "moe_expert_choice_permute")
     return xp
 
 

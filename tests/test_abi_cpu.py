@@ -209,10 +209,10 @@ def test_expert_choice_sizes_and_validation(lib):
                                         None) == M.MOE_ERR_ARG
     assert lib.moe_expert_choice_route(fake, fake, None, 10, 64, 65, M.MOE_BF16, fake,
                                        None) == M.MOE_ERR_ARG
-    assert lib.moe_expert_choice_gather(ctypes.c_void_p(0x10004), fake, 10, 64, 4, 3, M.MOE_BF16,
-                                        fake, 512, None) == M.MOE_ERR_ARG
-    assert lib.moe_expert_choice_gather(fake, fake, 10, 64, 4, 3, M.MOE_BF16, fake, 384,
-                                        None) == M.MOE_ERR_ARG
+    assert lib.moe_expert_choice_permute(ctypes.c_void_p(0x10004), fake, 10, 64, 4, 3,
+                                         M.MOE_BF16, fake, 512, None) == M.MOE_ERR_ARG
+    assert lib.moe_expert_choice_permute(fake, fake, 10, 64, 4, 3, M.MOE_BF16, fake, 384,
+                                         None) == M.MOE_ERR_ARG
     assert lib.moe_forward_expert_choice(fake, fake, None, fake, fake, fake, 64, 64, 64, 8, 2,
                                          1.0, M.MOE_SWIGLU, M.MOE_BF16, fake, fake, 16, None,
                                          None) == M.MOE_ERR_ARG

@@ -166,6 +166,35 @@ def test_forward_host_chunked_matches_device_forward(T, cf):
         assert np.array_equal(y_host.float().numpy(), g["y"])
 
 
+@pytest.mark.parametrize("depth,gating,cf", [(2, "topk_softmax", 0.0), (3, "softmax_topk", 1.0),
+                                             (1, "topk_softmax", 1.25)])
+def test_streaming_pipeline_matches_device_forward(depth, gating, cf):
+    """moe_pipeline_*: seven different host batches streamed through `depth`
+    slots (copies of one overlapping the forward of another) give, batch by
+    batch, the same bits as the device-resident forward."""
+    w = Workload("stream", T=1500, d=256, E=8, k=2, H=384, act="swiglu", dtype="bf16", cf=cf,
+                 seed=12)
+    inp = make_inputs(w, "cuda")
+    layer = M.MoELayer(inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], w.k, w.cf,
+                       w.act, gating=gating)
+    g = torch.Generator().manual_seed(3)
+    xs = [torch.randn(w.T, w.d, generator=g).bfloat16().pin_memory() for _ in range(7)]
+    want = [to_np(layer(x.cuda()).float()) for x in xs]
+    torch.cuda.synchronize()
+    pipe = M.Pipeline(layer, w.T, depth=depth)
+    ys = [torch.empty_like(x).pin_memory() for x in xs]
+    for i, x in enumerate(xs):
+        slot = i % depth
+        if i >= depth:
+            pipe.wait(slot)
+            assert np.array_equal(ys[i - depth].float().numpy(), want[i - depth])
+        pipe.submit(slot, x, ys[i])
+    for i in range(len(xs) - depth, len(xs)):
+        pipe.wait(i % depth)
+        assert np.array_equal(ys[i].float().numpy(), want[i])
+    pipe.close()
+
+
 def test_stage_entry_points_match_forward():
     """moe_route -> moe_permute -> moe_grouped_ffn -> moe_unpermute_combine
     called one by one give the same bits as moe_forward."""
@@ -262,3 +291,25 @@ def test_full_size_layer(name):
             rate = [float((~kept[(p >= a) & (p < a + span // 8)]).mean())
                     for a in range(0, span, span // 8)]
             print(f"drop rate by {label} octile:", [round(r, 4) for r in rate])
+
+
+@pytest.mark.parametrize("cf", [0.0, 1.0])
+def test_largest_expert_count_and_top_k(cf):
+    """E = 64 and k = 8 (the largest the library takes) on a 65536-token
+    batch (524288 assignments): routing away from near-ties and the whole
+    permutation bit-exact, sampled outputs within tolerance."""
+    w = Workload("max", T=65536, d=512, E=64, k=8, H=256, act="swiglu", dtype="bf16", cf=cf,
+                 seed=31, bias_var=0.5)
+    inp = make_inputs(w, "cuda")
+    g = run_gpu(w, inp)
+    assert int(g["dev_error"][0]) == 0
+    cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    logits = oracle.router_logits(cpu["x"], cpu["Wg"], cpu["bias"])
+    check_routing(g, logits, w.k)
+    kept, C = check_permutation(g, None, w.T, w.E, w.k, w.cf)
+    assert (C is None) == (cf == 0.0)
+    rng = np.random.default_rng(3)
+    sample = np.unique(np.concatenate([[0, w.T - 1], rng.choice(w.T, 64, replace=False)]))
+    y_ref, _ = oracle.moe_forward_tokens(cpu["x"][sample], logits[sample], g["idx"][sample],
+                                         kept[sample], cpu["W1"], cpu["W3"], cpu["W2"], w.act)
+    assert_y_close(g["y"][sample], y_ref, w.dtype)
