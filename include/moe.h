@@ -16,11 +16,14 @@
  * ---------------------------------------
  * - Every pointer argument is a DEVICE pointer unless the name says host.
  *   The caller allocates and owns every buffer; the library never allocates
- *   or frees device memory and keeps no pointer after a call returns.
+ *   or frees device memory and keeps no pointer after a call returns (a
+ *   moe_pipeline handle, created and destroyed by the caller, owns copy
+ *   streams, events and a few bytes of pinned host memory).
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream).  All work is enqueued on it; calls return without waiting for
- *   the GPU, except that moe_forward with a non-NULL `stats` and
- *   moe_forward_host wait for their own stream before returning.
+ *   the GPU, except that moe_forward(_ex) and moe_forward_expert_choice
+ *   with a non-NULL `stats`, moe_forward_host and moe_pipeline_wait wait
+ *   before returning.
  * - Layouts are row-major and dense: x [T, d]; W_g [d, E]; W1, W3 [E, d, H];
  *   W2 [E, H, d]; y [T, d]; idx, gate, pos [T, k].
  * - Element types: MOE_BF16 means x, W_g, W1, W3, W2, xp, h and y are bf16;

@@ -25,6 +25,8 @@ template <bool OUT_BF16, int CH>
 __global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ pos,
                    const float* __restrict__ gate, int T, int d, int k, void* __restrict__ y) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= T) return;
@@ -104,19 +106,13 @@ cudaError_t launch_combine(const CombineArgs& a, moe_dtype dtype, cudaStream_t s
   if (a.T == 0) return cudaSuccess;
   const int grid = (a.T + kCombineWarps - 1) / kCombineWarps;
   const float4* o = reinterpret_cast<const float4*>(a.o);
-  const int th = kCombineWarps * 32;
-  if (dtype == MOE_BF16) {
-    if (a.k <= 2)
-      combine_kernel<true, 2><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
-    else
-      combine_kernel<true, 1><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
-  } else {
-    if (a.k <= 2)
-      combine_kernel<false, 2><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
-    else
-      combine_kernel<false, 1><<<grid, th, 0, s>>>(o, a.pos, a.gate, a.T, a.d, a.k, a.y);
-  }
-  return cudaGetLastError();
+  const dim3 th(kCombineWarps * 32);
+  auto go = [&](auto kern) {
+    return launch_kernel(kern, dim3(grid), th, 0, s, 1, true, o, a.pos, a.gate, a.T, a.d, a.k, a.y);
+  };
+  if (dtype == MOE_BF16)
+    return a.k <= 2 ? go(combine_kernel<true, 2>) : go(combine_kernel<true, 1>);
+  return a.k <= 2 ? go(combine_kernel<false, 2>) : go(combine_kernel<false, 1>);
 }
 
 }  // namespace moe

@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kSelThreads)
   __shared__ int wsum_a[kSelWarps], wsum_b[kSelWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x / kSelCta;
   const uint32_t r = cluster_ctarank();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -253,6 +255,8 @@ __global__ void __launch_bounds__(kEcCombineWarps * 32)
                       void* __restrict__ y) {
   __shared__ int sp[kEcCombineWarps][kMaxE];
   __shared__ float sg[kEcCombineWarps][kMaxE];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kEcCombineWarps + warp;
   if (t >= T) return;
@@ -324,19 +328,9 @@ size_t ec_select_scratch_bytes(int T, int E) {
 cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad, void* scratch,
                              int32_t* tok, int32_t* pos, int32_t* kept_counts, int32_t* offsets,
                              cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(E * kSelCta);
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kSelCta;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ec_select_kernel, scores, T, E, n, npad,
-                            static_cast<uint32_t*>(scratch), tok, pos, kept_counts, offsets);
+  return launch_kernel(ec_select_kernel, dim3(E * kSelCta), dim3(kSelThreads), 0, s, kSelCta, true,
+                       scores, T, E, n, npad, static_cast<uint32_t*>(scratch), tok, pos,
+                       kept_counts, offsets);
 }
 
 cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,
@@ -344,11 +338,12 @@ cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* s
   if (T == 0) return cudaSuccess;
   const int grid = (T + kEcCombineWarps - 1) / kEcCombineWarps;
   const float4* o4 = reinterpret_cast<const float4*>(o);
+  const dim3 th(kEcCombineWarps * 32);
   if (dtype == MOE_BF16)
-    ec_combine_kernel<true><<<grid, kEcCombineWarps * 32, 0, s>>>(o4, pos, scores, T, d, E, y);
-  else
-    ec_combine_kernel<false><<<grid, kEcCombineWarps * 32, 0, s>>>(o4, pos, scores, T, d, E, y);
-  return cudaGetLastError();
+    return launch_kernel(ec_combine_kernel<true>, dim3(grid), th, 0, s, 1, true, o4, pos, scores, T,
+                         d, E, y);
+  return launch_kernel(ec_combine_kernel<false>, dim3(grid), th, 0, s, 1, true, o4, pos, scores, T,
+                       d, E, y);
 }
 
 }  // namespace moe

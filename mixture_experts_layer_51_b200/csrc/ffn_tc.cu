@@ -93,6 +93,7 @@ struct TcParams {
   int n_tiles;     // column tiles per expert
   int64_t rows;    // rows of the A and output buffers
   int b_chunked;   // 1: B maps are 4-D {64, K, N/64, E}; one load covers a CTA's chunks
+  int out_direct;  // 1: the epilogue stores rows straight to global memory, not by TMA
   const int32_t* offsets;
   const int32_t* kept;
   int32_t* err;
@@ -176,10 +177,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
     fence_async_shared();
   }
-  if (tid < p.E) {
-    c.off[tid] = p.offsets[tid];
-    c.kept[tid] = p.kept[tid];
-  }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
@@ -194,6 +191,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_alloc(smem_u32(&c.tmem_base), TMEM_COLS);
       tmem_relinquish();
     }
+  }
+  // Everything above overlaps the previous kernel's tail; the offsets and
+  // every operand are read only after it has finished.
+  pdl_wait();
+  if (tid < p.E) {
+    c.off[tid] = p.offsets[tid];
+    c.kept[tid] = p.kept[tid];
   }
   __syncthreads();
   if (tid == 0) {
@@ -468,6 +472,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ++nbox;
     };
+    // The same 32 rows x 128 bytes written by each lane straight to global
+    // memory (its own row; rows past the expert's kept rows skipped).
+    auto store_direct = [&](const uint4 (&v)[8], int col0, int row0, int valid_rows, int esz) {
+      if (lane >= valid_rows) return;
+      uint8_t* dst = static_cast<uint8_t*>(p.out) +
+                     (static_cast<int64_t>(row0 + lane) * p.ld_out + col0) * esz;
+      const int vec_elems = 16 / esz;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (col0 + q * vec_elems < p.n_out) reinterpret_cast<uint4*>(dst)[q] = v[q];
+    };
     auto release = [&](int a) {
       tc_fence_before();
       __syncwarp();
@@ -495,6 +510,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int blk_row = m * TILE_M + static_cast<int>(rank) * TM;
       const bool blk_ok = blk_row < c.kept[e];
       const int row0 = c.off[e] + blk_row + quad * 32;
+      const int valid_rows = c.kept[e] - (blk_row + quad * 32);  // rows of this warp's box to keep
       if (EPI == EPI_SWIGLU) {
         const int n0 = n * (TN / 2);
 #pragma unroll 1
@@ -519,7 +535,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               v[q].z = pack_bf16x2(silu_f(gg[4]) * uu[4], silu_f(gg[5]) * uu[5]);
               v[q].w = pack_bf16x2(silu_f(gg[6]) * uu[6], silu_f(gg[7]) * uu[7]);
             }
-            store_box(v, col0, row0);
+            if (p.out_direct)
+              store_direct(v, col0, row0, valid_rows, 2);
+            else
+              store_box(v, col0, row0);
           }
         }
       } else if (EPI == EPI_GELU) {
@@ -544,7 +563,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 v[q].z = pack_bf16x2(gelu_f(gg[4]), gelu_f(gg[5]));
                 v[q].w = pack_bf16x2(gelu_f(gg[6]), gelu_f(gg[7]));
               }
-              store_box(v, col0, row0);
+              if (p.out_direct)
+                store_direct(v, col0, row0, valid_rows, 2);
+              else
+                store_box(v, col0, row0);
             }
           }
         }
@@ -566,7 +588,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int q = 0; q < 8; ++q)
                 v[q] = make_uint4(__float_as_uint(g[b][4 * q + 0]), __float_as_uint(g[b][4 * q + 1]),
                                   __float_as_uint(g[b][4 * q + 2]), __float_as_uint(g[b][4 * q + 3]));
-              store_box(v, col0, row0);
+              if (p.out_direct)
+                store_direct(v, col0, row0, valid_rows, 4);
+              else
+                store_box(v, col0, row0);
             }
           }
         }
@@ -581,6 +606,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   // ---------------------------------------------------------- teardown
+  // The next kernel may launch now (not earlier: its CTAs would sit on the
+  // SMs for the whole of this persistent kernel).
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   if (CG == 2) cluster_sync();  // no CTA leaves while its pair may still touch its memory
@@ -689,19 +717,21 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<EPI, CG, TKS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(groups * CG, 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CG;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ffn_tc_kernel<EPI, CG, TKS>, a, b0, b1, out, p);
+  return launch_kernel(ffn_tc_kernel<EPI, CG, TKS>, dim3(groups * CG), dim3(NUM_THREADS), smem, s,
+                       CG, true, a, b0, b1, out, p);
+}
+
+// How the epilogue writes bf16 outputs (h): MOE_TC_STORE=direct or tma
+// (measurements); fp32 outputs (o) always go through TMA stores.
+int store_mode_env() {
+  static const int mode = [] {
+    const char* v = getenv("MOE_TC_STORE");
+    if (!v) return -1;
+    if (v[0] == 'd') return 1;
+    if (v[0] == 't') return 0;
+    return -1;
+  }();
+  return mode;
 }
 
 // CTA pairs by default; MOE_TC_CTA_PAIR=0 selects one CTA per tile.
@@ -765,6 +795,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.n_tiles = swiglu ? (a.H + TN / 2 - 1) / (TN / 2) : (a.H + TN - 1) / TN;
   up.rows = a.rows;
   up.b_chunked = up_chunked ? 1 : 0;
+  up.out_direct = store_mode_env() == 0 ? 0 : 1;
   up.offsets = a.offsets;
   up.kept = a.kept_counts;
   up.err = a.dev_error;
@@ -785,6 +816,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.n_tiles = (a.d + TN - 1) / TN;
   dn.rows = a.rows;
   dn.b_chunked = dn_chunked ? 1 : 0;
+  dn.out_direct = 0;
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;

@@ -196,12 +196,30 @@ MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, i
   return moe_route_ex(x, Wg, bias, T, d, E, k, dt, nullptr, idx, gate, margin, stream);
 }
 
+namespace {
+moe_status permute_enqueue(const void* x, const int32_t* idx, const int32_t* order,
+                           const int32_t* prior, int32_t T, int32_t d, int32_t E, int32_t k,
+                           int32_t capacity, moe_dtype dt, void* xp, int64_t xp_rows,
+                           int32_t* pos, int32_t* counts, int32_t* kept_counts, int32_t* offsets,
+                           void* ws, size_t ws_bytes, void* stream, bool ticket_zeroed);
+}  // namespace
+
 MOE_API moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order,
                                   const int32_t* prior, int32_t T, int32_t d, int32_t E,
                                   int32_t k, int32_t capacity, moe_dtype dt, void* xp,
                                   int64_t xp_rows, int32_t* pos, int32_t* counts,
                                   int32_t* kept_counts, int32_t* offsets, void* ws,
                                   size_t ws_bytes, void* stream) {
+  return permute_enqueue(x, idx, order, prior, T, d, E, k, capacity, dt, xp, xp_rows, pos, counts,
+                         kept_counts, offsets, ws, ws_bytes, stream, false);
+}
+
+namespace {
+moe_status permute_enqueue(const void* x, const int32_t* idx, const int32_t* order,
+                           const int32_t* prior, int32_t T, int32_t d, int32_t E, int32_t k,
+                           int32_t capacity, moe_dtype dt, void* xp, int64_t xp_rows,
+                           int32_t* pos, int32_t* counts, int32_t* kept_counts, int32_t* offsets,
+                           void* ws, size_t ws_bytes, void* stream, bool ticket_zeroed) {
   if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
   if (!counts || !kept_counts || !offsets) return MOE_ERR_ARG;
   if (T > 0) {
@@ -220,10 +238,11 @@ MOE_API moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32
       static_cast<uint8_t*>(ws) + align_up(nblk * static_cast<size_t>(E) * 4));
   PermuteArgs a{x,      idx,         T,       d,          E,     k,
                 capacity < 0 ? INT32_MAX : capacity, xp, pos, counts, kept_counts, offsets,
-                block_base, ticket, order, prior};
+                block_base, ticket, order, prior, ticket_zeroed};
   return launch_permute(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
                                                                                  : MOE_ERR_CUDA;
 }
+}  // namespace
 
 MOE_API moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d, int32_t E,
                                int32_t k, double cf, moe_dtype dt, void* xp, int64_t xp_rows,
@@ -347,6 +366,13 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
   int32_t* err = reinterpret_cast<int32_t*>(w + L.dev_error);
   if (clear_err && cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess)
     return MOE_ERR_CUDA;
+  // The permutation's completion counter is zeroed here, ahead of the
+  // router, so no memset separates the kernels of the forward (each may
+  // then start while its predecessor drains).
+  const size_t nblk = (static_cast<size_t>(T) + kPermBlock - 1) / kPermBlock;
+  unsigned int* ticket =
+      reinterpret_cast<unsigned int*>(w + L.scratch + align_up(nblk * static_cast<size_t>(E) * 4));
+  if (cudaMemsetAsync(ticket, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
   moe_status st = record_stage(0, s);
   if (st != MOE_OK) return st;
   st = moe_route_ex(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, s);
@@ -362,9 +388,9 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
     if (st != MOE_OK) return st;
     order = reinterpret_cast<const int32_t*>(w + L.order);
   }
-  st = moe_permute_ex(x, idx, order, nullptr, T, d, E, k, moe_capacity(T, E, k, cf), dt, w + L.xp,
-                      L.rows, pos, counts, kept, offsets, w + L.scratch,
-                      permute_scratch_bytes(T, E), s);
+  st = permute_enqueue(x, idx, order, nullptr, T, d, E, k, moe_capacity(T, E, k, cf), dt, w + L.xp,
+                       L.rows, pos, counts, kept, offsets, w + L.scratch,
+                       permute_scratch_bytes(T, E), s, /*ticket_zeroed=*/true);
   if (st == MOE_OK) st = record_stage(2, s);
   if (st != MOE_OK) return st;
   st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,

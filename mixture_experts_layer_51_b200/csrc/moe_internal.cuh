@@ -53,6 +53,16 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+// Programmatic dependent launch.  A kernel launched with
+// launch_kernel(..., pdl = true) may start while the previous kernel in the
+// stream is still running; it must call pdl_wait() before touching anything
+// that kernel (or any earlier stream work) writes.  pdl_trigger() lets the
+// next such kernel launch once every CTA of this one has called it.  Both
+// are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 __device__ __forceinline__ void fence_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -337,6 +347,39 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms);
 
+// Whether kernels of the forward chain are launched with programmatic
+// dependent launch (default on; MOE_PDL=0 turns it off, for measurements).
+bool pdl_enabled();
+
+// cudaLaunchKernelEx with an optional cluster size and, when `pdl` and
+// pdl_enabled(), programmatic stream serialization.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, int cluster, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl && pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 struct PermuteArgs {
   const void* x;
   const int32_t* idx;
@@ -351,6 +394,7 @@ struct PermuteArgs {
   unsigned int* ticket; // scratch counter
   const int32_t* order = nullptr;  // queue order (token at position i), or null
   const int32_t* prior = nullptr;  // per-expert assignments of earlier shards, or null
+  bool ticket_zeroed = false;      // the caller already zeroed *ticket on this stream
 };
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int E, int k, int32_t* counts,
                                  cudaStream_t s);

@@ -28,6 +28,8 @@
 // (queue position i serves token order[i]); rows of an expert block then
 // follow that order.
 
+#include <stdlib.h>
+
 #include <algorithm>
 
 #include "moe_internal.cuh"
@@ -68,6 +70,8 @@ __global__ void __launch_bounds__(kPermBlock)
   __shared__ int wcnt[kWarpsPerBlock][kMaxE];
   __shared__ int padded[kMaxE];
   __shared__ bool is_last;
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = blockIdx.x * kPermBlock + tid;
   const uint64_t mask = i < T ? expert_mask(idx, token_at(order, i, T), T, k, E) : 0ull;
@@ -139,6 +143,8 @@ __global__ void __launch_bounds__(kPermBlock)
                         const int32_t* __restrict__ block_base,
                         const int32_t* __restrict__ offsets, int32_t* __restrict__ pos) {
   __shared__ int wcnt[kWarpsPerBlock][kMaxE];
+  pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int blk = blockIdx.x;
   const int i = blk * kPermBlock + tid;
@@ -184,6 +190,8 @@ __global__ void __launch_bounds__(kCopyWarps * 32)
     row_copy_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ pos, int T,
                     int npos, int dvec, uint4* __restrict__ xp) {
   __shared__ int dst[kCopyWarps][kMaxE];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCopyWarps + warp;
   if (t >= T) return;
@@ -273,17 +281,20 @@ cudaError_t launch_permute(const PermuteArgs& a, moe_dtype dtype, cudaStream_t s
     return err;
   }
   const int nblk = (a.T + kPermBlock - 1) / kPermBlock;
-  cudaError_t err = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned int), s);
-  if (err != cudaSuccess) return err;
+  cudaError_t err = cudaSuccess;
+  if (!a.ticket_zeroed) {
+    err = cudaMemsetAsync(a.ticket, 0, sizeof(unsigned int), s);
+    if (err != cudaSuccess) return err;
+  }
   int32_t* cap = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a.ticket) + 256);
-  permute_count_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.order, a.T, a.E, a.k, a.capacity,
-                                                   a.prior, nblk, a.block_base, a.ticket, cap,
-                                                   a.counts, a.kept_counts, a.offsets);
-  err = cudaGetLastError();
+  err = launch_kernel(permute_count_kernel, dim3(nblk), dim3(kPermBlock), 0, s, 1, true, a.idx,
+                      a.order, a.T, a.E, a.k, a.capacity, a.prior, nblk, a.block_base, a.ticket,
+                      cap, a.counts, a.kept_counts, a.offsets);
   if (err != cudaSuccess) return err;
-  permute_rank_kernel<<<nblk, kPermBlock, 0, s>>>(a.idx, a.order, a.T, a.E, a.k, cap,
-                                                  a.block_base, a.offsets, a.pos);
-  err = cudaGetLastError();
+  err = launch_kernel(permute_rank_kernel, dim3(nblk), dim3(kPermBlock), 0, s, 1, true, a.idx,
+                      a.order, a.T, a.E, a.k, static_cast<const int32_t*>(cap),
+                      static_cast<const int32_t*>(a.block_base),
+                      static_cast<const int32_t*>(a.offsets), a.pos);
   if (err != cudaSuccess) return err;
   return launch_row_copy(a.x, a.pos, a.T, a.k, a.d, dtype, a.xp, s);
 }
@@ -292,9 +303,17 @@ cudaError_t launch_row_copy(const void* x, const int32_t* pos, int T, int npos, 
                             moe_dtype dtype, void* xp, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int dvec = d * (dtype == MOE_BF16 ? 2 : 4) / 16;
-  row_copy_kernel<<<(T + kCopyWarps - 1) / kCopyWarps, kCopyWarps * 32, 0, s>>>(
-      static_cast<const uint4*>(x), pos, T, npos, dvec, static_cast<uint4*>(xp));
-  return cudaGetLastError();
+  return launch_kernel(row_copy_kernel, dim3((T + kCopyWarps - 1) / kCopyWarps),
+                       dim3(kCopyWarps * 32), 0, s, 1, true, static_cast<const uint4*>(x), pos, T,
+                       npos, dvec, static_cast<uint4*>(xp));
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 }  // namespace moe

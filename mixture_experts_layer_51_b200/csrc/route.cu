@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int kc_end = (static_cast<int>(q) + 1) * nk_all / CL;
   const int nk = kc_end - kc_begin;
   const bool vec_wg = (E % 8) == 0;
+  pdl_wait();
+  pdl_trigger();
 
   auto x_tile = [&](int st) { return smem + st * SB; };
   auto w_tile = [&](int st) { return smem + st * SB + BM * XS * 2; };
@@ -459,21 +461,10 @@ cudaError_t launch_route_cfg(const RouteArgs& a, cudaStream_t s) {
   auto kern = route_bf16_kernel<NT, BM, BK, STAGES, CL, KM>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(((a.T + BM - 1) / BM) * CL);
-  cfg.blockDim = dim3(kRouteThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(a.x),
-                            static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T, a.d, a.E, a.k,
-                            a.idx, a.gate, a.margin, a.gating, a.gate_scale, a.scores);
+  return launch_kernel(kern, dim3(((a.T + BM - 1) / BM) * CL), dim3(kRouteThreads), smem, s, CL,
+                       true, static_cast<const __nv_bfloat16*>(a.x),
+                       static_cast<const __nv_bfloat16*>(a.Wg), a.bias, a.T, a.d, a.E, a.k, a.idx,
+                       a.gate, a.margin, a.gating, a.gate_scale, a.scores);
 }
 
 // CTAs per token tile: the largest of 1, 2, 4 that keeps the grid within

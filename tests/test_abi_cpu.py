@@ -216,3 +216,16 @@ def test_expert_choice_sizes_and_validation(lib):
     assert lib.moe_forward_expert_choice(fake, fake, None, fake, fake, fake, 64, 64, 64, 8, 2,
                                          1.0, M.MOE_SWIGLU, M.MOE_BF16, fake, fake, 16, None,
                                          None) == M.MOE_ERR_ARG
+
+
+def test_pipeline_arguments_are_checked_before_any_cuda_call(lib):
+    h = ctypes.c_void_p()
+    assert lib.moe_pipeline_create(0, ctypes.byref(h)) == M.MOE_ERR_ARG
+    assert lib.moe_pipeline_create(M.MOE_PIPELINE_MAX_DEPTH + 1, ctypes.byref(h)) == M.MOE_ERR_ARG
+    assert lib.moe_pipeline_create(2, None) == M.MOE_ERR_ARG
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.moe_pipeline_submit(None, 0, fake, fake, fake, fake, fake, None, fake, fake, fake,
+                                   64, 64, 64, 8, 2, 0.0, M.MOE_SWIGLU, M.MOE_BF16, None, fake,
+                                   1 << 20, None) == M.MOE_ERR_ARG
+    assert lib.moe_pipeline_wait(None, 0) == M.MOE_ERR_ARG
+    assert lib.moe_pipeline_destroy(None) == M.MOE_OK
