@@ -93,7 +93,6 @@ struct TcParams {
   int n_tiles;     // column tiles per expert
   int64_t rows;    // rows of the A and output buffers
   int b_chunked;   // 1: B maps are 4-D {64, K, N/64, E}; one load covers a CTA's chunks
-  int out_direct;  // 1: the epilogue stores rows straight to global memory, not by TMA
   const int32_t* offsets;
   const int32_t* kept;
   int32_t* err;
@@ -439,21 +438,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue
-    // Each warp drains its 32 TMEM lanes (tile rows) in batches of 32-column
-    // loads, applies the activation, writes 128-byte rows into a swizzled
-    // 32-row staging box and lets one TMA store per box carry it to global
-    // memory (whole lines, asynchronous; two boxes per warp alternate).  The
-    // accumulator is released as soon as its last batch is in registers.
-    // Rows of a box past the expert's kept rows are padding rows of the same
-    // expert block (never read as results); a CTA whose 128-row block starts
-    // past the kept rows stores nothing.
+    // Each warp drains its 32 TMEM lanes (tile rows), applies the
+    // activation and stores; the accumulator is released as soon as its last
+    // columns are in registers.  bf16 outputs (h): each lane writes its own
+    // row.  fp32 outputs (o): four 32-column loads per wait, then 128-byte
+    // rows go into a swizzled 32-row staging box in shared memory and one
+    // TMA store per box carries it to global memory (whole lines,
+    // asynchronous; two boxes per warp alternate) -- per-row 16-byte stores
+    // half-fill every sector and throttled the down projection of short-K
+    // layers.  Rows of a box past the expert's kept rows are padding rows of
+    // the same expert block (never read as results); a CTA whose 128-row
+    // block starts past the kept rows stores nothing.
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
     const uint32_t obuf0 = smem_base + STAGES * STAGE_BYTES + quad * 2 * OUT_BOX_BYTES;
     uint8_t* const obuf0_p = smem + STAGES * STAGE_BYTES + quad * 2 * OUT_BOX_BYTES;
     int nbox = 0;
-    // The outputs (h, o) are far larger than L2 and are not read again by
-    // this kernel: their lines go first, so the weight and activation tiles
-    // that other CTAs still read stay resident.
+    // o is far larger than L2 and not read again by this kernel: its lines
+    // go first, so the weight and activation tiles other CTAs still read
+    // stay resident.
     const uint64_t out_policy = make_policy_evict_first();
     // Stages this lane's 8 x 16 bytes as row `lane` of the next box and
     // issues its store at (col0, row0).
@@ -471,17 +473,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bulk_commit();
       }
       ++nbox;
-    };
-    // The same 32 rows x 128 bytes written by each lane straight to global
-    // memory (its own row; rows past the expert's kept rows skipped).
-    auto store_direct = [&](const uint4 (&v)[8], int col0, int row0, int valid_rows, int esz) {
-      if (lane >= valid_rows) return;
-      uint8_t* dst = static_cast<uint8_t*>(p.out) +
-                     (static_cast<int64_t>(row0 + lane) * p.ld_out + col0) * esz;
-      const int vec_elems = 16 / esz;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (col0 + q * vec_elems < p.n_out) reinterpret_cast<uint4*>(dst)[q] = v[q];
     };
     auto release = [&](int a) {
       tc_fence_before();
@@ -511,62 +502,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool blk_ok = blk_row < c.kept[e];
       const int row0 = c.off[e] + blk_row + quad * 32;
       const int valid_rows = c.kept[e] - (blk_row + quad * 32);  // rows of this warp's box to keep
-      if (EPI == EPI_SWIGLU) {
-        const int n0 = n * (TN / 2);
+      if (EPI == EPI_SWIGLU || EPI == EPI_GELU) {
+        // bf16 output (h): one 32-column chunk per TMEM wait, each lane
+        // storing its own row's 64 bytes.  (Loading several chunks per wait
+        // made this epilogue slower than the MMAs of a short tile: the
+        // up projection of the 1024-wide layer lost 40%.)
+        const int n0 = EPI == EPI_SWIGLU ? n * (TN / 2) : n * TN;
+        constexpr int NCH = EPI == EPI_SWIGLU ? 4 : TN / 32;
+        const bool row_ok = blk_ok && lane < valid_rows;
+        __nv_bfloat16* dst_row =
+            static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row0 + lane) * p.ld_out;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 4; c0 += 2) {
-          float g[2][32], u[2][32];
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            tc_ld_32cols(tbase + (c0 + b) * 32, g[b]);
-            tc_ld_32cols(tbase + TN / 2 + (c0 + b) * 32, u[b]);
-          }
+        for (int cc = 0; cc < NCH; ++cc) {
+          float g[32], u[32];
+          tc_ld_32cols(tbase + cc * 32, g);
+          if (EPI == EPI_SWIGLU) tc_ld_32cols(tbase + TN / 2 + cc * 32, u);
           tc_wait_ld();
-          if (c0 + 2 == 4) release(acc);
-          const int col0 = n0 + c0 * 32;
-          if (blk_ok && col0 < p.n_out) {
-            uint4 v[8];
+          if (cc == NCH - 1) release(acc);
+          if (row_ok) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float* gg = g[q >> 2] + (q & 3) * 8;
-              const float* uu = u[q >> 2] + (q & 3) * 8;
-              v[q].x = pack_bf16x2(silu_f(gg[0]) * uu[0], silu_f(gg[1]) * uu[1]);
-              v[q].y = pack_bf16x2(silu_f(gg[2]) * uu[2], silu_f(gg[3]) * uu[3]);
-              v[q].z = pack_bf16x2(silu_f(gg[4]) * uu[4], silu_f(gg[5]) * uu[5]);
-              v[q].w = pack_bf16x2(silu_f(gg[6]) * uu[6], silu_f(gg[7]) * uu[7]);
-            }
-            if (p.out_direct)
-              store_direct(v, col0, row0, valid_rows, 2);
-            else
-              store_box(v, col0, row0);
-          }
-        }
-      } else if (EPI == EPI_GELU) {
-        const int n0 = n * TN;
-#pragma unroll 1
-        for (int c0 = 0; c0 < TN / 32; c0 += 4) {
-          float g[4][32];
+            for (int v = 0; v < 4; ++v) {
+              const int col = n0 + cc * 32 + v * 8;
+              if (col < p.n_out) {
+                float r[8];
 #pragma unroll
-          for (int b = 0; b < 4; ++b) tc_ld_32cols(tbase + (c0 + b) * 32, g[b]);
-          tc_wait_ld();
-          if (c0 + 4 == TN / 32) release(acc);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int col0 = n0 + c0 * 32 + h * 64;
-            if (blk_ok && col0 < p.n_out) {
-              uint4 v[8];
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float* gg = g[2 * h + (q >> 2)] + (q & 3) * 8;
-                v[q].x = pack_bf16x2(gelu_f(gg[0]), gelu_f(gg[1]));
-                v[q].y = pack_bf16x2(gelu_f(gg[2]), gelu_f(gg[3]));
-                v[q].z = pack_bf16x2(gelu_f(gg[4]), gelu_f(gg[5]));
-                v[q].w = pack_bf16x2(gelu_f(gg[6]), gelu_f(gg[7]));
+                for (int i = 0; i < 8; ++i)
+                  r[i] = EPI == EPI_SWIGLU ? silu_f(g[v * 8 + i]) * u[v * 8 + i]
+                                           : gelu_f(g[v * 8 + i]);
+                uint4 pk;
+                pk.x = pack_bf16x2(r[0], r[1]);
+                pk.y = pack_bf16x2(r[2], r[3]);
+                pk.z = pack_bf16x2(r[4], r[5]);
+                pk.w = pack_bf16x2(r[6], r[7]);
+                *reinterpret_cast<uint4*>(dst_row + col) = pk;
               }
-              if (p.out_direct)
-                store_direct(v, col0, row0, valid_rows, 2);
-              else
-                store_box(v, col0, row0);
             }
           }
         }
@@ -588,10 +557,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int q = 0; q < 8; ++q)
                 v[q] = make_uint4(__float_as_uint(g[b][4 * q + 0]), __float_as_uint(g[b][4 * q + 1]),
                                   __float_as_uint(g[b][4 * q + 2]), __float_as_uint(g[b][4 * q + 3]));
-              if (p.out_direct)
-                store_direct(v, col0, row0, valid_rows, 4);
-              else
-                store_box(v, col0, row0);
+              store_box(v, col0, row0);
             }
           }
         }
@@ -721,19 +687,6 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
                        CG, true, a, b0, b1, out, p);
 }
 
-// How the epilogue writes bf16 outputs (h): MOE_TC_STORE=direct or tma
-// (measurements); fp32 outputs (o) always go through TMA stores.
-int store_mode_env() {
-  static const int mode = [] {
-    const char* v = getenv("MOE_TC_STORE");
-    if (!v) return -1;
-    if (v[0] == 'd') return 1;
-    if (v[0] == 't') return 0;
-    return -1;
-  }();
-  return mode;
-}
-
 // CTA pairs by default; MOE_TC_CTA_PAIR=0 selects one CTA per tile.
 bool use_cta_pairs() {
   static const bool pairs = [] {
@@ -795,7 +748,6 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.n_tiles = swiglu ? (a.H + TN / 2 - 1) / (TN / 2) : (a.H + TN - 1) / TN;
   up.rows = a.rows;
   up.b_chunked = up_chunked ? 1 : 0;
-  up.out_direct = store_mode_env() == 0 ? 0 : 1;
   up.offsets = a.offsets;
   up.kept = a.kept_counts;
   up.err = a.dev_error;
@@ -816,7 +768,6 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.n_tiles = (a.d + TN - 1) / TN;
   dn.rows = a.rows;
   dn.b_chunked = dn_chunked ? 1 : 0;
-  dn.out_direct = 0;
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
