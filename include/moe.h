@@ -29,7 +29,8 @@
  * - Element types: MOE_BF16 means x, W_g, W1, W3, W2, xp, h and y are bf16;
  *   MOE_FP32 means they are fp32.  Router bias, gates, margins and the
  *   expert output `o` are always fp32; indices and counts are int32.
- * - Limits: 1 <= k <= E <= 64, k <= 8, d % 8 == 0, H % 8 == 0, T >= 0.
+ * - Limits: 1 <= k <= E <= 64, k <= 8, d % 8 == 0, H % 8 == 0, T >= 0, and
+ *   at most 2^31 - 1 permuted rows (int32 row indices on the device).
  *   T == 0 is valid and does nothing.  Pointers must be 16-byte aligned.
  * - Errors: arguments are checked on the host before anything is enqueued;
  *   a bad argument returns MOE_ERR_ARG and enqueues nothing.  A failed CUDA

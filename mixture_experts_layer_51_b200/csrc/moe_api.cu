@@ -90,7 +90,8 @@ bool compute_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, doubl
       !valid_act(act))
     return false;
   const int64_t rows = moe_max_permuted_rows(T, E, k, cf);
-  if (rows < 0) return false;
+  // Row indices, offsets and positions are int32 on the device.
+  if (rows < 0 || rows > INT32_MAX) return false;
   const size_t tk = static_cast<size_t>(T) * k;
   const size_t es = elt_size(dt);
   size_t off = 0;
@@ -226,7 +227,8 @@ moe_status permute_enqueue(const void* x, const int32_t* idx, const int32_t* ord
     if (!x || !idx || !xp || !pos || !ws || !aligned16(x) || !aligned16(xp) ||
         !aligned16(ws))
       return MOE_ERR_ARG;
-    if (xp_rows < moe_rows_for_capacity(T, E, k, capacity)) return MOE_ERR_ARG;
+    const int64_t need_rows = moe_rows_for_capacity(T, E, k, capacity);
+    if (need_rows > INT32_MAX || xp_rows < need_rows) return MOE_ERR_ARG;
     if (ws_bytes < permute_scratch_bytes(T, E)) return MOE_ERR_ARG;
   }
   DeviceInfo di;
@@ -303,7 +305,7 @@ MOE_API moe_status moe_grouped_ffn(const void* xp, int64_t rows, const int32_t* 
                                    moe_dtype dt, void* h, float* o, int32_t* dev_error,
                                    void* stream) {
   if (!valid_ffn_sizes(d, H) || E < 1 || E > kMaxE || !valid_act(act) || !valid_dtype(dt) ||
-      rows < 0 || rows % kRowAlign != 0)
+      rows < 0 || rows > INT32_MAX || rows % kRowAlign != 0)
     return MOE_ERR_ARG;
   if (rows == 0) return MOE_OK;
   if (!xp || !offsets || !kept_counts || !W1 || !W2 || !h || !o || !dev_error) return MOE_ERR_ARG;
@@ -717,6 +719,7 @@ bool ec_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, double cf,
   if (n < 0) return false;
   const int64_t npad = pad_rows(n);
   const int64_t rows = static_cast<int64_t>(E) * npad;
+  if (rows > INT32_MAX || static_cast<int64_t>(T) * E > INT32_MAX) return false;
   const size_t es = elt_size(dt);
   const size_t te = static_cast<size_t>(T) * E;
   size_t off = 0;

@@ -229,3 +229,12 @@ def test_pipeline_arguments_are_checked_before_any_cuda_call(lib):
                                    1 << 20, None) == M.MOE_ERR_ARG
     assert lib.moe_pipeline_wait(None, 0) == M.MOE_ERR_ARG
     assert lib.moe_pipeline_destroy(None) == M.MOE_OK
+
+
+def test_sizes_past_int32_rows_are_rejected(lib):
+    """Rows, offsets and positions are int32 on the device: a layout whose
+    permuted buffer would pass 2^31 rows is refused (workspace size 0)."""
+    assert M.moe_workspace_bytes(300_000_000, 64, 64, 64, 8, 0.0, "bf16", "swiglu") == 0
+    assert M.moe_workspace_bytes(1_000_000, 64, 64, 64, 8, 0.0, "bf16", "swiglu") > 0
+    assert lib.moe_expert_choice_workspace_bytes(40_000_000, 64, 64, 64, 8, 1.0, M.MOE_BF16,
+                                                 M.MOE_SWIGLU) == 0
