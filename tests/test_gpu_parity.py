@@ -313,3 +313,35 @@ def test_largest_expert_count_and_top_k(cf):
     y_ref, _ = oracle.moe_forward_tokens(cpu["x"][sample], logits[sample], g["idx"][sample],
                                          kept[sample], cpu["W1"], cpu["W3"], cpu["W2"], w.act)
     assert_y_close(g["y"][sample], y_ref, w.dtype)
+
+
+def test_batch_priority_routing_full_size_openmoe():
+    """Batch Priority Routing on the full OpenMoE-shaped batch (16384 tokens,
+    E = 32, capacity 1024): the device order equals the oracle's stable
+    argsort of the device gates, every position is bit-exact, and sampled
+    outputs meet the tolerance; the dropped tokens are the least important
+    at every expert."""
+    w = WORKLOADS["openmoe_skew_bf16"]
+    inp = make_inputs(w, "cuda")
+    g = run_gpu(w, inp, priority="gate")
+    assert int(g["dev_error"][0]) == 0
+    cpu = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    logits = oracle.router_logits(cpu["x"], cpu["Wg"], cpu["bias"])
+    check_routing(g, logits, w.k)
+    kept, C = check_permutation(g, None, w.T, w.E, w.k, w.cf, priority="gate")
+    assert not kept.all()
+    prio = g["gate"][:, 0]
+    for e in range(w.E):
+        pk = prio[np.nonzero((g["idx"] == e) & kept)[0]]
+        pd = prio[np.nonzero((g["idx"] == e) & ~kept)[0]]
+        if pk.size and pd.size:
+            assert pd.max() <= pk.min()
+    rng = np.random.default_rng(5)
+    sample = np.unique(np.concatenate([[0, w.T - 1], rng.choice(w.T, 64, replace=False)]))
+    experts = np.unique(g["idx"][sample])
+    W1 = {int(e): cpu["W1"][int(e)] for e in experts}
+    W3 = {int(e): cpu["W3"][int(e)] for e in experts}
+    W2 = {int(e): cpu["W2"][int(e)] for e in experts}
+    y_ref, _ = oracle.moe_forward_tokens(cpu["x"][sample], logits[sample], g["idx"][sample],
+                                         kept[sample], W1, W3, W2, w.act)
+    assert_y_close(g["y"][sample], y_ref, w.dtype)
