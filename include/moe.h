@@ -372,7 +372,8 @@ moe_status moe_set_stage_events(void* const* events);
  * a fixed number of tokens, so a token may be processed by no expert, by
  * several, or by all.  Here the affinity of token t to expert e is the
  * router probability S[t, e] = Softmax(x_t . W_g (+ bias))_e over all E
- * experts ("How do Mixture of Expert Models Work?", "The Math Behind MoEs");
+ * experts ("How do Mixture of Expert Models Work?", "The Math Behind MoEs"),
+ * stored expert-major (scores[e * T + t] = S[t, e]);
  * expert e takes the n = min(C, T) tokens with the largest S[:, e]
  * (C = moe_capacity(T, E, k, cf), k read as the average number of experts
  * per token; equal affinities -> lower position first), and
@@ -385,16 +386,17 @@ moe_status moe_set_stage_events(void* const* events);
  * positive number (expert choice has no dropless form) or sizes are invalid. */
 int32_t moe_expert_choice_tokens(int32_t T, int32_t E, int32_t k, double capacity_factor);
 
-/* scores [T, E] fp32 (device) = softmax over all E logits of every token.
- * Sizes as moe_route (no k). */
+/* scores [E, T] fp32 (device, expert-major: scores[e * T + t]) = softmax
+ * over all E logits of token t.  Sizes as moe_route (no k). */
 moe_status moe_expert_choice_route(const void* x, const void* Wg, const float* bias, int32_t T,
                                    int32_t d, int32_t E, moe_dtype dtype, float* scores,
                                    void* stream);
 
-/* Scratch bytes for moe_expert_choice_select (a transposed key copy, T*E*4). */
+/* Scratch bytes for moe_expert_choice_select (expert-major positions, T*E*4). */
 size_t moe_expert_choice_select_workspace_bytes(int32_t T, int32_t E);
 
-/* Each expert's choice of n tokens (0 <= n <= T).  Outputs (device):
+/* Each expert's choice of n tokens (0 <= n <= T) from scores [E, T].
+ * Outputs (device):
  * tok [E, n] int32 (expert e's tokens, ascending position), pos [T, E]
  * int32 (row in xp, or -1), kept_counts [E] (= n), offsets [E + 1]
  * (= e * npad).  Deterministic: the selection and the row order follow
@@ -412,7 +414,7 @@ moe_status moe_expert_choice_permute(const void* x, const int32_t* pos, int32_t 
                                      int64_t xp_rows, void* stream);
 
 /* y [T, d] (dtype) = sum over e with pos[t, e] >= 0, ascending e, of
- * scores[t, e] * o[pos[t, e]] (o fp32 from moe_grouped_ffn), fp32
+ * scores[e, t] * o[pos[t, e]] (o fp32 from moe_grouped_ffn), fp32
  * accumulation, one rounding.  Every y row is written. */
 moe_status moe_expert_choice_combine(const float* o, const int32_t* pos, const float* scores,
                                      int32_t T, int32_t d, int32_t E, moe_dtype dtype, void* y,
@@ -420,7 +422,7 @@ moe_status moe_expert_choice_combine(const float* o, const int32_t* pos, const f
 
 /* Byte offsets inside the moe_forward_expert_choice workspace. */
 typedef struct {
-  size_t scores;       /* fp32  [T, E]  affinities                         */
+  size_t scores;       /* fp32  [E, T]  affinities (expert-major)          */
   size_t pos;          /* int32 [T, E]  row in xp/h/o, or -1               */
   size_t tok;          /* int32 [E, n]  each expert's tokens               */
   size_t kept_counts;  /* int32 [E]     (= n)                              */

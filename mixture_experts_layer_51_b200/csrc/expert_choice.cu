@@ -7,18 +7,20 @@
 // affinity an expert ranks tokens by is the router probability
 // Softmax(x . W_g) over all experts ("How do Mixture of Expert Models
 // Work?", "The Math Behind MoEs"), computed by the router kernel
-// (RouteArgs::scores).  Each expert takes n = min(C, T) tokens,
+// (RouteArgs::scores) as an expert-major [E, T] matrix.  Each expert takes n = min(C, T) tokens,
 // C = ceil(cf * T * k / E); equal affinities go to the lower position.
 //
 // Kernels here:
 //   ec_select_kernel   a cluster of CTAs per expert: radix select of the n-th
-//                      largest affinity in its column (4 passes of 8 bits
-//                      over order-preserving 32-bit keys, histograms merged
-//                      through distributed shared memory), then one ordered
-//                      pass that marks the chosen tokens and ranks them in
-//                      position order (CTA-wide ballot scans, slice offsets
-//                      from the cluster) -- writes the expert's token list
-//                      and pos[t, e].
+//                      largest affinity in its (contiguous, expert-major)
+//                      column (4 passes of 8 bits over order-preserving
+//                      32-bit keys, histograms merged through distributed
+//                      shared memory), then one ordered pass that marks the
+//                      chosen tokens and ranks them in position order
+//                      (CTA-wide ballot scans, slice offsets from the
+//                      cluster) -- writes the expert's token list and its
+//                      row of positions, pos_t[e, t];
+//   ec_transpose_kernel  pos [T, E] from pos_t, through shared memory.
 // The chosen x rows are copied by the token-major row copy of the
 // permutation (read once, written once per expert that took the token).
 //   ec_combine_kernel  one warp per token: y_t = sum over the experts that
@@ -79,11 +81,13 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
     atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
 }
 
+// scores: [E, T] (expert-major: each expert's column is contiguous).
+// pos_t: [E, T] (expert-major) positions; ec_transpose_kernel turns them
+// into the token-major pos [T, E] the copy and the combine read.
 __global__ void __launch_bounds__(kSelThreads)
     ec_select_kernel(const float* __restrict__ scores, int T, int E, int n, int npad,
-                     uint32_t* __restrict__ keys_t, int32_t* __restrict__ tok,
-                     int32_t* __restrict__ pos, int32_t* __restrict__ kept_counts,
-                     int32_t* __restrict__ offsets) {
+                     int32_t* __restrict__ pos_t, int32_t* __restrict__ tok,
+                     int32_t* __restrict__ kept_counts, int32_t* __restrict__ offsets) {
   __shared__ uint32_t hist[2][256];  // alternate passes, so one cluster barrier per pass
   __shared__ uint32_t tot[256];      // cluster-wide histogram of the current pass
   __shared__ int slice_cnt[2];       // this slice's keys below the cut and equal to it
@@ -97,21 +101,17 @@ __global__ void __launch_bounds__(kSelThreads)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (T + kSelCta - 1) / kSelCta;
   const int t_begin = min(T, static_cast<int>(r) * per), t_end = min(T, t_begin + per);
-  uint32_t* keys = keys_t + (int64_t)e * T;
+  const float* col = scores + (int64_t)e * T;  // this expert's affinities, contiguous
+  auto key_at = [&](int t) { return desc_key(__ldg(col + t)); };
 
   for (int i = tid; i < 512; i += kSelThreads) (&hist[0][0])[i] = 0;
   __syncthreads();
-  // The slice of the affinity column as keys (a strided read of [T, E]; the
-  // transposed copy makes the later passes contiguous) and the histogram of
-  // the top byte.  All lanes run the same trip count for the warp votes.
+  // The histogram of the keys' top byte over this slice.  All lanes run the
+  // same trip count for the warp votes.
   for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
     const int t = b0 + tid;
     uint32_t bin = 256u;
-    if (t < t_end) {
-      const uint32_t key = desc_key(scores[(int64_t)t * E + e]);
-      keys[t] = key;
-      bin = key >> 24;
-    }
+    if (t < t_end) bin = key_at(t) >> 24;
     hist_add(hist[0], bin);
   }
 
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kSelThreads)
         const int t = b0 + tid;
         uint32_t bin = 256u;
         if (t < t_end) {
-          const uint32_t key = keys[t];
+          const uint32_t key = key_at(t);
           if ((key >> (shift + 8)) == (prefix >> (shift + 8))) bin = (key >> shift) & 255u;
         }
         hist_add(h, bin);
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kSelThreads)
   // counts of the lower slices give this slice's starting ranks.
   int lt_n = 0, eq_n = 0;
   for (int t = t_begin + tid; t < t_end; t += kSelThreads) {
-    const uint32_t key = keys[t];
+    const uint32_t key = key_at(t);
     lt_n += (n > 0 && key < prefix);
     eq_n += (n > 0 && key == prefix);
   }
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kSelThreads)
   int carry_eq = eq_before, carry_sel = row_before;
   for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
     const int t = b0 + tid;
-    const uint32_t key = t < t_end ? keys[t] : 0xffffffffu;
+    const uint32_t key = t < t_end ? key_at(t) : 0xffffffffu;
     const bool eq = n > 0 && t < t_end && key == prefix;
     const bool lt = n > 0 && t < t_end && key < prefix;
     int tot_eq, tot_sel;
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kSelThreads)
     const bool chosen = lt || (eq && eq_rank < need);
     const int row = carry_sel + cta_exclusive_scan(chosen, wsum_b, &tot_sel);
     if (t < t_end) {
-      pos[(int64_t)t * E + e] = chosen ? row0 + row : -1;
+      pos_t[(int64_t)e * T + t] = chosen ? row0 + row : -1;
       if (chosen) tok[(int64_t)e * n + row] = t;
     }
     carry_eq += tot_eq;
@@ -244,6 +244,27 @@ __global__ void __launch_bounds__(kSelThreads)
   if (r == 0 && tid == 0) kept_counts[e] = n;
   if (blockIdx.x == 0)
     for (int i = tid; i <= E; i += kSelThreads) offsets[i] = i * npad;
+}
+
+// pos [T, E] from pos_t [E, T], through a 32 x 64 shared-memory tile:
+// reads run along tokens, writes along experts.
+constexpr int kTrE = 32, kTrT = 64;
+__global__ void __launch_bounds__(256)
+    ec_transpose_kernel(const int32_t* __restrict__ pos_t, int T, int E,
+                        int32_t* __restrict__ pos) {
+  __shared__ int32_t tile[kTrE][kTrT + 1];
+  pdl_wait();
+  pdl_trigger();
+  const int t0 = blockIdx.x * kTrT, e0 = blockIdx.y * kTrE;
+  for (int i = threadIdx.x; i < kTrE * kTrT; i += 256) {
+    const int el = i / kTrT, tl = i - el * kTrT;
+    if (e0 + el < E && t0 + tl < T) tile[el][tl] = pos_t[(int64_t)(e0 + el) * T + t0 + tl];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kTrE * kTrT; i += 256) {
+    const int tl = i / kTrE, el = i - tl * kTrE;
+    if (e0 + el < E && t0 + tl < T) pos[(int64_t)(t0 + tl) * E + e0 + el] = tile[el][tl];
+  }
 }
 
 constexpr int kEcCombineWarps = 8;
@@ -269,7 +290,7 @@ __global__ void __launch_bounds__(kEcCombineWarps * 32)
     if (p >= 0) {
       const int i = nsel + __popc(b & ((1u << lane) - 1u));
       sp[warp][i] = p;
-      sg[warp][i] = scores[(int64_t)t * E + e];
+      sg[warp][i] = scores[(int64_t)e * T + t];
     }
     nsel += __popc(b);
   }
@@ -328,9 +349,13 @@ size_t ec_select_scratch_bytes(int T, int E) {
 cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad, void* scratch,
                              int32_t* tok, int32_t* pos, int32_t* kept_counts, int32_t* offsets,
                              cudaStream_t s) {
-  return launch_kernel(ec_select_kernel, dim3(E * kSelCta), dim3(kSelThreads), 0, s, kSelCta, true,
-                       scores, T, E, n, npad, static_cast<uint32_t*>(scratch), tok, pos,
-                       kept_counts, offsets);
+  int32_t* pos_t = static_cast<int32_t*>(scratch);
+  cudaError_t err = launch_kernel(ec_select_kernel, dim3(E * kSelCta), dim3(kSelThreads), 0, s,
+                                  kSelCta, true, scores, T, E, n, npad, pos_t, tok, kept_counts,
+                                  offsets);
+  if (err != cudaSuccess) return err;
+  return launch_kernel(ec_transpose_kernel, dim3((T + kTrT - 1) / kTrT, (E + kTrE - 1) / kTrE),
+                       dim3(256), 0, s, 1, true, static_cast<const int32_t*>(pos_t), T, E, pos);
 }
 
 cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,

@@ -343,7 +343,7 @@ struct RouteArgs {
   float* margin;
   int gating;        // moe_gating
   float gate_scale;  // multiplies every gate
-  float* scores = nullptr;  // non-null: write softmax over all E to [T, E] instead of TopK
+  float* scores = nullptr;  // non-null: write softmax over all E to [E, T] instead of TopK
 };
 cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms);
 

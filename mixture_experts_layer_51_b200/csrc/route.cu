@@ -326,8 +326,22 @@ __global__ void __launch_bounds__(kRouteThreads)
 #pragma unroll
     for (int o = P / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv = 1.f / sum;
-    if (t < T)
-      for (int e = p; e < E; e += P) scores[(int64_t)t * E + e] = expf(lrow[e] - m) * inv;
+    // Expert-major output scores[e, t]: the tile is written with consecutive
+    // threads on consecutive tokens, each value recomputed from the same
+    // logit, maximum and reciprocal as the sum used.
+    float* rowstat = fin + TPC * LS;  // [TPC][2]: max, 1/sum
+    if (p == 0) {
+      rowstat[2 * rr] = m;
+      rowstat[2 * rr + 1] = inv;
+    }
+    __syncthreads();
+    const int t_base = t0 + static_cast<int>(q) * TPC;
+    for (int i = tid; i < TPC * E; i += kRouteThreads) {
+      const int e = i / TPC, r2 = i - e * TPC;
+      if (t_base + r2 < T)
+        scores[(int64_t)e * T + t_base + r2] =
+            expf(fin[r2 * LS + e] - rowstat[2 * r2]) * rowstat[2 * r2 + 1];
+    }
     return;
   }
   // This thread's experts [e_lo, e_hi), then the butterfly merge.
@@ -447,7 +461,7 @@ __global__ void __launch_bounds__(256)
     float sum = 0.f;
     for (int e = 0; e < E; ++e) sum += expf(get(e) - m);
     const float inv = 1.f / sum;
-    for (int e = lane; e < E; e += 32) scores[(int64_t)t * E + e] = expf(get(e) - m) * inv;
+    for (int e = lane; e < E; e += 32) scores[(int64_t)e * T + t] = expf(get(e) - m) * inv;
     return;
   }
   if (lane == 0) topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
@@ -457,7 +471,7 @@ template <int NT, int BM, int BK, int STAGES, int CL, int KM>
 cudaError_t launch_route_cfg(const RouteArgs& a, cudaStream_t s) {
   constexpr int smem = STAGES * stage_bytes(NT, BM, BK);
   constexpr int TPC = BM / CL;
-  static_assert((BM + TPC) * (NT * 8 + 1) * 4 <= smem, "epilogue buffers");
+  static_assert((BM + TPC) * (NT * 8 + 1) * 4 + TPC * 8 <= smem, "epilogue buffers");
   auto kern = route_bf16_kernel<NT, BM, BK, STAGES, CL, KM>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;

@@ -568,11 +568,12 @@ def moe_expert_choice_tokens(T, E, k, capacity_factor):
 
 
 def moe_expert_choice_route(x, Wg, bias, scores=None, stream=None):
-    """Affinities [T, E] fp32: softmax over all E logits of every token."""
+    """Affinities, expert-major [E, T] fp32: scores[e, t] = softmax over the
+    E logits of token t, at expert e."""
     T, d = x.shape
     E = Wg.shape[1]
     dev = x.device
-    scores = scores if scores is not None else torch.empty((T, E), dtype=torch.float32, device=dev)
+    scores = scores if scores is not None else torch.empty((E, T), dtype=torch.float32, device=dev)
     _check(lib().moe_expert_choice_route(_ptr(x), _ptr(Wg), _ptr(bias), T, d, E, _dtype_code(x),
                                          _ptr(scores), _stream(dev, stream)),
            "moe_expert_choice_route")
@@ -580,8 +581,9 @@ def moe_expert_choice_route(x, Wg, bias, scores=None, stream=None):
 
 
 def moe_expert_choice_select(scores, n, stream=None):
-    """Each expert's n tokens: tok [E, n], pos [T, E], kept_counts, offsets."""
-    T, E = scores.shape
+    """Each expert's n tokens from scores [E, T]: tok [E, n], pos [T, E],
+    kept_counts, offsets."""
+    E, T = scores.shape
     dev = scores.device
     tok = torch.empty((E, max(n, 0)), dtype=torch.int32, device=dev)
     pos = torch.empty((T, E), dtype=torch.int32, device=dev)
@@ -661,7 +663,7 @@ class ExpertChoiceLayer:
             nbytes = count * torch.empty((), dtype=dt).element_size()
             return ws[off:off + nbytes].view(dt)
         return dict(
-            scores=view(L.scores, T * self.E, torch.float32).view(T, self.E),
+            scores=view(L.scores, T * self.E, torch.float32).view(self.E, T),
             pos=view(L.pos, T * self.E, torch.int32).view(T, self.E),
             tok=view(L.tok, self.E * L.n, torch.int32).view(self.E, L.n),
             kept_counts=view(L.kept_counts, self.E, torch.int32),

@@ -56,7 +56,7 @@ def _check(w, inp):
     n = M.moe_expert_choice_tokens(w.T, w.E, w.k, w.cf)
     assert n == min(w.T, oracle.capacity(w.T, w.E, w.k, w.cf))
     assert st.device_error == 0 and v["n"] == n
-    S_gpu = to_np(v["scores"]).astype(np.float64)
+    S_gpu = to_np(v["scores"]).T.astype(np.float64)
     pos = to_np(v["pos"])
     tok = to_np(v["tok"])
     # teacher-forced selection: bit-exact
@@ -155,7 +155,7 @@ def test_expert_choice_full_size_selection():
     t, layer, y, st, v = _run(w, inp)
     assert st.device_error == 0
     n = M.moe_expert_choice_tokens(w.T, w.E, w.k, w.cf)
-    S_gpu = to_np(v["scores"]).astype(np.float64)
+    S_gpu = to_np(v["scores"]).T.astype(np.float64)
     sel, tokens = oracle.expert_choice_select(S_gpu, n)
     pos = to_np(v["pos"])
     assert np.array_equal(pos >= 0, sel)
@@ -187,7 +187,7 @@ def test_expert_choice_many_ties_across_slices():
     inp["x"] = rows[torch.randint(0, 12, (w.T,), generator=g)].contiguous()
     inp["Wg"] = torch.randint(-1, 2, (w.d, w.E), generator=g).to(torch.bfloat16)
     t, layer, y, st, v = _run(w, inp)
-    S_gpu = to_np(v["scores"]).astype(np.float64)
+    S_gpu = to_np(v["scores"]).T.astype(np.float64)
     n = v["n"]
     assert all(len(np.unique(S_gpu[:, e])) <= 12 for e in range(w.E))
     sel, tokens = oracle.expert_choice_select(S_gpu, n)
