@@ -43,6 +43,7 @@
 #include <stdlib.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -96,6 +97,7 @@ struct TcParams {
   const int32_t* offsets;
   const int32_t* kept;
   int32_t* err;
+  int debug_stall;  // 1: the MMA issuer first waits on a barrier nobody arms (tests only)
 };
 
 struct Control {
@@ -104,6 +106,7 @@ struct Control {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  uint64_t never;  // armed by nobody: the failure-detection test waits on it
   uint32_t tmem_base;
   volatile int abort_flag;
   int total_tiles;
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&c.tempty[a]), 4 * CG);  // one arrive per epilogue warp of the group
     }
     mbar_init(smem_u32(&c.drain), 1);
+    mbar_init(smem_u32(&c.never), 1);
     c.abort_flag = 0;
     fence_mbar_init();
     fence_async_shared();
@@ -365,6 +369,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true, timed_out = false, issued_any = false;
+      // Failure-detection test: a wait that runs out, as if a load never
+      // arrived; every role then gives up within its own bounded wait.
+      if (p.debug_stall && !mbar_wait(smem_u32(&c.never), 0)) {
+        ok = false;
+        timed_out = true;
+      }
       for (int t = group; t < total && ok; t += ngroups) {
         if (c.abort_flag) {
           ok = false;
@@ -687,6 +697,20 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
                        CG, true, a, b0, b1, out, p);
 }
 
+// Failure-detection tests: MOE_DEBUG_STALL_MMA=N makes the next N up
+// projections stall their MMA issuer on a barrier nobody arms, so the
+// bounded waits run out and the kernel reports through its error word.
+int take_debug_stall() {
+  static std::atomic<int> budget{[] {
+    const char* v = getenv("MOE_DEBUG_STALL_MMA");
+    return v ? atoi(v) : 0;
+  }()};
+  int cur = budget.load();
+  while (cur > 0 && !budget.compare_exchange_weak(cur, cur - 1)) {
+  }
+  return cur > 0 ? 1 : 0;
+}
+
 // CTA pairs by default; MOE_TC_CTA_PAIR=0 selects one CTA per tile.
 bool use_cta_pairs() {
   static const bool pairs = [] {
@@ -751,6 +775,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.offsets = a.offsets;
   up.kept = a.kept_counts;
   up.err = a.dev_error;
+  up.debug_stall = take_debug_stall();
   cudaError_t err =
       swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, mh_out, up, num_sms,
                                        mtiles_max * up.n_tiles, up_wide, s)
@@ -771,6 +796,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.offsets = a.offsets;
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
+  dn.debug_stall = 0;
   err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, mo_out, dn, num_sms, mtiles_max * dn.n_tiles,
                                    dn_wide, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
