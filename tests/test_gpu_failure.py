@@ -96,3 +96,52 @@ def test_stalled_wait_times_out_and_the_context_survives():
     assert err_line, r.stdout
     assert int(err_line[0].split()[1]) & ERR_TIMEOUT_MMA
     assert "RECOVERED" in lines
+
+
+CANARY = 0xA5
+
+
+@pytest.mark.parametrize("case", [
+    dict(T=1000, d=256, E=8, k=2, H=384, cf=0.0),
+    dict(T=1100, d=136, E=6, k=3, H=200, cf=0.5),
+    dict(T=700, d=256, E=64, k=8, H=384, cf=1.25),
+])
+def test_no_writes_outside_the_caller_buffers(case):
+    """Every output and the workspace are bracketed by canary bytes; a
+    forward (token choice, then expert choice) must leave them untouched."""
+    from mixture_experts_layer_51_b200.workloads import Workload, make_inputs
+    w = Workload("canary", act="swiglu", dtype="bf16", seed=17, **case)
+    t = make_inputs(w, "cuda")
+    pad = 4096
+
+    def bracketed(nbytes):
+        buf = torch.full((nbytes + 2 * pad,), CANARY, dtype=torch.uint8, device="cuda")
+        return buf, buf[pad:pad + nbytes]
+
+    def intact(buf, nbytes):
+        head, tail = buf[:pad], buf[pad + nbytes:]
+        return bool((head == CANARY).all()) and bool((tail == CANARY).all())
+
+    need = M.moe_workspace_bytes(w.T, w.d, w.H, w.E, w.k, w.cf, torch.bfloat16, w.act)
+    ws_buf, ws = bracketed(need)
+    ybytes = w.T * w.d * 2
+    y_buf, y_raw = bracketed(ybytes)
+    y = y_raw.view(torch.bfloat16).view(w.T, w.d)
+    M.moe_forward(t["x"], t["Wg"], t["bias"], t["W1"], t["W3"], t["W2"], w.k, w.cf, w.act, y=y,
+                  ws=ws)
+    torch.cuda.synchronize()
+    assert intact(ws_buf, need) and intact(y_buf, ybytes)
+    assert torch.isfinite(y.float()).all()
+
+    ec_cf = w.cf if w.cf > 0 else 1.0
+    L = M.moe_expert_choice_layout(w.T, w.d, w.H, w.E, w.k, ec_cf, "bf16", w.act)
+    ws_buf, ws = bracketed(L.total)
+    y_buf, y_raw = bracketed(ybytes)
+    y = y_raw.view(torch.bfloat16).view(w.T, w.d)
+    st = M.lib().moe_forward_expert_choice(
+        M._ptr(t["x"]), M._ptr(t["Wg"]), M._ptr(t["bias"]), M._ptr(t["W1"]), M._ptr(t["W3"]),
+        M._ptr(t["W2"]), w.T, w.d, w.H, w.E, w.k, ec_cf, M.MOE_SWIGLU, M.MOE_BF16, M._ptr(y),
+        M._ptr(ws), ws.numel(), None, M._stream(y.device))
+    assert st == M.MOE_OK
+    torch.cuda.synchronize()
+    assert intact(ws_buf, L.total) and intact(y_buf, ybytes)
