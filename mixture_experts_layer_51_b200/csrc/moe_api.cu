@@ -172,10 +172,11 @@ MOE_API moe_status moe_workspace_layout(int32_t T, int32_t d, int32_t H, int32_t
   return compute_layout(T, d, H, E, k, cf, dt, act, out) ? MOE_OK : MOE_ERR_ARG;
 }
 
-MOE_API moe_status moe_route_ex(const void* x, const void* Wg, const float* bias, int32_t T,
-                                int32_t d, int32_t E, int32_t k, moe_dtype dt,
-                                const moe_options* opt, int32_t* idx, float* gate, float* margin,
-                                void* stream) {
+namespace {
+// Router; `err` (nullable) receives the tensor-core router's time-out bits.
+moe_status route_enqueue(const void* x, const void* Wg, const float* bias, int32_t T, int32_t d,
+                         int32_t E, int32_t k, moe_dtype dt, const moe_options* opt,
+                         int32_t* idx, float* gate, float* margin, void* stream, int32_t* err) {
   int gating;
   float gate_scale;
   if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt) || !read_options(opt, &gating, &gate_scale))
@@ -186,9 +187,18 @@ MOE_API moe_status moe_route_ex(const void* x, const void* Wg, const float* bias
   moe_status st = device_info(&di);
   if (st != MOE_OK) return st;
   RouteArgs a{x, Wg, bias, T, d, E, k, idx, gate, margin, gating, gate_scale};
+  a.err = err;
   return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
+}
+}  // namespace
+
+MOE_API moe_status moe_route_ex(const void* x, const void* Wg, const float* bias, int32_t T,
+                                int32_t d, int32_t E, int32_t k, moe_dtype dt,
+                                const moe_options* opt, int32_t* idx, float* gate, float* margin,
+                                void* stream) {
+  return route_enqueue(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, stream, nullptr);
 }
 
 MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, int32_t T,
@@ -377,7 +387,7 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
   if (cudaMemsetAsync(ticket, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
   moe_status st = record_stage(0, s);
   if (st != MOE_OK) return st;
-  st = moe_route_ex(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, s);
+  st = route_enqueue(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, s, err);
   if (st == MOE_OK) st = record_stage(1, s);
   if (st != MOE_OK) return st;
   int gating, priority;
@@ -753,9 +763,9 @@ MOE_API int32_t moe_expert_choice_tokens(int32_t T, int32_t E, int32_t k, double
   return C < 0 ? -1 : std::min(C, T);
 }
 
-MOE_API moe_status moe_expert_choice_route(const void* x, const void* Wg, const float* bias,
-                                           int32_t T, int32_t d, int32_t E, moe_dtype dt,
-                                           float* scores, void* stream) {
+namespace {
+moe_status ec_route_enqueue(const void* x, const void* Wg, const float* bias, int32_t T, int32_t d,
+                            int32_t E, moe_dtype dt, float* scores, void* stream, int32_t* err) {
   if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || !valid_dtype(dt)) return MOE_ERR_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !Wg || !scores || !aligned16(x) || !aligned16(Wg)) return MOE_ERR_ARG;
@@ -764,9 +774,17 @@ MOE_API moe_status moe_expert_choice_route(const void* x, const void* Wg, const 
   if (st != MOE_OK) return st;
   RouteArgs a{x, Wg, bias, T, d, E, 1, nullptr, nullptr, nullptr, MOE_GATE_TOPK_SOFTMAX, 1.0f,
               scores};
+  a.err = err;
   return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
+}
+}  // namespace
+
+MOE_API moe_status moe_expert_choice_route(const void* x, const void* Wg, const float* bias,
+                                           int32_t T, int32_t d, int32_t E, moe_dtype dt,
+                                           float* scores, void* stream) {
+  return ec_route_enqueue(x, Wg, bias, T, d, E, dt, scores, stream, nullptr);
 }
 
 MOE_API size_t moe_expert_choice_select_workspace_bytes(int32_t T, int32_t E) {
@@ -863,7 +881,7 @@ MOE_API moe_status moe_forward_expert_choice(const void* x, const void* Wg, cons
   int32_t* err = reinterpret_cast<int32_t*>(w + L.dev_error);
   if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   moe_status st = record_stage(0, s);
-  if (st == MOE_OK) st = moe_expert_choice_route(x, Wg, bias, T, d, E, dt, scores, s);
+  if (st == MOE_OK) st = ec_route_enqueue(x, Wg, bias, T, d, E, dt, scores, s, err);
   if (st == MOE_OK) st = record_stage(1, s);
   if (st == MOE_OK)
     st = moe_expert_choice_select(scores, T, E, L.n, tok, pos, kept, offsets, w + L.scratch,

@@ -344,8 +344,13 @@ struct RouteArgs {
   int gating;        // moe_gating
   float gate_scale;  // multiplies every gate
   float* scores = nullptr;  // non-null: write softmax over all E to [E, T] instead of TopK
+  int32_t* err = nullptr;   // device error word for the tensor-core router's bounded waits
 };
 cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms);
+// Tensor-core router (route_tc.cu): bf16, E % 8 == 0.  MOE_ROUTE_TC=0 turns
+// it off, for measurements.
+bool route_tc_supported(const RouteArgs& a);
+cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 
 // Whether kernels of the forward chain are launched with programmatic
 // dependent launch (default on; MOE_PDL=0 turns it off, for measurements).

@@ -542,6 +542,10 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
                                                     a.gating, a.gate_scale, a.scores);
     return cudaGetLastError();
   }
+  if (route_tc_supported(a)) {
+    const cudaError_t err = launch_route_tc(a, s);
+    if (err != cudaErrorInvalidValue) return err;  // else: no tensor map, use mma.sync
+  }
   return launch_route_bf16(a, s);
 }
 

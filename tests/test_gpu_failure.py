@@ -145,3 +145,4 @@ def test_no_writes_outside_the_caller_buffers(case):
     assert st == M.MOE_OK
     torch.cuda.synchronize()
     assert intact(ws_buf, L.total) and intact(y_buf, ybytes)
+
