@@ -15,7 +15,7 @@
 // one accumulator holds both halves of the SwiGLU and the epilogue writes
 // SiLU(gate) * up directly: the two pre-activations never reach HBM.
 //
-// Roles (192 threads):
+// Roles (192 threads; 320 with MOE_EPI_WARPS=8):
 //   warp 0      one thread issues TMA loads of A (K-major, 128B swizzle) and
 //               B (weights [E, K, N] read N-major, 128B swizzle) into a
 //               4-stage shared-memory ring;
@@ -25,7 +25,11 @@
 //               accumulators, so the epilogue of tile i overlaps the MMAs of
 //               tile i+1);
 //   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, activation,
-//               16-byte global stores of the kept rows.
+//               16-byte global stores of the kept rows.  (Eight epilogue
+//               warps, two per lane quadrant, measured no faster once the
+//               SiLU division was the approximate one: the IEEE division had
+//               made the SwiGLU epilogue, not the MMAs, the limit of layers
+//               with K = 1024, by 1.6x.)
 // The tile list (expert, m-block, n-block) is built on the device from the
 // per-expert offsets, with the experts that have the most m-blocks first and
 // m-blocks fastest, so concurrent CTAs share weight tiles in L2.  No host
@@ -53,13 +57,23 @@ namespace {
 
 constexpr int TM = 128;  // tile rows held by one CTA (UMMA M per CTA)
 constexpr int TN = 256;  // accumulator columns (UMMA N)
-constexpr int NUM_THREADS = 192;
+#ifndef MOE_EPI_WARPS
+#define MOE_EPI_WARPS 4
+#endif
+// Epilogue warps: 4 (one per TMEM lane quadrant) or 8 (two per quadrant,
+// each taking half of the accumulator's columns).
+constexpr int EPI_WARPS = MOE_EPI_WARPS;
+static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "4 or 8 epilogue warps");
+constexpr int EPI_SPLIT = EPI_WARPS / 4;  // epilogue warps per lane quadrant
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 2 * TN;
 constexpr int CONTROL_BYTES = 1536;
-// Epilogue output staging: per epilogue warp two 4 KB boxes (32 rows x
-// 128 bytes, 128-byte swizzled) that TMA stores drain to global memory.
+// Epilogue output staging: eight 4 KB boxes (32 rows x 128 bytes, 128-byte
+// swizzled) that TMA stores drain to global memory; two per warp with four
+// epilogue warps, one per warp with eight.
 constexpr int OUT_BOX_BYTES = 32 * 128;
-constexpr int OUT_STAGE_BYTES = 4 * 2 * OUT_BOX_BYTES;
+constexpr int OUT_BOXES_PER_WARP = 8 / EPI_WARPS;
+constexpr int OUT_STAGE_BYTES = 8 * OUT_BOX_BYTES;
 #ifndef MOE_PAIR_STAGES
 #define MOE_PAIR_STAGES 6  // ring depth of the CTA-pair kernel with 64-wide K steps
 #endif
@@ -129,7 +143,20 @@ __device__ __forceinline__ void decode_tile(const Control& c, int t, int& e, int
   m = local - n * mt;
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+#ifndef MOE_FAST_SILU
+#define MOE_FAST_SILU 1
+#endif
+// SiLU(z) = z / (1 + e^-z).  The fast form divides with the approximate
+// reciprocal (__fdividef): its error is a few fp32 ulps, far below the bf16
+// rounding of h; for z < -88 the denominator overflows and the result is 0,
+// SiLU's limit.
+__device__ __forceinline__ float silu_f(float z) {
+#if MOE_FAST_SILU
+  return __fdividef(z, 1.0f + __expf(-z));
+#else
+  return z / (1.0f + __expf(-z));
+#endif
+}
 __device__ __forceinline__ float gelu_f(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
 }
@@ -172,7 +199,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&c.tfull[a]), 1);
-      mbar_init(smem_u32(&c.tempty[a]), 4 * CG);  // one arrive per epilogue warp of the group
+      mbar_init(smem_u32(&c.tempty[a]), EPI_WARPS * CG);  // one arrive per epilogue warp of the group
     }
     mbar_init(smem_u32(&c.drain), 1);
     mbar_init(smem_u32(&c.never), 1);
@@ -460,8 +487,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // the same expert block (never read as results); a CTA whose 128-row
     // block starts past the kept rows stores nothing.
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
-    const uint32_t obuf0 = smem_base + STAGES * STAGE_BYTES + quad * 2 * OUT_BOX_BYTES;
-    uint8_t* const obuf0_p = smem + STAGES * STAGE_BYTES + quad * 2 * OUT_BOX_BYTES;
+    const int ew = warp - 2;    // epilogue warp index
+    const int half = ew / 4;    // which share of the columns (0 with four warps)
+    const uint32_t obuf0 = smem_base + STAGES * STAGE_BYTES + ew * OUT_BOXES_PER_WARP * OUT_BOX_BYTES;
+    uint8_t* const obuf0_p = smem + STAGES * STAGE_BYTES + ew * OUT_BOXES_PER_WARP * OUT_BOX_BYTES;
     int nbox = 0;
     // o is far larger than L2 and not read again by this kernel: its lines
     // go first, so the weight and activation tiles other CTAs still read
@@ -470,8 +499,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Stages this lane's 8 x 16 bytes as row `lane` of the next box and
     // issues its store at (col0, row0).
     auto store_box = [&](const uint4 (&v)[8], int col0, int row0) {
-      const int b = nbox & 1;
-      if (nbox >= 2 && lane == 0) bulk_wait_read<1>();  // the box two stores ago is read
+      const int b = nbox % OUT_BOXES_PER_WARP;
+      // the store that last used this box has read it
+      if (nbox >= OUT_BOXES_PER_WARP && lane == 0) bulk_wait_read<OUT_BOXES_PER_WARP - 1>();
       __syncwarp();
       uint8_t* rowp = obuf0_p + b * OUT_BOX_BYTES + lane * 128;
 #pragma unroll
@@ -518,17 +548,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // made this epilogue slower than the MMAs of a short tile: the
         // up projection of the 1024-wide layer lost 40%.)
         const int n0 = EPI == EPI_SWIGLU ? n * (TN / 2) : n * TN;
-        constexpr int NCH = EPI == EPI_SWIGLU ? 4 : TN / 32;
+        constexpr int NCH = (EPI == EPI_SWIGLU ? 4 : TN / 32) / EPI_SPLIT;  // chunks of this warp
         const bool row_ok = blk_ok && lane < valid_rows;
         __nv_bfloat16* dst_row =
             static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row0 + lane) * p.ld_out;
 #pragma unroll 1
-        for (int cc = 0; cc < NCH; ++cc) {
+        for (int ci = 0; ci < NCH; ++ci) {
+          const int cc = half * NCH + ci;
           float g[32], u[32];
           tc_ld_32cols(tbase + cc * 32, g);
           if (EPI == EPI_SWIGLU) tc_ld_32cols(tbase + TN / 2 + cc * 32, u);
           tc_wait_ld();
-          if (cc == NCH - 1) release(acc);
+          if (ci == NCH - 1) release(acc);
           if (row_ok) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -551,13 +582,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else {
         const int n0 = n * TN;
+        constexpr int NCH = TN / 32 / EPI_SPLIT;  // 32-column chunks of this warp
 #pragma unroll 1
-        for (int c0 = 0; c0 < TN / 32; c0 += 4) {
+        for (int c0 = half * NCH; c0 < (half + 1) * NCH; c0 += 4) {
           float g[4][32];
 #pragma unroll
           for (int b = 0; b < 4; ++b) tc_ld_32cols(tbase + (c0 + b) * 32, g[b]);
           tc_wait_ld();
-          if (c0 + 4 == TN / 32) release(acc);
+          if (c0 + 4 == (half + 1) * NCH) release(acc);
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
             const int col0 = n0 + (c0 + b) * 32;

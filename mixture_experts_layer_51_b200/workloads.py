@@ -11,8 +11,8 @@ layer shape, an OpenMoE-style skewed layer and a fine-grained layer):
 * x ~ N(0, 1) unless ``tokens == "zipf"``.
 * Router W_g [d, E] ~ N(0, 1/d); expert W1, W3 [E, d, H] ~ N(0, 1/d);
   W2 [E, H, d] ~ N(0, 1/H)  (variance = 1/fan_in).
-* ``tokens == "zipf"``: token ids drawn from P(r) ~ r^-1.1 over a 32000-id
-  vocabulary; x = emb[id] + 0.1 N(0, 1) with emb ~ N(0, 1) [32000, d], so the
+* ``tokens == "zipf"``: token ids drawn (inverse CDF) from P(r) ~ r^-1.1 over
+  a 32000-id vocabulary; x = emb[id] + 0.1 N(0, 1) with emb ~ N(0, 1) [32000, d], so the
   routing is dominated by the token id ("Context-independent Specialization"
   on "Take a Closer Look at the MoE LLM Routing").
 * ``bias_var > 0``: a per-expert router bias ~ N(0, bias_var) in fp32.
@@ -77,6 +77,18 @@ ZIPF_VOCAB = 32000
 ZIPF_S = 1.1
 
 
+def _zipf_ids(gen, n, device):
+    """n token ids with P(id = r - 1) proportional to r^-ZIPF_S, r = 1..ZIPF_VOCAB,
+    by inverse-CDF sampling: one uniform draw per id and a binary search in
+    the fp64 CDF (built on the host).  Unlike a multinomial draw on the GPU,
+    this gives the same ids for the same seed in every process."""
+    ranks = torch.arange(1, ZIPF_VOCAB + 1, dtype=torch.float64)
+    cdf = torch.cumsum(ranks.pow(-ZIPF_S), 0)
+    cdf = (cdf / cdf[-1]).to(device)
+    u = torch.rand(n, generator=gen, device=device, dtype=torch.float64)
+    return torch.searchsorted(cdf, u, right=True).clamp_(max=ZIPF_VOCAB - 1)
+
+
 def _normal(gen, shape, std, device):
     return torch.randn(shape, generator=gen, device=device,
                        dtype=torch.float32) * std
@@ -95,11 +107,7 @@ def make_inputs(w: Workload, device="cpu"):
     dt = w.torch_dtype
     out = {}
     if w.tokens == "zipf":
-        ranks = torch.arange(1, ZIPF_VOCAB + 1, dtype=torch.float64,
-                             device=device)
-        p = ranks.pow(-ZIPF_S)
-        p = (p / p.sum()).to(torch.float32)
-        ids = torch.multinomial(p, w.T, replacement=True, generator=gen)
+        ids = _zipf_ids(gen, w.T, device)
         emb = _normal(gen, (ZIPF_VOCAB, w.d), 1.0, device)
         x = emb[ids] + _normal(gen, (w.T, w.d), 0.1, device)
         del emb

@@ -7,7 +7,9 @@ import math
 import os
 import re
 
+import numpy as np
 import pytest
+import torch
 
 from mixture_experts_layer_51_b200 import moe as M
 from mixture_experts_layer_51_b200.workloads import WORKLOADS
@@ -238,3 +240,22 @@ def test_sizes_past_int32_rows_are_rejected(lib):
     assert M.moe_workspace_bytes(1_000_000, 64, 64, 64, 8, 0.0, "bf16", "swiglu") > 0
     assert lib.moe_expert_choice_workspace_bytes(40_000_000, 64, 64, 64, 8, 1.0, M.MOE_BF16,
                                                  M.MOE_SWIGLU) == 0
+
+
+def test_zipf_token_ids_are_reproducible_and_follow_the_law():
+    """The skewed workload's token ids: the same seed gives the same ids, and
+    the frequencies of the most common ids follow P(r) ~ r^-1.1 (within five
+    standard errors of a 200000-draw sample)."""
+    from mixture_experts_layer_51_b200.workloads import ZIPF_S, ZIPF_VOCAB, _zipf_ids
+    n = 200000
+    a = _zipf_ids(torch.Generator().manual_seed(3), n, "cpu").numpy()
+    b = _zipf_ids(torch.Generator().manual_seed(3), n, "cpu").numpy()
+    assert np.array_equal(a, b)
+    assert a.min() >= 0 and a.max() < ZIPF_VOCAB
+    r = np.arange(1, ZIPF_VOCAB + 1, dtype=np.float64)
+    p = r ** -ZIPF_S
+    p /= p.sum()
+    freq = np.bincount(a, minlength=ZIPF_VOCAB) / n
+    top = slice(0, 20)
+    se = np.sqrt(p[top] * (1 - p[top]) / n)
+    assert np.all(np.abs(freq[top] - p[top]) <= 5 * se)
