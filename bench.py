@@ -91,9 +91,9 @@ def algorithmic(w, n_kept, tokens_with_kept, routing="token_choice"):
         "permute": 2 * T * k * 4 + tokens_with_kept * d * s + n_kept * d * s + T * k * 4,
         # weights once, activations in and out
         "ffn_up": n_w_up * s + n_kept * d * s + n_kept * H * s,
-        "ffn_down": E * H * d * s + n_kept * H * s + n_kept * d * 4,
-        # read kept rows of o (fp32), pos and gate; write y
-        "combine": n_kept * d * 4 + T * k * 8 + T * d * s,
+        "ffn_down": E * H * d * s + n_kept * H * s + n_kept * d * s,
+        # read kept rows of o (layer dtype), pos and gate; write y
+        "combine": n_kept * d * s + T * k * 8 + T * d * s,
     }
     if routing == "expert_choice":
         # route: read x and W_g, write the [T, E] affinities; select + gather:
@@ -102,7 +102,7 @@ def algorithmic(w, n_kept, tokens_with_kept, routing="token_choice"):
         # kept rows of o, pos and affinities [T, E], write y
         byts["route"] = T * d * s + d * E * s + T * E * 4
         byts["permute"] = 2 * T * E * 4 + n_kept * 4 + tokens_with_kept * d * s + n_kept * d * s
-        byts["combine"] = n_kept * d * 4 + T * E * 8 + T * d * s
+        byts["combine"] = n_kept * d * s + T * E * 8 + T * d * s
     total_flop = flop["route"] + flop["ffn_up"] + flop["ffn_down"]
     return flop, byts, total_flop
 

@@ -26,9 +26,10 @@
  *   before returning.
  * - Layouts are row-major and dense: x [T, d]; W_g [d, E]; W1, W3 [E, d, H];
  *   W2 [E, H, d]; y [T, d]; idx, gate, pos [T, k].
- * - Element types: MOE_BF16 means x, W_g, W1, W3, W2, xp, h and y are bf16;
- *   MOE_FP32 means they are fp32.  Router bias, gates, margins and the
- *   expert output `o` are always fp32; indices and counts are int32.
+ * - Element types: MOE_BF16 means x, W_g, W1, W3, W2, xp, h, the expert
+ *   outputs o and y are bf16; MOE_FP32 means they are fp32.  Router bias,
+ *   gates, margins and affinities are always fp32 (so is every accumulation);
+ *   indices and counts are int32.
  * - Limits: 1 <= k <= E <= 64, k <= 8, d % 8 == 0, H % 8 == 0, T >= 0, and
  *   at most 2^31 - 1 permuted rows (int32 row indices on the device).
  *   T == 0 is valid and does nothing.  Pointers must be 16-byte aligned.
@@ -125,7 +126,7 @@ typedef struct {
   size_t scratch;      /* permute scratch (moe_permute_workspace_bytes)     */
   size_t xp;           /* dtype [rows, d] permuted tokens                   */
   size_t h;            /* dtype [rows, H] expert hidden activations         */
-  size_t o;            /* fp32  [rows, d] expert outputs                    */
+  size_t o;            /* dtype [rows, d] expert outputs                    */
   size_t total;        /* == moe_workspace_bytes(...)                       */
   int64_t rows;        /* rows of xp/h/o (moe_max_permuted_rows)            */
   size_t order;        /* int32 [T] queue order (priority routing only)     */
@@ -272,25 +273,26 @@ moe_status moe_permute_static(const void* x, const int32_t* idx, int32_t T, int3
  *   xp [rows, d] (dtype), offsets [E+1], kept_counts [E] as from moe_permute.
  *   W1, W3 [E, d, H] (W3 unused and may be NULL for MOE_GELU), W2 [E, H, d].
  *   Out: h [rows, H] (dtype) = SiLU(xp W1_e) * (xp W3_e)  or GELU(xp W1_e);
- *        o [rows, d] fp32 = h W2_e.  Only kept rows are written.
+ *        o [rows, d] (dtype) = h W2_e.  Only kept rows are written.
  *   dev_error: int32 device word; a kernel that gives up on a bounded wait
  *   ORs a nonzero code into it (the caller zeroes it beforehand).
  *   bf16 runs on the tcgen05 tensor cores with fp32 accumulation (h is
- *   rounded to bf16 before the second GEMM); fp32 runs on fp32 FMA. */
+ *   rounded to bf16 before the second GEMM, o when it is stored); fp32 runs
+ *   on fp32 FMA. */
 moe_status moe_grouped_ffn(const void* xp, int64_t rows, const int32_t* offsets,
                            const int32_t* kept_counts, const void* W1, const void* W3,
                            const void* W2, int32_t E, int32_t d, int32_t H, moe_act act,
-                           moe_dtype dtype, void* h, float* o, int32_t* dev_error,
+                           moe_dtype dtype, void* h, void* o, int32_t* dev_error,
                            void* stream);
 
 /* Un-permute and gate-weighted combine ("[Paper Club] Upcycling ...": the
  * tokens are put back in their original order and scaled by the router
  * probability; y = sum_i G(x)_i E_i(x)).
- *   o [rows, d] fp32, pos [T, k], gate [T, k].
+ *   o [rows, d] (dtype), pos [T, k], gate [T, k].
  *   Out: y [T, d] (dtype), y_t = sum over kept j, in slot order, of
  *   gate[t,j] * o[pos[t,j]], accumulated in fp32 and rounded once; a token
  *   with every slot dropped gets y_t = 0.  No atomics: deterministic. */
-moe_status moe_unpermute_combine(const float* o, const int32_t* pos, const float* gate,
+moe_status moe_unpermute_combine(const void* o, const int32_t* pos, const float* gate,
                                  int32_t T, int32_t d, int32_t k, moe_dtype dtype,
                                  void* y, void* stream);
 
@@ -414,9 +416,9 @@ moe_status moe_expert_choice_permute(const void* x, const int32_t* pos, int32_t 
                                      int64_t xp_rows, void* stream);
 
 /* y [T, d] (dtype) = sum over e with pos[t, e] >= 0, ascending e, of
- * scores[e, t] * o[pos[t, e]] (o fp32 from moe_grouped_ffn), fp32
+ * scores[e, t] * o[pos[t, e]] (o (dtype) from moe_grouped_ffn), fp32
  * accumulation, one rounding.  Every y row is written. */
-moe_status moe_expert_choice_combine(const float* o, const int32_t* pos, const float* scores,
+moe_status moe_expert_choice_combine(const void* o, const int32_t* pos, const float* scores,
                                      int32_t T, int32_t d, int32_t E, moe_dtype dtype, void* y,
                                      void* stream);
 
@@ -429,7 +431,7 @@ typedef struct {
   size_t offsets;      /* int32 [E + 1] (= e * npad)                       */
   size_t dev_error;    /* int32 [1]     device error word                  */
   size_t scratch;      /* select scratch                                   */
-  size_t xp, h, o;     /* rows x d (dtype), rows x H (dtype), rows x d fp32 */
+  size_t xp, h, o;     /* rows x d, rows x H, rows x d (all dtype)         */
   size_t total;
   int64_t rows;        /* E * npad                                         */
   int32_t n;           /* tokens per expert                                */

@@ -269,9 +269,10 @@ __global__ void __launch_bounds__(256)
 
 constexpr int kEcCombineWarps = 8;
 
-template <bool OUT_BF16>
+// BF16: o and y are bf16 (else both fp32).
+template <bool BF16>
 __global__ void __launch_bounds__(kEcCombineWarps * 32)
-    ec_combine_kernel(const float4* __restrict__ o, const int32_t* __restrict__ pos,
+    ec_combine_kernel(const void* __restrict__ o, const int32_t* __restrict__ pos,
                       const float* __restrict__ scores, int T, int d, int E,
                       void* __restrict__ y) {
   __shared__ int sp[kEcCombineWarps][kMaxE];
@@ -301,31 +302,15 @@ __global__ void __launch_bounds__(kEcCombineWarps * 32)
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     for (int j0 = 0; j0 < nsel; j0 += 4) {
-      float4 v[4][2];
+      Row8<BF16> v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (j0 + u < nsel) {
-          const float4* row = o + (int64_t)sp[warp][j0 + u] * d4 + c8 * 2;
-          v[u][0] = __ldcs(row);
-          v[u][1] = __ldcs(row + 1);
-        }
-      }
+      for (int u = 0; u < 4; ++u)
+        if (j0 + u < nsel) v[u].load(o, sp[warp][j0 + u], d, c8);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (j0 + u < nsel) {
-          const float g = sg[warp][j0 + u];
-          acc[0] = fmaf(g, v[u][0].x, acc[0]);
-          acc[1] = fmaf(g, v[u][0].y, acc[1]);
-          acc[2] = fmaf(g, v[u][0].z, acc[2]);
-          acc[3] = fmaf(g, v[u][0].w, acc[3]);
-          acc[4] = fmaf(g, v[u][1].x, acc[4]);
-          acc[5] = fmaf(g, v[u][1].y, acc[5]);
-          acc[6] = fmaf(g, v[u][1].z, acc[6]);
-          acc[7] = fmaf(g, v[u][1].w, acc[7]);
-        }
-      }
+      for (int u = 0; u < 4; ++u)
+        if (j0 + u < nsel) v[u].fma_into(sg[warp][j0 + u], acc);
     }
-    if (OUT_BF16) {
+    if (BF16) {
       uint4 q;
       q.x = pack_bf16x2(acc[0], acc[1]);
       q.y = pack_bf16x2(acc[2], acc[3]);
@@ -358,16 +343,15 @@ cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad,
                        dim3(256), 0, s, 1, true, static_cast<const int32_t*>(pos_t), T, E, pos);
 }
 
-cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,
+cudaError_t launch_ec_combine(const void* o, const int32_t* pos, const float* scores, int T,
                               int d, int E, moe_dtype dtype, void* y, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int grid = (T + kEcCombineWarps - 1) / kEcCombineWarps;
-  const float4* o4 = reinterpret_cast<const float4*>(o);
   const dim3 th(kEcCombineWarps * 32);
   if (dtype == MOE_BF16)
-    return launch_kernel(ec_combine_kernel<true>, dim3(grid), th, 0, s, 1, true, o4, pos, scores, T,
+    return launch_kernel(ec_combine_kernel<true>, dim3(grid), th, 0, s, 1, true, o, pos, scores, T,
                          d, E, y);
-  return launch_kernel(ec_combine_kernel<false>, dim3(grid), th, 0, s, 1, true, o4, pos, scores, T,
+  return launch_kernel(ec_combine_kernel<false>, dim3(grid), th, 0, s, 1, true, o, pos, scores, T,
                        d, E, y);
 }
 

@@ -120,7 +120,7 @@ moe_status launch_ffn_simt(const FfnArgs& a, cudaStream_t s, cudaEvent_t between
   if (between && cudaEventRecord(between, s) != cudaSuccess) return MOE_ERR_CUDA;
   dim3 g2(row_tiles, (a.d + BN - 1) / BN);
   ffn_simt_kernel<0><<<g2, 256, 0, s>>>(h, a.offsets, a.kept_counts, a.E,
-                                        static_cast<const float*>(a.W2), nullptr, a.o, a.H, a.d);
+                                        static_cast<const float*>(a.W2), nullptr, static_cast<float*>(a.o), a.H, a.d);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -9,7 +9,7 @@
 //
 // Two launches of one persistent, warp-specialised kernel:
 //   up:   h[rows, H] = SiLU(xp W1_e) * (xp W3_e)   (bf16 out; GELU variant)
-//   down: o[rows, d] = h W2_e                      (fp32 out)
+//   down: o[rows, d] = h W2_e                      (bf16 out)
 // Tiles are 128 rows x 256 accumulator columns.  For the up projection the
 // 256 columns are 128 columns of W1 next to the same 128 columns of W3, so
 // one accumulator holds both halves of the SwiGLU and the epilogue writes
@@ -97,7 +97,7 @@ struct Cfg {
 constexpr int MAX_STAGES = 8;
 constexpr int B_BOX_BYTES = 64 * 64 * 2;  // a 64 x 64 box (3-D fallback loads, TKS = 64)
 
-enum Epi { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_PLAIN_F32 = 2 };
+enum Epi { EPI_SWIGLU = 0, EPI_GELU = 1, EPI_PLAIN = 2 };
 
 struct TcParams {
   void* out;
@@ -477,13 +477,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // --------------------------------------------------------- epilogue
     // Each warp drains its 32 TMEM lanes (tile rows), applies the
     // activation and stores; the accumulator is released as soon as its last
-    // columns are in registers.  bf16 outputs (h): each lane writes its own
-    // row.  fp32 outputs (o): four 32-column loads per wait, then 128-byte
-    // rows go into a swizzled 32-row staging box in shared memory and one
-    // TMA store per box carries it to global memory (whole lines,
-    // asynchronous; two boxes per warp alternate) -- per-row 16-byte stores
-    // half-fill every sector and throttled the down projection of short-K
-    // layers.  Rows of a box past the expert's kept rows are padding rows of
+    // columns are in registers.  Up projection (h): each lane writes its own
+    // row.  Down projection (o): four 32-column loads per wait, rounded to
+    // bf16; each 64-column row segment (128 bytes) goes into a swizzled
+    // 32-row staging box in shared memory and one TMA store per box carries
+    // it to global memory (whole lines, asynchronous; two boxes per warp
+    // alternate) -- per-row 16-byte stores half-filled every sector and
+    // throttled the down projection of short-K layers when o was fp32.  Rows of a box past the expert's kept rows are padding rows of
     // the same expert block (never read as results); a CTA whose 128-row
     // block starts past the kept rows stores nothing.
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
@@ -591,14 +591,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_wait_ld();
           if (c0 + 4 == (half + 1) * NCH) release(acc);
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          for (int b = 0; b < 4; b += 2) {
+            // Two 32-column chunks = one 64-column (128-byte) bf16 row
+            // segment of the box.
             const int col0 = n0 + (c0 + b) * 32;
             if (blk_ok && col0 < p.n_out) {
               uint4 v[8];
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                v[q] = make_uint4(__float_as_uint(g[b][4 * q + 0]), __float_as_uint(g[b][4 * q + 1]),
-                                  __float_as_uint(g[b][4 * q + 2]), __float_as_uint(g[b][4 * q + 3]));
+              for (int q = 0; q < 8; ++q) {
+                const float* src = &g[b + (q >> 2)][(q & 3) * 8];
+                v[q] = make_uint4(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]),
+                                  pack_bf16x2(src[4], src[5]), pack_bf16x2(src[6], src[7]));
+              }
               store_box(v, col0, row0);
             }
           }
@@ -791,7 +795,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   ok = ok && (dn_chunked ? make_map_w4d(&mw2, a.W2, a.E, a.H, a.d, dn_chunks, dn_kr)
                          : make_map_3d(&mw2, a.W2, a.E, a.H, a.d));
   ok = ok && make_map_out(&mh_out, a.h, a.rows, a.H, false) &&
-       make_map_out(&mo_out, a.o, a.rows, a.d, true);
+       make_map_out(&mo_out, a.o, a.rows, a.d, false);
   if (!ok) return MOE_ERR_CUDA;
   const int64_t mtiles_max = (a.rows + TM - 1) / TM;
 
@@ -829,7 +833,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
   dn.debug_stall = 0;
-  err = launch_gemm<EPI_PLAIN_F32>(mh, mw2, mw2, mo_out, dn, num_sms, mtiles_max * dn.n_tiles,
+  err = launch_gemm<EPI_PLAIN>(mh, mw2, mw2, mo_out, dn, num_sms, mtiles_max * dn.n_tiles,
                                    dn_wide, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -114,7 +114,7 @@ bool compute_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, doubl
   L->prio_scratch = take(priority_scratch_bytes(T));
   L->xp = take(static_cast<size_t>(rows) * d * es);
   L->h = take(static_cast<size_t>(rows) * H * es);
-  L->o = take(static_cast<size_t>(rows) * d * 4);
+  L->o = take(static_cast<size_t>(rows) * d * es);
   L->total = off;
   L->rows = rows;
   return true;
@@ -312,7 +312,7 @@ MOE_API moe_status moe_priority_order(const float* gate, int32_t T, int32_t k, i
 MOE_API moe_status moe_grouped_ffn(const void* xp, int64_t rows, const int32_t* offsets,
                                    const int32_t* kept_counts, const void* W1, const void* W3,
                                    const void* W2, int32_t E, int32_t d, int32_t H, moe_act act,
-                                   moe_dtype dt, void* h, float* o, int32_t* dev_error,
+                                   moe_dtype dt, void* h, void* o, int32_t* dev_error,
                                    void* stream) {
   if (!valid_ffn_sizes(d, H) || E < 1 || E > kMaxE || !valid_act(act) || !valid_dtype(dt) ||
       rows < 0 || rows > INT32_MAX || rows % kRowAlign != 0)
@@ -346,7 +346,7 @@ MOE_API moe_status moe_set_stage_events(void* const* events) {
   return MOE_OK;
 }
 
-MOE_API moe_status moe_unpermute_combine(const float* o, const int32_t* pos, const float* gate,
+MOE_API moe_status moe_unpermute_combine(const void* o, const int32_t* pos, const float* gate,
                                          int32_t T, int32_t d, int32_t k, moe_dtype dt, void* y,
                                          void* stream) {
   if (T < 0 || d <= 0 || d % 8 != 0 || k < 1 || k > kMaxK || !valid_dtype(dt)) return MOE_ERR_ARG;
@@ -406,10 +406,10 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
   if (st == MOE_OK) st = record_stage(2, s);
   if (st != MOE_OK) return st;
   st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,
-                       reinterpret_cast<float*>(w + L.o), err, s);
+                       w + L.o, err, s);
   if (st == MOE_OK) st = record_stage(4, s);
   if (st != MOE_OK) return st;
-  st = moe_unpermute_combine(reinterpret_cast<float*>(w + L.o), pos, gate, T, d, k, dt, y, s);
+  st = moe_unpermute_combine(w + L.o, pos, gate, T, d, k, dt, y, s);
   if (st == MOE_OK) st = record_stage(5, s);
   return st;
 }
@@ -748,7 +748,7 @@ bool ec_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, double cf,
   L->scratch = take(ec_select_scratch_bytes(T, E));
   L->xp = take(static_cast<size_t>(rows) * d * es);
   L->h = take(static_cast<size_t>(rows) * H * es);
-  L->o = take(static_cast<size_t>(rows) * d * 4);
+  L->o = take(static_cast<size_t>(rows) * d * es);
   L->total = off;
   L->rows = rows;
   L->n = n;
@@ -828,7 +828,7 @@ MOE_API moe_status moe_expert_choice_permute(const void* x, const int32_t* pos, 
              : MOE_ERR_CUDA;
 }
 
-MOE_API moe_status moe_expert_choice_combine(const float* o, const int32_t* pos,
+MOE_API moe_status moe_expert_choice_combine(const void* o, const int32_t* pos,
                                              const float* scores, int32_t T, int32_t d,
                                              int32_t E, moe_dtype dt, void* y, void* stream) {
   if (T < 0 || d <= 0 || d % 8 != 0 || E < 1 || E > kMaxE || !valid_dtype(dt)) return MOE_ERR_ARG;
@@ -890,12 +890,12 @@ MOE_API moe_status moe_forward_expert_choice(const void* x, const void* Wg, cons
   if (st == MOE_OK) st = record_stage(2, s);
   if (st == MOE_OK && L.rows > 0)
     st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,
-                         reinterpret_cast<float*>(w + L.o), err, s);
+                         w + L.o, err, s);
   else if (st == MOE_OK)
     st = record_stage(3, s);
   if (st == MOE_OK) st = record_stage(4, s);
   if (st == MOE_OK)
-    st = moe_expert_choice_combine(reinterpret_cast<float*>(w + L.o), pos, scores, T, d, E, dt, y,
+    st = moe_expert_choice_combine(w + L.o, pos, scores, T, d, E, dt, y,
                                    s);
   if (st == MOE_OK) st = record_stage(5, s);
   if (st != MOE_OK || !stats) return st;

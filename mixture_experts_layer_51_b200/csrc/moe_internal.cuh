@@ -332,6 +332,50 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Eight consecutive elements of a row of the expert outputs o, as loaded
+// (one 16-byte vector of bf16, or two of fp32), so a caller can issue every
+// load of an iteration before any arithmetic.  Streaming loads: o is read
+// once.
+template <bool BF16>
+struct Row8;
+template <>
+struct Row8<true> {
+  uint4 v;
+  __device__ __forceinline__ void load(const void* o, int64_t row, int d, int c8) {
+    v = __ldcs(reinterpret_cast<const uint4*>(o) + row * (d / 8) + c8);
+  }
+  __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
+  // acc[i] += g * element i (bf16 -> fp32 is exact: the high 16 bits).
+  __device__ __forceinline__ void fma_into(float g, float (&acc)[8]) const {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xffff0000u), acc[2 * i + 1]);
+    }
+  }
+};
+template <>
+struct Row8<false> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const void* o, int64_t row, int d, int c8) {
+    const float4* r = reinterpret_cast<const float4*>(o) + row * (d / 4) + c8 * 2;
+    a = __ldcs(r);
+    b = __ldcs(r + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void fma_into(float g, float (&acc)[8]) const {
+    acc[0] = fmaf(g, a.x, acc[0]);
+    acc[1] = fmaf(g, a.y, acc[1]);
+    acc[2] = fmaf(g, a.z, acc[2]);
+    acc[3] = fmaf(g, a.w, acc[3]);
+    acc[4] = fmaf(g, b.x, acc[4]);
+    acc[5] = fmaf(g, b.y, acc[5]);
+    acc[6] = fmaf(g, b.z, acc[6]);
+    acc[7] = fmaf(g, b.w, acc[7]);
+  }
+};
+
 // ------------------------------------------------- launchers (host side)
 struct RouteArgs {
   const void* x;
@@ -422,7 +466,8 @@ size_t ec_select_scratch_bytes(int T, int E);
 cudaError_t launch_ec_select(const float* scores, int T, int E, int n, int npad, void* scratch,
                              int32_t* tok, int32_t* pos, int32_t* kept_counts, int32_t* offsets,
                              cudaStream_t s);
-cudaError_t launch_ec_combine(const float* o, const int32_t* pos, const float* scores, int T,
+// o [rows, d] in the layer dtype (bf16 or fp32).
+cudaError_t launch_ec_combine(const void* o, const int32_t* pos, const float* scores, int T,
                               int d, int E, moe_dtype dtype, void* y, cudaStream_t s);
 
 struct FfnArgs {
@@ -436,7 +481,7 @@ struct FfnArgs {
   int E, d, H;
   moe_act act;
   void* h;
-  float* o;
+  void* o;  // [rows, d] in the layer dtype
   int32_t* dev_error;
 };
 // `between` (may be null) is recorded on the stream after the up projection.
@@ -445,7 +490,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms,
 moe_status launch_ffn_simt(const FfnArgs& a, cudaStream_t s, cudaEvent_t between);  // fp32
 
 struct CombineArgs {
-  const float* o;
+  const void* o;  // [rows, d] in the layer dtype
   const int32_t* pos;
   const float* gate;
   int T, d, k;

@@ -289,7 +289,7 @@ def workspace_views(ws, layout, T, d, H, E, k, dtype):
         dev_error=view(layout.dev_error, 1, torch.int32),
         xp=view(layout.xp, rows * d, dtype).view(rows, d),
         h=view(layout.h, rows * H, dtype).view(rows, H),
-        o=view(layout.o, rows * d, torch.float32).view(rows, d),
+        o=view(layout.o, rows * d, dtype).view(rows, d),
     )
 
 
@@ -395,7 +395,7 @@ def moe_grouped_ffn(xp, offsets, kept_counts, W1, W3, W2, act, h=None, o=None, d
     E, _, H = W1.shape
     dev = xp.device
     h = h if h is not None else torch.empty((rows, H), dtype=xp.dtype, device=dev)
-    o = o if o is not None else torch.empty((rows, d), dtype=torch.float32, device=dev)
+    o = o if o is not None else torch.empty((rows, d), dtype=xp.dtype, device=dev)
     dev_error = dev_error if dev_error is not None else torch.zeros(1, dtype=torch.int32, device=dev)
     _check(lib().moe_grouped_ffn(_ptr(xp), rows, _ptr(offsets), _ptr(kept_counts), _ptr(W1),
                                  _ptr(W3), _ptr(W2), E, d, H, _act_code(act), _dtype_code(xp),
@@ -405,6 +405,10 @@ def moe_grouped_ffn(xp, offsets, kept_counts, W1, W3, W2, act, h=None, o=None, d
 
 
 def moe_unpermute_combine(o, pos, gate, dtype, y=None, stream=None):
+    """y [T, d] (dtype) from the expert outputs o, which are in the layer
+    dtype too."""
+    if o.dtype != dtype:
+        raise TypeError(f"o is {o.dtype}; the combine reads o in the layer dtype {dtype}")
     T, k = pos.shape
     d = o.shape[1]
     dev = o.device
@@ -610,6 +614,8 @@ def moe_expert_choice_permute(x, pos, n, xp=None, stream=None):
 
 
 def moe_expert_choice_combine(o, pos, scores, dtype, y=None, stream=None):
+    if o.dtype != dtype:
+        raise TypeError(f"o is {o.dtype}; the combine reads o in the layer dtype {dtype}")
     T, E = pos.shape
     d = o.shape[1]
     y = y if y is not None else torch.empty((T, d), dtype=dtype, device=o.device)

@@ -95,8 +95,12 @@ def test_workspace_layout_is_consistent(lib):
             L.scratch, L.order, L.prio_scratch, L.xp, L.h, L.o]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     assert L.rows == M.moe_max_permuted_rows(8192, 8, 2, 0.0)
-    assert L.total >= L.o + L.rows * 4096 * 4
+    # xp, h and o in the layer dtype (bf16: 2 bytes)
+    assert L.h - L.xp >= L.rows * 4096 * 2 and L.o - L.h >= L.rows * 14336 * 2
+    assert L.total >= L.o + L.rows * 4096 * 2
     assert M.moe_workspace_bytes(8192, 4096, 14336, 8, 2, 0.0, "bf16", "swiglu") == L.total
+    F = M.moe_workspace_layout(256, 64, 128, 4, 1, 1.25, "fp32", "gelu")
+    assert F.total >= F.o + F.rows * 64 * 4
 
 
 def test_invalid_arguments_are_rejected_before_any_cuda_call(lib):
@@ -200,7 +204,7 @@ def test_expert_choice_sizes_and_validation(lib):
     offs = [L.scores, L.pos, L.tok, L.kept_counts, L.offsets, L.dev_error, L.scratch, L.xp, L.h,
             L.o]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
-    assert L.total >= L.o + L.rows * 256 * 4
+    assert L.total >= L.o + L.rows * 256 * 2  # o in the layer dtype (bf16)
     assert lib.moe_expert_choice_workspace_bytes(700, 256, 384, 64, 8, 1.0, M.MOE_BF16,
                                                  M.MOE_SWIGLU) == L.total
     assert lib.moe_expert_choice_workspace_bytes(700, 256, 384, 64, 8, 0.0, M.MOE_BF16,

@@ -237,7 +237,7 @@ def test_grouped_ffn_against_oracle(act):
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     h = to_np(h.float())
-    o = to_np(o)
+    o = to_np(o.float())
     for e in range(E):
         r = slice(off[e], off[e] + kept[e])
         if kept[e] == 0:
@@ -250,9 +250,11 @@ def test_grouped_ffn_against_oracle(act):
             h_ref = oracle.gelu(xr.double().numpy() @ W1[e].double().numpy())
         # h is rounded to bf16 once: relative error <= 2^-8 per element.
         assert np.all(np.abs(h[r] - h_ref) <= 2.0 ** -8 * np.abs(h_ref) + 1e-6), f"h expert {e}"
-        # o given the GPU's own h: only fp32 accumulation differs.
+        # o given the GPU's own h: fp32 accumulation, then one rounding to
+        # bf16 (relative error <= 2^-9, plus the accumulation's own).
         o_ref = h[r].astype(np.float64) @ W2[e].double().numpy()
-        _, rel = assert_y_close(o[r], o_ref, "fp32", f"o expert {e}")
+        bound = 2.0 ** -8 * np.abs(o_ref) + 1e-5 * np.abs(o_ref).max()
+        assert np.all(np.abs(o[r] - o_ref) <= bound), f"o expert {e}"
 
 
 # ------------------------------------------------------ full-size layers
