@@ -339,9 +339,9 @@ def main(argv=None):
             stage_ms[s] += v / n_stage
 
     # Kernels of ours per timed forward: router, count, rank, copy, two
-    # GEMMs, combine (token choice); router, select, copy, two GEMMs,
-    # combine (expert choice).
-    kernels_per_forward = 6 if ec else 7
+    # GEMMs, combine (token choice); router, select, transpose, copy, two
+    # GEMMs, combine (expert choice).
+    kernels_per_forward = 7
     ms_per_step = elapsed_ms / a.steps
     tokens_per_s = whole_job_rate(w.T, world, a.steps, elapsed_ms)
     tflops = total_flop * world * a.steps / (elapsed_ms / 1e3) / 1e12
