@@ -358,6 +358,28 @@ moe_status moe_pipeline_wait(moe_pipeline* p, int32_t slot);
 /* Waits for every slot, then releases the handle (NULL is a no-op). */
 moe_status moe_pipeline_destroy(moe_pipeline* p);
 
+/* One forward captured as a CUDA graph, for small layers whose forward is
+ * shorter than the host's launch work (seven kernels and two memsets).
+ * moe_forward_graph_create records moe_forward_ex with these arguments
+ * (stats not available) on a private stream and instantiates it; nothing
+ * runs yet.  The graph keeps the pointers it was made with: x, y, ws and the
+ * weights must stay allocated while it exists, and each launch reads
+ * whatever x holds when it runs.  moe_forward_graph_launch enqueues one
+ * forward on `stream` (same device); moe_forward_graph_destroy releases the
+ * graph (NULL is a no-op; the caller finishes its launches first).  Errors:
+ * MOE_ERR_ARG for the sizes and pointers moe_forward_ex rejects, for T == 0
+ * and for a NULL out; MOE_ERR_CUDA if capture or instantiation fails (the
+ * stream the caller uses is not touched). */
+typedef struct moe_graph moe_graph;
+moe_status moe_forward_graph_create(const void* x, const void* Wg, const float* bias,
+                                    const void* W1, const void* W3, const void* W2,
+                                    int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
+                                    double capacity_factor, moe_act act, moe_dtype dtype,
+                                    const moe_options* opt, void* y, void* ws, size_t ws_bytes,
+                                    moe_graph** out);
+moe_status moe_forward_graph_launch(moe_graph* g, void* stream);
+moe_status moe_forward_graph_destroy(moe_graph* g);
+
 /* Stage timing.  `events` points to MOE_NUM_STAGE_EVENTS cudaEvent_t
  * handles (passed as void*) created by the caller, or is NULL to stop.  The
  * next moe_forward / moe_forward_host calls on the calling host thread

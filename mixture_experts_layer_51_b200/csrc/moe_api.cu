@@ -717,6 +717,89 @@ MOE_API moe_status moe_pipeline_destroy(moe_pipeline* p) {
   return st;
 }
 
+// ================================================================ graphs
+struct moe_graph {
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+  int device;
+};
+
+MOE_API moe_status moe_forward_graph_create(const void* x, const void* Wg, const float* bias,
+                                            const void* W1, const void* W3, const void* W2,
+                                            int32_t T, int32_t d, int32_t H, int32_t E,
+                                            int32_t k, double cf, moe_act act, moe_dtype dt,
+                                            const moe_options* opt, void* y, void* ws,
+                                            size_t ws_bytes, moe_graph** out) {
+  if (!out) return MOE_ERR_ARG;
+  *out = nullptr;
+  moe_ws_layout L;
+  int gating, priority;
+  float gate_scale;
+  if (!compute_layout(T, d, H, E, k, cf, dt, act, &L) ||
+      !read_options(opt, &gating, &gate_scale, &priority))
+    return MOE_ERR_ARG;
+  if (T == 0 || !x || !Wg || !W1 || !W2 || (act == MOE_SWIGLU && !W3) || !y || !ws ||
+      ws_bytes < L.total || !aligned16(ws))
+    return MOE_ERR_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return MOE_ERR_CUDA;
+  // Stage events are never recorded into a graph.
+  const bool events_on = g_stage_events_on;
+  g_stage_events_on = false;
+  moe_status st = MOE_OK;
+  cudaGraph_t graph = nullptr;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    st = MOE_ERR_CUDA;
+  } else {
+    st = forward_enqueue(x, Wg, bias, W1, W3, W2, T, d, H, E, k, cf, act, dt, y, ws, ws_bytes, L,
+                         cs, true, opt);
+    // The capture always ends, whatever the enqueue returned.
+    if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == MOE_OK) st = MOE_ERR_CUDA;
+  }
+  g_stage_events_on = events_on;
+  cudaGraphExec_t exec = nullptr;
+  if (st == MOE_OK && (!graph || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess))
+    st = MOE_ERR_CUDA;
+  cudaStreamDestroy(cs);
+  moe_graph* g = nullptr;
+  if (st == MOE_OK) {
+    g = static_cast<moe_graph*>(malloc(sizeof(moe_graph)));
+    if (!g) st = MOE_ERR_CUDA;
+  }
+  if (st != MOE_OK) {
+    if (exec) cudaGraphExecDestroy(exec);
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();  // a failed capture leaves no sticky error behind
+    return st;
+  }
+  g->graph = graph;
+  g->exec = exec;
+  g->device = dev;
+  *out = g;
+  return MOE_OK;
+}
+
+MOE_API moe_status moe_forward_graph_launch(moe_graph* g, void* stream) {
+  if (!g) return MOE_ERR_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev != g->device) return MOE_ERR_ARG;
+  return cudaGraphLaunch(g->exec, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+MOE_API moe_status moe_forward_graph_destroy(moe_graph* g) {
+  if (!g) return MOE_OK;
+  moe_status st = MOE_OK;
+  if (cudaGraphExecDestroy(g->exec) != cudaSuccess) st = MOE_ERR_CUDA;
+  if (cudaGraphDestroy(g->graph) != cudaSuccess) st = MOE_ERR_CUDA;
+  free(g);
+  return st;
+}
+
 // ============================================================ expert choice
 namespace {
 

@@ -35,6 +35,7 @@ EXPORTED = (
     "moe_expert_choice_permute", "moe_expert_choice_combine", "moe_expert_choice_layout",
     "moe_expert_choice_workspace_bytes", "moe_forward_expert_choice", "moe_pipeline_create",
     "moe_pipeline_submit", "moe_pipeline_wait", "moe_pipeline_destroy",
+    "moe_forward_graph_create", "moe_forward_graph_launch", "moe_forward_graph_destroy",
 )
 MOE_PIPELINE_MAX_DEPTH = 4
 MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
@@ -193,6 +194,14 @@ def lib():
     L.moe_pipeline_wait.argtypes = [_P, _I32]
     L.moe_pipeline_destroy.restype = ctypes.c_int
     L.moe_pipeline_destroy.argtypes = [_P]
+    L.moe_forward_graph_create.restype = ctypes.c_int
+    L.moe_forward_graph_create.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                           ctypes.c_double, ctypes.c_int, ctypes.c_int, _P, _P,
+                                           _P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_forward_graph_launch.restype = ctypes.c_int
+    L.moe_forward_graph_launch.argtypes = [_P, _P]
+    L.moe_forward_graph_destroy.restype = ctypes.c_int
+    L.moe_forward_graph_destroy.argtypes = [_P]
     L.moe_forward_expert_choice.restype = ctypes.c_int
     L.moe_forward_expert_choice.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                             _D, ctypes.c_int, ctypes.c_int, _P, _P, _SZ,
@@ -524,6 +533,42 @@ def stage_times_ms(events):
     return {name: events[i].elapsed_time(events[i + 1]) for i, name in enumerate(STAGES)}
 
 
+class ForwardGraph:
+    """One forward of ``layer`` on the tensors x -> y captured as a CUDA graph
+    (moe_forward_graph_*): launch() replays it with one host call.  x, y and
+    the workspace are held for the graph's lifetime; each launch reads what x
+    holds when it runs."""
+
+    def __init__(self, layer, x, y):
+        T, d = x.shape
+        assert d == layer.d and y.shape == x.shape and y.dtype == x.dtype
+        self.x, self.y, self.ws = x, y, layer.workspace(T)
+        self.layer = layer
+        h = ctypes.c_void_p()
+        _check(lib().moe_forward_graph_create(
+            _ptr(x), _ptr(layer.Wg), _ptr(layer.bias), _ptr(layer.W1), _ptr(layer.W3),
+            _ptr(layer.W2), T, d, layer.H, layer.E, layer.k, _cf(layer.cf), _act_code(layer.act),
+            _dtype_code(x), ctypes.byref(_options(layer.gating, layer.gate_scale, layer.priority)),
+            _ptr(y), _ptr(self.ws), self.ws.numel(), ctypes.byref(h)), "moe_forward_graph_create")
+        self._h = h
+
+    def launch(self, stream=None):
+        _check(lib().moe_forward_graph_launch(self._h, _stream(self.x.device, stream)),
+               "moe_forward_graph_launch")
+        return self.y
+
+    def close(self):
+        if self._h:
+            _check(lib().moe_forward_graph_destroy(self._h), "moe_forward_graph_destroy")
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 class MoELayer:
     """Weights plus a persistent workspace for repeated forwards on one
     device (no allocation per call)."""
@@ -562,6 +607,11 @@ class MoELayer:
                            self.act, y=y, ws=self.workspace(x.shape[0]), stats=stats,
                            stream=stream, gating=self.gating, gate_scale=self.gate_scale,
                            priority=self.priority)
+
+    def graph(self, x, y=None):
+        """A ForwardGraph of this layer on x (and y, allocated if None)."""
+        y = y if y is not None else torch.empty_like(x)
+        return ForwardGraph(self, x, y)
 
 
 # ------------------------------------------------ expert-choice routing

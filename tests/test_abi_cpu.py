@@ -263,3 +263,34 @@ def test_zipf_token_ids_are_reproducible_and_follow_the_law():
     top = slice(0, 20)
     se = np.sqrt(p[top] * (1 - p[top]) / n)
     assert np.all(np.abs(freq[top] - p[top]) <= 5 * se)
+
+
+def test_combines_require_o_in_the_layer_dtype():
+    """o is stored in the layer dtype; handing the combines an fp32 o for a
+    bf16 layer is refused before any library call."""
+    o = torch.zeros(128, 64, dtype=torch.float32)
+    pos = torch.zeros(4, 2, dtype=torch.int32)
+    with pytest.raises(TypeError):
+        M.moe_unpermute_combine(o, pos, torch.zeros(4, 2), torch.bfloat16)
+    with pytest.raises(TypeError):
+        M.moe_expert_choice_combine(o, pos, torch.zeros(2, 4), torch.bfloat16)
+
+
+def test_graph_arguments_are_checked_before_any_cuda_call(lib):
+    fake = ctypes.c_void_p(256)
+    out = ctypes.c_void_p()
+    args = [fake] * 6 + [64, 64, 128, 4, 2, 0.0, M.MOE_SWIGLU, M.MOE_BF16, None, fake, fake,
+                         1 << 30]
+    assert lib.moe_forward_graph_create(*args, None) == M.MOE_ERR_ARG          # no out
+    bad_T = list(args)
+    bad_T[6] = 0
+    assert lib.moe_forward_graph_create(*bad_T, ctypes.byref(out)) == M.MOE_ERR_ARG
+    small_ws = list(args)
+    small_ws[-1] = 16
+    assert lib.moe_forward_graph_create(*small_ws, ctypes.byref(out)) == M.MOE_ERR_ARG
+    no_w3 = list(args)
+    no_w3[4] = None
+    assert lib.moe_forward_graph_create(*no_w3, ctypes.byref(out)) == M.MOE_ERR_ARG
+    assert not out.value
+    assert lib.moe_forward_graph_launch(None, None) == M.MOE_ERR_ARG
+    assert lib.moe_forward_graph_destroy(None) == M.MOE_OK
