@@ -62,7 +62,8 @@ extern "C" {
 #define MOE_MAX_EXPERTS 64
 #define MOE_MAX_TOPK 8
 #define MOE_ROW_ALIGN 128
-#define MOE_ABI_VERSION 1
+/* 2: the expert outputs o are in the layer dtype; moe_forward_graph_*. */
+#define MOE_ABI_VERSION 2
 
 typedef enum {
   MOE_OK = 0,

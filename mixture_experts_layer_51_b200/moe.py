@@ -38,6 +38,7 @@ EXPORTED = (
     "moe_forward_graph_create", "moe_forward_graph_launch", "moe_forward_graph_destroy",
 )
 MOE_PIPELINE_MAX_DEPTH = 4
+MOE_ABI_VERSION = 2
 MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
 MOE_PRIORITY_POSITION, MOE_PRIORITY_GATE = 0, 1
 MOE_PERMUTE_STATIC_MAX_INTS = 1 << 18
@@ -118,6 +119,10 @@ def lib():
     L.moe_status_string.restype = ctypes.c_char_p
     L.moe_status_string.argtypes = [ctypes.c_int]
     L.moe_abi_version.restype = _I32
+    if L.moe_abi_version() != MOE_ABI_VERSION:
+        raise RuntimeError(
+            f"{_LIB_PATH} has ABI version {L.moe_abi_version()}, this binding expects "
+            f"{MOE_ABI_VERSION}: rebuild it with `python -m mixture_experts_layer_51_b200.build`")
     L.moe_capacity.restype = _I32
     L.moe_capacity.argtypes = [_I32, _I32, _I32, _D]
     L.moe_max_permuted_rows.restype = _I64

@@ -40,7 +40,7 @@ def test_header_declares_the_binding_names():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == M.MOE_ABI_VERSION == 2
 
 
 def test_status_strings(lib):
