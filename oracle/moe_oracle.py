@@ -7,7 +7,7 @@ Every array is cast to float64 on entry.  Inputs stored as bf16 are exactly
 representable in float64, so the oracle sees the same numbers the GPU sees and
 computes the definition without any intermediate rounding.
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open:
 
 * Order of TopK and Softmax: Softmax over the k selected logits (the Mixtral
   form in "The Math Behind MoEs"); the non-selected gates are 0.
