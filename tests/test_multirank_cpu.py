@@ -124,3 +124,24 @@ def test_sharded_capacity_exchange_gloo():
     assert g0 == g1 == [np.bincount(idx[a:b].reshape(-1), minlength=8).tolist()
                         for a, b in zip(bounds[:-1], bounds[1:])]
     assert (np.concatenate([np.array(kept0), np.array(kept1)]) == want).all()
+
+
+def test_bench_algorithmic_units_and_l2_note():
+    """The roofline's algorithmic units: FLOPs and bytes of each stage, kept
+    assignments only, o counted in the layer dtype."""
+    import bench
+    from mixture_experts_layer_51_b200.workloads import WORKLOADS
+    w = WORKLOADS["mixtral_bf16"]
+    T, d, E, k, H = w.T, w.d, w.E, w.k, w.H
+    n_kept = T * k
+    flop, byts, total = bench.algorithmic(w, n_kept, T)
+    assert flop["ffn_up"] == 4 * d * H * n_kept and flop["ffn_down"] == 2 * d * H * n_kept
+    assert total == 2 * T * d * E + 6 * d * H * n_kept
+    assert byts["route"] == T * d * 2 + d * E * 2 + 8 * T * k + 4 * T
+    assert byts["combine"] == n_kept * d * 2 + 8 * T * k + T * d * 2
+    assert byts["ffn_down"] == E * H * d * 2 + n_kept * H * 2 + n_kept * d * 2
+    f32 = WORKLOADS["switch_tiny_fp32"]
+    _, b32, _ = bench.algorithmic(f32, 200, 200)
+    assert b32["combine"] == 200 * f32.d * 4 + 8 * f32.T * f32.k + f32.T * f32.d * 4
+    assert bench.l2_note(w).startswith("inputs larger than L2")
+    assert bench.l2_note(f32).startswith("inputs fit in L2")
