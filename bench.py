@@ -25,6 +25,8 @@ import sys
 import tempfile
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -294,6 +296,12 @@ def main(argv=None):
     pos = layer.intermediates(w.T)["pos"]
     tokens_with_kept = int((pos >= 0).any(dim=1).sum().item())
     flop, byts, total_flop = algorithmic(w, n_kept, tokens_with_kept, a.routing)
+    routing = None
+    if not ec:
+        try:
+            routing = routing_report(w, list(st.counts), (pos >= 0).cpu().numpy())
+        except Exception as exc:  # a report, never a reason to lose the measurement
+            routing = {"error": str(exc)}
 
     # Token choice replays the forward as one CUDA graph (moe_forward_graph_*):
     # the same kernels, one host call per step, so layers whose forward is
@@ -451,7 +459,7 @@ def main(argv=None):
             "tflops": round(tflops, 2),
             "frac_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
             "frac_bf16_peak_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
-            "kept_assignments": n_kept, "flop_per_step": total_flop,
+            "kept_assignments": n_kept, "flop_per_step": total_flop, "routing_stats": routing,
             "stages": stages, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_forward * a.steps, "clocks": clk,
             "peaks": {**peaks, "source": peak_src},
@@ -463,6 +471,26 @@ def main(argv=None):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def routing_report(w, counts, kept_mask):
+    """Observability of one forward's routing: load imbalance (largest
+    expert count over the mean), assignments dropped by the capacity, and,
+    with a capacity, the drop rate per octile of batch position and of
+    position inside each sequence ("Drop-towards-the-End").  counts: [E]
+    assignments per expert; kept_mask: [T, k] bool (pos >= 0)."""
+    counts = np.asarray(counts[:w.E], dtype=np.float64)
+    kept_mask = np.asarray(kept_mask, dtype=bool)
+    rep = {"load_imbalance": round(float(counts.max() / max(counts.mean(), 1e-30)), 4),
+           "assignments": int(kept_mask.size), "dropped": int((~kept_mask).sum())}
+    if w.cf > 0 and w.T >= 8:
+        seq = w.seq_len or w.T
+        for label, p, span in (("drop_rate_by_batch_octile", np.arange(w.T), w.T),
+                               ("drop_rate_by_sequence_octile", np.arange(w.T) % seq, seq)):
+            step = max(1, span // 8)
+            rep[label] = [round(float((~kept_mask[(p >= a) & (p < a + step)]).mean()), 4)
+                          for a in range(0, step * 8, step) if ((p >= a) & (p < a + step)).any()]
+    return rep
 
 
 def l2_note(w):

@@ -145,3 +145,22 @@ def test_bench_algorithmic_units_and_l2_note():
     assert b32["combine"] == 200 * f32.d * 4 + 8 * f32.T * f32.k + f32.T * f32.d * 4
     assert bench.l2_note(w).startswith("inputs larger than L2")
     assert bench.l2_note(f32).startswith("inputs fit in L2")
+
+
+def test_bench_routing_report():
+    """Load imbalance, drops and drop rate by position octile from counts and
+    the kept mask (the statistics forward's numbers)."""
+    import numpy as np
+    import bench
+    from mixture_experts_layer_51_b200.workloads import WORKLOADS
+    w = WORKLOADS["openmoe_skew_bf16"].replace(T=64, E=4, k=2, seq_len=16, cf=1.0)
+    kept = np.ones((64, 2), dtype=bool)
+    kept[48:, 1] = False            # the last quarter of the batch loses its 2nd slot
+    counts = [64, 32, 16, 16]
+    r = bench.routing_report(w, counts, kept)
+    assert r["load_imbalance"] == 2.0 and r["assignments"] == 128 and r["dropped"] == 16
+    assert r["drop_rate_by_batch_octile"] == [0, 0, 0, 0, 0, 0, 0.5, 0.5]
+    # position inside each 16-token sequence: only the last sequence drops
+    assert r["drop_rate_by_sequence_octile"] == [0.125] * 8
+    dropless = bench.routing_report(w.replace(cf=0.0), counts, np.ones((64, 2), bool))
+    assert dropless["dropped"] == 0 and "drop_rate_by_batch_octile" not in dropless
