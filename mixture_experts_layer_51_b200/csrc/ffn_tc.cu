@@ -10,26 +10,33 @@
 // Two launches of one persistent, warp-specialised kernel:
 //   up:   h[rows, H] = SiLU(xp W1_e) * (xp W3_e)   (bf16 out; GELU variant)
 //   down: o[rows, d] = h W2_e                      (bf16 out)
-// Tiles are 128 rows x 256 accumulator columns.  For the up projection the
-// 256 columns are 128 columns of W1 next to the same 128 columns of W3, so
-// one accumulator holds both halves of the SwiGLU and the epilogue writes
-// SiLU(gate) * up directly: the two pre-activations never reach HBM.
+// Tiles are 256 rows x 256 accumulator columns, computed by a cluster of two
+// CTAs (tcgen05 cta_group::2: each CTA holds 128 rows of A and half of the
+// 256 B columns; the pair MMA writes each CTA's 128 rows into its own TMEM).
+// For the up projection the 256 columns are 128 columns of W1 next to the
+// same 128 columns of W3 (one CTA loads each), so one accumulator holds both
+// halves of the SwiGLU and the epilogue writes SiLU(gate) * up directly: the
+// two pre-activations never reach HBM.  MOE_TC_CTA_PAIR=0 selects one CTA
+// per 128 x 256 tile instead.
 //
-// Roles (192 threads; 320 with MOE_EPI_WARPS=8):
+// Roles per CTA (192 threads; 320 with MOE_EPI_WARPS=8):
 //   warp 0      one thread issues TMA loads of A (K-major, 128B swizzle) and
-//               B (weights [E, K, N] read N-major, 128B swizzle) into a
-//               4-stage shared-memory ring;
-//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
-//               fp32 accumulate in tensor memory) and commits stage releases;
-//               the warp also owns the 512-column TMEM allocation (two
-//               accumulators, so the epilogue of tile i overlaps the MMAs of
-//               tile i+1);
-//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, activation,
-//               16-byte global stores of the kept rows.  (Eight epilogue
-//               warps, two per lane quadrant, measured no faster once the
-//               SiLU division was the approximate one: the IEEE division had
-//               made the SwiGLU epilogue, not the MMAs, the limit of layers
-//               with K = 1024, by 1.6x.)
+//               B (weights [E, K, N] read N-major, 128B swizzle) into a ring
+//               of three 64 KB stages of 128-wide K steps (six 32 KB stages
+//               of 64-wide steps when K or N is not a multiple of 64), the
+//               peer's bytes completing on the leader's barrier;
+//   warp 1      the leader's thread issues tcgen05.mma (M=256, N=256, K=16,
+//               bf16 in, fp32 accumulate in tensor memory) and commits stage
+//               releases to both CTAs; the warp also owns the 512-column TMEM
+//               allocation (two accumulators, so the epilogue of tile i
+//               overlaps the MMAs of tile i+1);
+//   warps 2-5   epilogue: tcgen05.ld of their 32 TMEM lanes, activation or
+//               rounding to bf16, stores of the kept rows (h: 16-byte stores
+//               per row; o: swizzled 32-row staging boxes and TMA stores).
+//               (Eight epilogue warps, two per lane quadrant, measured no
+//               faster once the SiLU division was the approximate one: the
+//               IEEE division had made the SwiGLU epilogue, not the MMAs,
+//               the limit of layers with K = 1024, by 1.6x.)
 // The tile list (expert, m-block, n-block) is built on the device from the
 // per-expert offsets, with the experts that have the most m-blocks first and
 // m-blocks fastest, so concurrent CTAs share weight tiles in L2.  No host
