@@ -18,7 +18,8 @@
  *   The caller allocates and owns every buffer; the library never allocates
  *   or frees device memory and keeps no pointer after a call returns (a
  *   moe_pipeline handle, created and destroyed by the caller, owns copy
- *   streams, events and a few bytes of pinned host memory).
+ *   streams, events and a few bytes of pinned host memory; a moe_graph
+ *   handle holds the pointers its forward was captured with).
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream).  All work is enqueued on it; calls return without waiting for
  *   the GPU, except that moe_forward(_ex) and moe_forward_expert_choice
