@@ -60,6 +60,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-kernels", action="store_true",
+                    help="skip the back-to-back timing of the HBM-bound kernels")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the timed loops of the other layer shapes")
     ap.add_argument("--cpu-sample", type=int, default=None,
                     help="tokens per oracle sample (default: sized to ~10-20 s)")
     return ap.parse_args(argv)
@@ -109,6 +113,38 @@ def algorithmic(w, n_kept, tokens_with_kept, routing="token_choice"):
         byts["combine"] = n_kept * d * s + T * E * 8 + T * d * s
     total_flop = flop["route"] + flop["ffn_up"] + flop["ffn_down"]
     return flop, byts, total_flop
+
+
+# A roofline fraction above this means the timed kernel is not doing the
+# work it is credited with (or the wrong peak was used): the line is refused.
+MAX_ROOFLINE_FRAC = 1.05
+
+
+def choose_bf16_peak(peaks, loop_s, clk, src="measured"):
+    """The bf16 denominator that fits the timed region: the sustained
+    (power-capped) figure only when the region is a loop of at least a second
+    whose sampled clocks show sw_power_cap with the median SM clock below 92 %
+    of max; the burst figure otherwise.  Returns (peak, description)."""
+    sustained = (loop_s >= 1.0 and clk is not None and "sw_power_cap" in clk.get("reasons", [])
+                 and clk.get("sm_mhz", 0) < 0.92 * clk.get("sm_max_mhz", 1))
+    clock = (f", median SM clock {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} MHz"
+             f"{' (' + ', '.join(clk['reasons']) + ')' if clk.get('reasons') else ''}"
+             if clk else ", clocks not sampled")
+    if sustained:
+        return peaks["bf16_tflops_sustained"], (
+            f"{src} bf16 sustained: timed loop of {loop_s:.2f} s under the power cap{clock}")
+    return peaks["bf16_tflops"], f"{src} bf16 burst: timed loop of {loop_s:.3f} s{clock}"
+
+
+def roofline_fraction(achieved, peak):
+    """achieved / peak, refusing a value no correct measurement can give."""
+    if achieved is None or not peak:
+        return None
+    frac = achieved / peak
+    if frac > MAX_ROOFLINE_FRAC:
+        raise ValueError(f"roofline fraction {frac:.3f} > {MAX_ROOFLINE_FRAC}: "
+                         f"{achieved:.1f} against a peak of {peak:.1f}")
+    return round(frac, 4)
 
 
 def traffic_for(kernel_file, kernel, w):
@@ -245,6 +281,156 @@ def default_cpu_sample(w):
     return int(max(16, min(w.T, 3e12 / per_token)))
 
 
+# ------------------------------------------------------------- timing
+def forward_loop(step, steps, stream, dev, clocks=None, world=1):
+    """K calls of step() between two events on the launching stream, bracketed
+    by a barrier (N > 1) and a device synchronise; returns (ms, clocks)."""
+    import torch
+    import torch.distributed as dist
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop() if clocks else None
+    return start.elapsed_time(end), clk
+
+
+def stage_loop(M, layer, x, y, n, stream, dev):
+    """n forwards with events recorded between the stages
+    (moe_set_stage_events); returns the mean ms of each stage."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(M.MOE_NUM_STAGE_EVENTS)]
+           for _ in range(n)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize(dev)
+    for i in range(n):
+        M.moe_set_stage_events(evs[i])
+        layer(x, y=y)
+    M.moe_set_stage_events(None)
+    torch.cuda.synchronize(dev)
+    stage_ms = {s: 0.0 for s in M.STAGES}
+    for i in range(n):
+        for s, v in M.stage_times_ms(evs[i]).items():
+            stage_ms[s] += v / n
+    return stage_ms
+
+
+def back_to_back_ms(launches, reps, stream, dev):
+    """Mean ms per launch of `reps` rounds over the list `launches` (each a
+    callable enqueuing one kernel on `stream`), launched back to back between
+    two events after one untimed round."""
+    import torch
+    for fn in launches:
+        fn()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(reps):
+        for fn in launches:
+            fn()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    return start.elapsed_time(end) / (reps * len(launches))
+
+
+def hbm_kernels(M, w, layer, x, inp, byts, hbm, stream, dev):
+    """The HBM-bound stages timed as kernels: each launched back to back
+    through its own entry point on inputs that rotate through copies of x
+    (more than twice the 126 MB L2 between two reads of one copy), beside a
+    plain streaming read of the same bytes (moe_probe_stream_read).  The
+    stage-event loop's figures include the gap every event opens between two
+    kernels; these do not."""
+    import torch
+    T = w.T
+    nbytes = x.numel() * x.element_size()
+    copies = max(2, min(64, -(-252_000_000 // max(nbytes, 1)) + 1))
+    xs = [x.clone() for _ in range(copies)]
+    v = layer.intermediates(T)
+    idx, gate, margin, pos = v["idx"], v["gate"], v["margin"], v["pos"]
+    idx2, gate2, margin2 = torch.empty_like(idx), torch.empty_like(gate), torch.empty_like(margin)
+    perm = {k: torch.empty_like(v[k]) for k in ("pos", "counts", "kept_counts", "offsets")}
+    xp = torch.empty_like(v["xp"])
+    ws = torch.empty(M.moe_permute_workspace_bytes(T, w.E), dtype=torch.uint8, device=dev)
+    yb = torch.empty_like(x)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    reps = 10
+    out = {}
+    ms = back_to_back_ms([lambda xx=xx: M.moe_probe_stream_read(xx, sink) for xx in xs],
+                         reps, stream, dev)
+    out["plain_read"] = {"ms": round(ms, 5), "bytes": nbytes,
+                         "gbs": round(nbytes / (ms / 1e3) / 1e9, 1),
+                         "frac_hbm": round(nbytes / (ms / 1e3) / 1e9 / hbm, 4)}
+    routes = [lambda xx=xx: M.moe_route(xx, inp["Wg"], inp["bias"], w.k, idx2, gate2, margin2)
+              for xx in xs]
+    permutes = [lambda xx=xx: M.moe_permute(xx, idx, w.E, w.cf, xp=xp, ws=ws, **perm)
+                for xx in xs]
+    combines = [lambda: M.moe_unpermute_combine(v["o"], pos, gate, x.dtype, y=yb)]
+    for name, fns in (("route", routes), ("permute", permutes), ("combine", combines)):
+        ms = back_to_back_ms(fns, reps if len(fns) > 1 else 2 * copies, stream, dev)
+        gbs = byts[name] / (ms / 1e3) / 1e9
+        out[name] = {"ms": round(ms, 5), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                     "of_plain_read": round(out["plain_read"]["ms"] * byts[name] / nbytes / ms, 4)}
+    out["method"] = (f"each entry point launched back to back ({reps} rounds over {copies} copies "
+                     f"of x, {copies * nbytes / 1e6:.0f} MB; combine re-reads o "
+                     f"{v['o'].numel() * v['o'].element_size() / 1e6:.0f} MB), CUDA events on "
+                     "the launching stream; of_plain_read = the probe's time for the stage's "
+                     "algorithmic bytes / the stage's time")
+    del xs
+    return out
+
+
+def workload_record(M, w, make_inputs, peaks, peak_src, dev, stream, seconds=1.5,
+                    sample_clocks=True):
+    """One workload's forward, replayed as its CUDA graph in a timed loop of
+    about `seconds` (clocks sampled), plus its stage breakdown."""
+    import torch
+    inp = make_inputs(w, dev)
+    layer = M.MoELayer(inp["Wg"], inp["bias"], inp["W1"], inp["W3"], inp["W2"], w.k, w.cf,
+                       w.act, max_tokens=w.T)
+    x = inp["x"]
+    y = torch.empty_like(x)
+    _, st = layer(x, y=y, stats=True)
+    n_kept = int(st.kept)
+    pos = layer.intermediates(w.T)["pos"]
+    tokens_with_kept = int((pos >= 0).any(dim=1).sum().item())
+    flop, byts, total_flop = algorithmic(w, n_kept, tokens_with_kept)
+    graph = layer.graph(x, y)
+    for _ in range(5):
+        graph.launch()
+    cal_ms, _ = forward_loop(graph.launch, 10, stream, dev)
+    steps = int(min(50000, max(20, seconds * 1e3 / max(cal_ms / 10, 1e-3))))
+    clocks = ClockSampler(dev.index or 0) if sample_clocks else None
+    ms, clk = forward_loop(graph.launch, steps, stream, dev, clocks)
+    graph.close()
+    stage_ms = stage_loop(M, layer, x, y, 20, stream, dev)
+    ms_step = ms / steps
+    tflops = total_flop / (ms_step / 1e3) / 1e12
+    rec = {"T": w.T, "d": w.d, "E": w.E, "k": w.k, "H": w.H, "act": w.act, "dtype": w.dtype,
+           "capacity_factor": w.cf, "steps": steps, "ms_per_step": round(ms_step, 5),
+           "tokens_per_s": round(w.T / (ms_step / 1e3), 1), "tflops": round(tflops, 2),
+           "kept_assignments": n_kept, "clocks": clk,
+           "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()}}
+    if w.dtype == "bf16":
+        peak, src = choose_bf16_peak(peaks, ms / 1e3, clk, peak_src)
+        rec.update({"frac_bf16_peak": roofline_fraction(tflops, peak), "peak": peak,
+                    "peak_source": src})
+    else:
+        rec["bound"] = "latency (8.5 MFLOP per forward; a fraction of an FP32 peak means nothing)"
+    del layer, inp, x, y
+    torch.cuda.empty_cache()
+    return rec
+
+
 # ----------------------------------------------------------------- main
 def main(argv=None):
     a = parse_args(argv)
@@ -312,6 +498,7 @@ def main(argv=None):
             graph = layer.graph(x, y)
         except M.MoeError as exc:
             print(f"graph capture unavailable ({exc}); timing eager launches", file=sys.stderr)
+    launch_kind = "cuda_graph" if graph is not None else "eager"
     step = graph.launch if graph is not None else (lambda: layer(x, y=y))
     for _ in range(a.warmup):
         step()
@@ -320,21 +507,8 @@ def main(argv=None):
     # The timed loop: K forwards back to back, nothing recorded between
     # their kernels (an event between two kernels would stop the next one
     # from starting while the previous drains).
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local) if not a.no_clocks else None
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    start.record(stream)
-    for i in range(a.steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    clk = clocks.stop() if clocks else None
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms, clk = forward_loop(step, a.steps, stream, dev, clocks, world)
     if world > 1:
         dist.barrier()
     elapsed_ms = max_over_ranks(elapsed_ms, dev)
@@ -342,21 +516,9 @@ def main(argv=None):
     # Stage breakdown from a separate loop with events recorded between the
     # stages (moe_set_stage_events), on the launching stream.
     n_stage = min(a.steps, 50)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(M.MOE_NUM_STAGE_EVENTS)]
-           for _ in range(n_stage)]
-    for row in evs:  # torch creates the CUDA event on first record
-        for ev in row:
-            ev.record(stream)
-    torch.cuda.synchronize(dev)
-    for i in range(n_stage):
-        M.moe_set_stage_events(evs[i])
-        layer(x, y=y)
-    M.moe_set_stage_events(None)
-    torch.cuda.synchronize(dev)
-    stage_ms = {s: 0.0 for s in M.STAGES}
-    for i in range(n_stage):
-        for s, v in M.stage_times_ms(evs[i]).items():
-            stage_ms[s] += v / n_stage
+    t_stage = time.perf_counter()
+    stage_ms = stage_loop(M, layer, x, y, n_stage, stream, dev)
+    stage_loop_s = time.perf_counter() - t_stage
 
     # Kernels of ours per timed forward: router, count, rank, copy, two
     # GEMMs, combine (token choice); router, select, transpose, copy, two
@@ -365,6 +527,11 @@ def main(argv=None):
     ms_per_step = elapsed_ms / a.steps
     tokens_per_s = whole_job_rate(w.T, world, a.steps, elapsed_ms)
     tflops = total_flop * world * a.steps / (elapsed_ms / 1e3) / 1e12
+    hbm = peaks["hbm_gbs"]
+
+    kernels = None
+    if not ec and world == 1 and not a.no_kernels:
+        kernels = hbm_kernels(M, w, layer, x, inp, byts, hbm, stream, dev)
 
     # End to end: every step copies its own batch from pinned host memory,
     # runs the layer and copies y back, through the streaming pipeline API
@@ -413,9 +580,9 @@ def main(argv=None):
         cpu = {"value": T_s / secs, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"first {T_s} tokens of the {w.name} batch (routing, capacity, expert "
                          f"FFNs, combine in fp64 NumPy), {secs:.1f} s"}
+        del cpu_inp
 
     up_ms = stage_ms["ffn_up"]
-    hbm = peaks["hbm_gbs"]
     stages = {}
     for s in M.STAGES:
         ms = stage_ms[s]
@@ -429,11 +596,14 @@ def main(argv=None):
     act_name = "SwiGLU" if w.act == "swiglu" else "GELU"
     achieved = flop["ffn_up"] / (up_ms / 1e3) / 1e12 if up_ms > 0 else None
     if w.dtype == "bf16":
-        roof_peak = peaks["bf16_tflops_sustained"]
+        # The achieved rate comes from the stage loop, so its length and the
+        # clocks of the headline loop just before it pick the peak.
+        roof_peak, roof_src = choose_bf16_peak(peaks, stage_loop_s, clk, peak_src)
         roofline = {"kernel": f"ffn_tc_kernel<{act_name}> (grouped up projection)",
                     "bound": "tensor",
                     "traffic": traffic_for("ffn_tc.cu", "ffn_up", w),
-                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long loop)"}
+                    "peak_source": roof_src + f"; achieved from the stage loop of {n_stage} "
+                                              "forwards"}
     else:
         # fp32 FMA on the SIMT pipes: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
         roof_peak = FP32_SIMT_TFLOPS
@@ -441,8 +611,28 @@ def main(argv=None):
                     "bound": "alu", "traffic": None,
                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz"}
     roofline.update({"achieved": round(achieved, 2) if achieved else None, "peak": roof_peak,
-                     "unit": "TFLOP/s",
-                     "frac": round(achieved / roof_peak, 4) if achieved else None})
+                     "unit": "TFLOP/s", "frac": roofline_fraction(achieved, roof_peak)})
+    layer_peak, layer_src = (choose_bf16_peak(peaks, elapsed_ms / 1e3, clk, peak_src)
+                             if w.dtype == "bf16" else (peaks["bf16_tflops"], ""))
+
+    # The other layer shapes, each in a timed loop of its own (N = 1 only).
+    others = None
+    if rank == 0 and world == 1 and not a.no_workloads and not ec and a.workload == DEFAULT_WORKLOAD \
+            and not (a.tokens or a.experts or a.hidden) and a.capacity_factor is None:
+        if graph is not None:
+            graph.close()
+            graph = None
+        del layer, inp, x, y
+        torch.cuda.empty_cache()
+        others = {}
+        for name, wl in WORKLOADS.items():
+            if name == w.name:
+                continue
+            try:
+                others[name] = workload_record(M, wl, make_inputs, peaks, peak_src, dev, stream,
+                                               sample_clocks=not a.no_clocks)
+            except Exception as exc:  # one shape failing must not lose the headline
+                others[name] = {"error": f"{type(exc).__name__}: {exc}"}
 
     if rank == 0:
         line = {
@@ -454,15 +644,19 @@ def main(argv=None):
             "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "H": w.H,
                        "act": w.act, "capacity_factor": w.cf, "routing": a.routing,
                        "parallelism": f"replicas x{world}",
-                       "launch": "cuda_graph" if graph is not None else "eager",
+                       "launch": launch_kind,
                        "l2": l2_note(w)},
             "tflops": round(tflops, 2),
-            "frac_bf16_peak": round(tflops / peaks["bf16_tflops"], 4),
+            "frac_bf16_peak": round(tflops / layer_peak, 4),
+            "frac_bf16_peak_source": layer_src,
+            "frac_bf16_peak_burst": round(tflops / peaks["bf16_tflops"], 4),
             "frac_bf16_peak_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4),
             "kept_assignments": n_kept, "flop_per_step": total_flop, "routing_stats": routing,
-            "stages": stages, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "stages": stages, "hbm_kernels": kernels, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": kernels_per_forward * a.steps, "clocks": clk,
             "peaks": {**peaks, "source": peak_src},
+            "workloads": others,
         }
         print(json.dumps(line), flush=True)
     if graph is not None:

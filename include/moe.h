@@ -481,6 +481,18 @@ moe_status moe_forward_expert_choice(const void* x, const void* Wg, const float*
                                      void* y, void* ws, size_t ws_bytes, moe_stats* stats,
                                      void* stream);
 
+/* ------------------------------------------------------ measurement aid
+ * No counterpart on the pages: a yardstick for the HBM-bound stages.  Reads
+ * `bytes` of the device buffer `buf` once with streaming 16-byte loads (two
+ * 512-thread CTAs per SM, each a contiguous slice, eight loads in flight per
+ * thread) and XORs one word per warp into *sink (device, 4 bytes, caller
+ * owned; its value means nothing).  The router reads x once and the
+ * permutation and combine copy rows, so the time this takes for the same
+ * number of bytes is what "as fast as a plain read" means on this GPU at
+ * that size.  bytes must be a multiple of 16 and buf 16-byte aligned
+ * (MOE_ERR_ARG otherwise); bytes == 0 is a no-op.  Enqueued on `stream`. */
+moe_status moe_probe_stream_read(const void* buf, size_t bytes, uint32_t* sink, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

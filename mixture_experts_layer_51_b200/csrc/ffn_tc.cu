@@ -382,11 +382,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!mbar_wait(full0 + 8 * s, static_cast<uint32_t>(fills - 1) & 1u))
               atomicOr(p.err, kErrTimeoutDrain);
           }
-        } else {
-          // The peer's copies complete on the leader's barrier, which this
-          // CTA cannot poll; give them time to land.
-          for (int i = 0; i < 100; ++i) __nanosleep(1000);
         }
+        // The peer's copies complete on the leader's barriers, which the peer
+        // cannot poll.  Nothing is needed here for them: a copy the leader
+        // armed is covered by the leader's wait above, which ends before the
+        // leader reaches the teardown cluster barrier, and the peer cannot
+        // leave before that barrier.  A copy the leader never armed exists
+        // only if the leader stopped issuing first; the MMA then stalls on
+        // that stage and releases no more stages, so the peer issues nothing
+        // more and leaves its loop only when one of its own bounded waits
+        // (2 s) runs out -- its producer's on a stage that is never released,
+        // or its epilogue's on an accumulator the stalled MMA never fills --
+        // long after its last copy landed.
       }
     }
   } else if (warp == 1) {

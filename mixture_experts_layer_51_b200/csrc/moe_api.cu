@@ -992,3 +992,16 @@ MOE_API moe_status moe_forward_expert_choice(const void* x, const void* Wg, cons
     return MOE_ERR_CUDA;
   return stats->device_error ? MOE_ERR_DEVICE : MOE_OK;
 }
+
+MOE_API moe_status moe_probe_stream_read(const void* buf, size_t bytes, uint32_t* sink,
+                                         void* stream) {
+  if (bytes == 0) return MOE_OK;
+  if (!buf || !sink || bytes % 16 != 0 || !aligned16(buf)) return MOE_ERR_ARG;
+  DeviceInfo di;
+  moe_status st = device_info(&di);
+  if (st != MOE_OK) return st;
+  return launch_stream_read(buf, bytes, sink, di.num_sms, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}

@@ -498,4 +498,9 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, moe_dtype dtype, cudaStream_t s);
 
+// Measurement aid (probe.cu): read `bytes` (a multiple of 16) of `buf` once
+// with streaming 16-byte loads; one XOR word per warp lands in *sink.
+cudaError_t launch_stream_read(const void* buf, size_t bytes, uint32_t* sink, int num_sms,
+                               cudaStream_t s);
+
 }  // namespace moe

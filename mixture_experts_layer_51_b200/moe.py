@@ -36,6 +36,7 @@ EXPORTED = (
     "moe_expert_choice_workspace_bytes", "moe_forward_expert_choice", "moe_pipeline_create",
     "moe_pipeline_submit", "moe_pipeline_wait", "moe_pipeline_destroy",
     "moe_forward_graph_create", "moe_forward_graph_launch", "moe_forward_graph_destroy",
+    "moe_probe_stream_read",
 )
 MOE_PIPELINE_MAX_DEPTH = 4
 MOE_ABI_VERSION = 2
@@ -217,6 +218,8 @@ def lib():
     L.moe_priority_order.argtypes = [_P, _I32, _I32, _P, _P, _SZ, _P]
     L.moe_set_stage_events.restype = ctypes.c_int
     L.moe_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_probe_stream_read.restype = ctypes.c_int
+    L.moe_probe_stream_read.argtypes = [_P, _SZ, _P, _P]
     _lib_handle = L
     return L
 
@@ -519,6 +522,14 @@ class Pipeline:
             self.close()
         except Exception:
             pass
+
+
+def moe_probe_stream_read(buf, sink, stream=None):
+    """Measurement aid: read every byte of the device tensor ``buf`` once
+    (a plain streaming read); ``sink`` is a 1-element int32 device tensor."""
+    nbytes = buf.numel() * buf.element_size()
+    _check(lib().moe_probe_stream_read(_ptr(buf), nbytes, _ptr(sink),
+                                       _stream(buf.device, stream)), "moe_probe_stream_read")
 
 
 def moe_set_stage_events(events):

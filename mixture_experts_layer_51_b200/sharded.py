@@ -47,7 +47,12 @@ def moe_forward_sharded(layer, x, global_tokens=None, group=None, stream=None):
     layer: an ``moe.MoELayer`` (position priority; Batch Priority Routing
     ranks tokens over the whole batch and is not sharded here).
     global_tokens: tokens in the whole batch; default T_r * world (equal
-    shards).  Returns y [T_r, d] and a dict of the intermediates.
+    shards).  stream: the CUDA stream to run on (default: the current one).
+    Every kernel, the all-gather and every allocation run on that one stream,
+    which first waits for the caller's current stream (where x was made);
+    the caller's stream then waits for it, and the returned tensors are
+    recorded as used there.  Returns y [T_r, d] and a dict of the
+    intermediates.
     """
     if layer.priority != "position":
         raise ValueError("sharded capacity supports position priority only")
@@ -55,14 +60,25 @@ def moe_forward_sharded(layer, x, global_tokens=None, group=None, stream=None):
     rank = dist.get_rank(group)
     world = dist.get_world_size(group)
     T_all = T * world if global_tokens is None else int(global_tokens)
-    idx, gate, _ = M.moe_route(x, layer.Wg, layer.bias, layer.k, stream=stream,
-                               gating=layer.gating, gate_scale=layer.gate_scale)
-    counts = M.moe_expert_counts(idx, layer.E, stream=stream)
-    gathered = gather_expert_counts(counts, group)
-    prior = M.moe_rank_prefix(gathered, rank, stream=stream)
-    C = M.moe_capacity(T_all, layer.E, layer.k, layer.cf)
-    perm = M.moe_permute(x, idx, layer.E, layer.cf, stream=stream, prior=prior, capacity=C)
-    h, o, dev_error = M.moe_grouped_ffn(perm["xp"], perm["offsets"], perm["kept_counts"],
-                                        layer.W1, layer.W3, layer.W2, layer.act, stream=stream)
-    y = M.moe_unpermute_combine(o, perm["pos"], gate, x.dtype, stream=stream)
-    return y, dict(idx=idx, gate=gate, prior=prior, capacity=C, dev_error=dev_error, **perm)
+    caller = torch.cuda.current_stream(x.device)
+    s = caller if stream is None else stream
+    if s != caller:
+        s.wait_stream(caller)
+    with torch.cuda.stream(s):
+        idx, gate, _ = M.moe_route(x, layer.Wg, layer.bias, layer.k, gating=layer.gating,
+                                   gate_scale=layer.gate_scale)
+        counts = M.moe_expert_counts(idx, layer.E)
+        gathered = gather_expert_counts(counts, group)
+        prior = M.moe_rank_prefix(gathered, rank)
+        C = M.moe_capacity(T_all, layer.E, layer.k, layer.cf)
+        perm = M.moe_permute(x, idx, layer.E, layer.cf, prior=prior, capacity=C)
+        h, o, dev_error = M.moe_grouped_ffn(perm["xp"], perm["offsets"], perm["kept_counts"],
+                                            layer.W1, layer.W3, layer.W2, layer.act)
+        y = M.moe_unpermute_combine(o, perm["pos"], gate, x.dtype)
+    info = dict(idx=idx, gate=gate, prior=prior, capacity=C, dev_error=dev_error, **perm)
+    if s != caller:
+        caller.wait_stream(s)
+        x.record_stream(s)
+        for t in [y] + [v for v in info.values() if torch.is_tensor(v)]:
+            t.record_stream(caller)
+    return y, info

@@ -95,10 +95,31 @@ def check_routing(g, logits, k, gating="topk_softmax", gate_scale=1.0):
     return int((~far).sum()), idx_o
 
 
+def check_xp_rows(xp_view, x, want_pos, kept, chunk=1 << 16):
+    """Every kept row of xp is a bit-exact copy of its token's x row, at the
+    row the oracle's positions name.  x: a torch tensor (compared on xp's
+    device, in chunks, so full-size buffers never reach the host) or a numpy
+    array (small cases)."""
+    tt, jj = np.nonzero(kept)
+    rows = want_pos[tt, jj]
+    if torch.is_tensor(x):
+        x = x.to(xp_view.device)
+        for a in range(0, tt.size, chunk):
+            r = torch.as_tensor(rows[a:a + chunk], device=xp_view.device, dtype=torch.long)
+            s = torch.as_tensor(tt[a:a + chunk], device=xp_view.device, dtype=torch.long)
+            assert torch.equal(xp_view.index_select(0, r), x.index_select(0, s)), (
+                f"xp rows {a}..{a + r.numel()} are not exact copies")
+        return
+    r = torch.as_tensor(rows, device=xp_view.device, dtype=torch.long)
+    got = to_np(xp_view.index_select(0, r).float())
+    assert np.array_equal(got, x[tt].astype(np.float32)), "xp rows are not exact copies"
+
+
 def check_permutation(g, x_np, T, E, k, cf, xp_view=None, priority="position"):
     """Teacher-forced permutation: bit-exact against the oracle's capacity
     step run on the GPU's own indices (and, for priority routing, on the
-    oracle's order of the GPU's own gates)."""
+    oracle's order of the GPU's own gates).  With xp_view, every kept row of
+    xp is checked too (x_np: the layer input, numpy or torch)."""
     C = oracle.capacity(T, E, k, cf)
     order = None
     if priority == "gate" and C is not None:
@@ -112,10 +133,7 @@ def check_permutation(g, x_np, T, E, k, cf, xp_view=None, priority="position"):
     want_pos = np.where(kept, off[g["idx"]] + rank, -1)
     assert (g["pos"] == want_pos).all()
     if xp_view is not None and kept.any():
-        tt, jj = np.nonzero(kept)
-        rows = torch.as_tensor(want_pos[tt, jj], device=xp_view.device, dtype=torch.long)
-        got = to_np(xp_view.index_select(0, rows).float())
-        assert np.array_equal(got, x_np[tt].astype(np.float32)), "xp rows are not exact copies"
+        check_xp_rows(xp_view, x_np, want_pos, kept)
     return kept, C
 
 

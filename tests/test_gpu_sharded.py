@@ -102,8 +102,11 @@ def _free_port():
     return port
 
 
-def test_forward_sharded_single_rank_equals_forward():
-    """moe_forward_sharded over a one-rank NCCL group is the plain layer."""
+@pytest.mark.parametrize("side_stream", [False, True])
+def test_forward_sharded_single_rank_equals_forward(side_stream):
+    """moe_forward_sharded over a one-rank NCCL group is the plain layer, on
+    the current stream or on a side stream (whose kernels, gather and
+    allocations must be ordered against the caller's stream)."""
     import torch.distributed as dist
     from mixture_experts_layer_51_b200.sharded import moe_forward_sharded
     w = Workload("shard1", T=700, d=128, E=8, k=2, H=256, act="swiglu", dtype="bf16", cf=1.0,
@@ -116,12 +119,16 @@ def test_forward_sharded_single_rank_equals_forward():
                             world_size=1,
                             device_id=torch.device("cuda", torch.cuda.current_device()))
     try:
-        y, info = moe_forward_sharded(layer, t["x"])
+        side = torch.cuda.Stream() if side_stream else None
+        y, info = moe_forward_sharded(layer, t["x"], stream=side)
+        # read on the caller's stream without a device-wide synchronise
+        y = y.clone()
+        err = info["dev_error"].clone()
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
     y_ref = layer(t["x"])
     torch.cuda.synchronize()
     assert info["capacity"] == M.moe_capacity(w.T, w.E, w.k, w.cf)
-    assert int(info["dev_error"].item()) == 0
+    assert int(err.item()) == 0
     assert torch.equal(y, y_ref)

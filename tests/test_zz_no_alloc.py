@@ -6,8 +6,9 @@ whose host framework forbids allocation inside its execute call).  For them
 moe_permute_static keeps the permutation's scratch in a fixed array inside
 the library instead of a caller-provided buffer.  These tests call it through
 the C ABI and check that two calls in a row give exactly what moe_permute
-(the entry point with caller-provided scratch) gives.  The file is named to
-be collected last.
+(the entry point with caller-provided scratch) gives, and, directly, what the
+fp64 oracle's capacity step gives on the same expert indices.  The file is
+named to be collected last.
 """
 
 import ctypes
@@ -16,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mixture_experts_layer_51_b200 import moe as M
 from mixture_experts_layer_51_b200.workloads import Workload, make_inputs
 
@@ -48,6 +50,22 @@ def _static_call(x, idx, E, cf):
     return out
 
 
+def _matches_oracle(got, idx, E, k, cf):
+    """Counts, kept counts, 128-row aligned offsets and every position equal
+    the oracle's first-C-by-position queue on the same indices."""
+    T = idx.shape[0]
+    idx_np = idx.cpu().numpy()
+    C = oracle.capacity(T, E, k, cf)
+    counts, kept_counts, rank, kept = oracle.assign_capacity(idx_np, E, C)
+    assert np.array_equal(got["counts"].cpu().numpy(), counts)
+    assert np.array_equal(got["kept_counts"].cpu().numpy(), kept_counts)
+    align = M.MOE_ROW_ALIGN
+    off = np.concatenate([[0], np.cumsum((kept_counts + align - 1) // align * align)])
+    assert np.array_equal(got["offsets"].cpu().numpy(), off)
+    want_pos = np.where(kept, off[idx_np] + rank, -1)
+    assert np.array_equal(got["pos"].cpu().numpy(), want_pos)
+
+
 def _same(ref, got):
     for key in ("counts", "kept_counts", "offsets", "pos"):
         assert torch.equal(ref[key], got[key]), key
@@ -69,6 +87,8 @@ def test_static_permute_matches_permute_on_two_calls(w):
     torch.cuda.synchronize()
     _same(ref, first)
     _same(ref, second)
+    _matches_oracle(first, idx, w.E, w.k, w.cf)
+    _matches_oracle(second, idx, w.E, w.k, w.cf)
     assert int(ref["kept_counts"].sum()) == int((ref["pos"] >= 0).sum())
 
 
@@ -85,6 +105,7 @@ def test_static_permute_after_a_larger_call():
         got = _static_call(inp["x"], idx, w.E, w.cf)
         torch.cuda.synchronize()
         _same(ref, got)
+        _matches_oracle(got, idx, w.E, w.k, w.cf)
 
 
 def test_static_permute_rejects_sizes_beyond_its_scratch():
