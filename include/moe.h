@@ -155,7 +155,8 @@ int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double capacity_f
  * shard of a batch under the whole batch's capacity (moe_permute_ex). */
 int64_t moe_rows_for_capacity(int32_t T, int32_t E, int32_t k, int32_t C);
 
-/* Scratch bytes moe_permute needs in `ws` (per-block counts and a counter). */
+/* Scratch bytes moe_permute needs in `ws`: the per-range expert counts,
+ * 256 x E int32 whatever T is (T only has to be valid). */
 size_t moe_permute_workspace_bytes(int32_t T, int32_t E);
 
 /* Workspace bytes moe_forward needs; 0 on invalid sizes. */
@@ -199,7 +200,11 @@ moe_status moe_route_ex(const void* x, const void* Wg, const float* bias,
  *   moe_max_permuted_rows); pos [T, k] int32 = row of (t, j) in xp, or -1
  *   if dropped; counts [E], kept_counts [E], offsets [E+1] int32.
  *   ws: device scratch of at least moe_permute_workspace_bytes(T, E).
- *   Deterministic: the result does not depend on scheduling. */
+ *   Deterministic: the result does not depend on scheduling.  Two kernels:
+ *   per range of tokens (the streaming router's ranges), each assignment's
+ *   rank among the range's earlier assignments to its expert and the
+ *   range's counts; then, per range, the prefix over earlier ranges gives
+ *   every assignment its place in its expert's queue, and the row copy. */
 moe_status moe_permute(const void* x, const int32_t* idx, int32_t T, int32_t d,
                        int32_t E, int32_t k, double capacity_factor, moe_dtype dtype,
                        void* xp, int64_t xp_rows, int32_t* pos, int32_t* counts,

@@ -109,7 +109,7 @@ bool compute_layout(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k, doubl
   L->kept_counts = take(kMaxE * 4);
   L->offsets = take((kMaxE + 1) * 4);
   L->dev_error = take(4);
-  L->scratch = take(permute_scratch_bytes(T, E));
+  L->scratch = take(ranked_permute_scratch_bytes(E));
   L->order = take(static_cast<size_t>(T) * 4);
   L->prio_scratch = take(priority_scratch_bytes(T));
   L->xp = take(static_cast<size_t>(rows) * d * es);
@@ -157,7 +157,7 @@ MOE_API int64_t moe_max_permuted_rows(int32_t T, int32_t E, int32_t k, double cf
 
 MOE_API size_t moe_permute_workspace_bytes(int32_t T, int32_t E) {
   if (T < 0 || E < 1 || E > kMaxE) return 0;
-  return permute_scratch_bytes(T, E);
+  return ranked_permute_scratch_bytes(E);
 }
 
 MOE_API size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t H, int32_t E, int32_t k,
@@ -173,10 +173,15 @@ MOE_API moe_status moe_workspace_layout(int32_t T, int32_t d, int32_t H, int32_t
 }
 
 namespace {
-// Router; `err` (nullable) receives the tensor-core router's time-out bits.
+// Router; `err` (nullable) receives the routers' time-out bits.  With
+// lrank/hist (nullable) the streaming router also writes the permutation's
+// local ranks and per-range counts; *ranked says whether it did.
 moe_status route_enqueue(const void* x, const void* Wg, const float* bias, int32_t T, int32_t d,
                          int32_t E, int32_t k, moe_dtype dt, const moe_options* opt,
-                         int32_t* idx, float* gate, float* margin, void* stream, int32_t* err) {
+                         int32_t* idx, float* gate, float* margin, void* stream, int32_t* err,
+                         int32_t* lrank = nullptr, int32_t* hist = nullptr,
+                         bool* ranked = nullptr) {
+  if (ranked) *ranked = false;
   int gating;
   float gate_scale;
   if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt) || !read_options(opt, &gating, &gate_scale))
@@ -188,7 +193,9 @@ moe_status route_enqueue(const void* x, const void* Wg, const float* bias, int32
   if (st != MOE_OK) return st;
   RouteArgs a{x, Wg, bias, T, d, E, k, idx, gate, margin, gating, gate_scale};
   a.err = err;
-  return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms) == cudaSuccess
+  a.lrank = lrank;
+  a.hist = hist;
+  return launch_route(a, dt, static_cast<cudaStream_t>(stream), di.num_sms, ranked) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }
@@ -208,11 +215,13 @@ MOE_API moe_status moe_route(const void* x, const void* Wg, const float* bias, i
 }
 
 namespace {
+// `ranked`: pos and the scratch already hold the router's local ranks and
+// per-range counts (the forward), so only the placement and copy run.
 moe_status permute_enqueue(const void* x, const int32_t* idx, const int32_t* order,
                            const int32_t* prior, int32_t T, int32_t d, int32_t E, int32_t k,
                            int32_t capacity, moe_dtype dt, void* xp, int64_t xp_rows,
                            int32_t* pos, int32_t* counts, int32_t* kept_counts, int32_t* offsets,
-                           void* ws, size_t ws_bytes, void* stream, bool ticket_zeroed);
+                           void* ws, size_t ws_bytes, void* stream, bool ranked);
 }  // namespace
 
 MOE_API moe_status moe_permute_ex(const void* x, const int32_t* idx, const int32_t* order,
@@ -230,7 +239,7 @@ moe_status permute_enqueue(const void* x, const int32_t* idx, const int32_t* ord
                            const int32_t* prior, int32_t T, int32_t d, int32_t E, int32_t k,
                            int32_t capacity, moe_dtype dt, void* xp, int64_t xp_rows,
                            int32_t* pos, int32_t* counts, int32_t* kept_counts, int32_t* offsets,
-                           void* ws, size_t ws_bytes, void* stream, bool ticket_zeroed) {
+                           void* ws, size_t ws_bytes, void* stream, bool ranked) {
   if (!valid_route_sizes(T, d, E, k) || !valid_dtype(dt)) return MOE_ERR_ARG;
   if (!counts || !kept_counts || !offsets) return MOE_ERR_ARG;
   if (T > 0) {
@@ -239,20 +248,17 @@ moe_status permute_enqueue(const void* x, const int32_t* idx, const int32_t* ord
       return MOE_ERR_ARG;
     const int64_t need_rows = moe_rows_for_capacity(T, E, k, capacity);
     if (need_rows > INT32_MAX || xp_rows < need_rows) return MOE_ERR_ARG;
-    if (ws_bytes < permute_scratch_bytes(T, E)) return MOE_ERR_ARG;
+    if (ws_bytes < ranked_permute_scratch_bytes(E)) return MOE_ERR_ARG;
   }
   DeviceInfo di;
   moe_status st = device_info(&di);
   if (st != MOE_OK) return st;
-  const size_t nblk = (static_cast<size_t>(T) + kPermBlock - 1) / kPermBlock;
-  int32_t* block_base = static_cast<int32_t*>(ws);
-  unsigned int* ticket = reinterpret_cast<unsigned int*>(
-      static_cast<uint8_t*>(ws) + align_up(nblk * static_cast<size_t>(E) * 4));
-  PermuteArgs a{x,      idx,         T,       d,          E,     k,
-                capacity < 0 ? INT32_MAX : capacity, xp, pos, counts, kept_counts, offsets,
-                block_base, ticket, order, prior, ticket_zeroed};
-  return launch_permute(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK
-                                                                                 : MOE_ERR_CUDA;
+  RankedPermuteArgs a{x, idx, T, d, E, k, capacity < 0 ? INT32_MAX : capacity, xp, pos, counts,
+                      kept_counts, offsets, static_cast<int32_t*>(ws), order, prior, ranked,
+                      di.num_sms};
+  return launch_ranked_permute(a, dt, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 }  // namespace
 
@@ -378,31 +384,30 @@ moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, con
   int32_t* err = reinterpret_cast<int32_t*>(w + L.dev_error);
   if (clear_err && cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  // The permutation's completion counter is zeroed here, ahead of the
-  // router, so no memset separates the kernels of the forward (each may
-  // then start while its predecessor drains).
-  const size_t nblk = (static_cast<size_t>(T) + kPermBlock - 1) / kPermBlock;
-  unsigned int* ticket =
-      reinterpret_cast<unsigned int*>(w + L.scratch + align_up(nblk * static_cast<size_t>(E) * 4));
-  if (cudaMemsetAsync(ticket, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
-  moe_status st = record_stage(0, s);
-  if (st != MOE_OK) return st;
-  st = route_enqueue(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, s, err);
-  if (st == MOE_OK) st = record_stage(1, s);
-  if (st != MOE_OK) return st;
   int gating, priority;
   float gate_scale;
   read_options(opt, &gating, &gate_scale, &priority);
+  const bool by_gate = priority == MOE_PRIORITY_GATE && moe_capacity(T, E, k, cf) >= 0;
+  int32_t* hist = reinterpret_cast<int32_t*>(w + L.scratch);
+  moe_status st = record_stage(0, s);
+  if (st != MOE_OK) return st;
+  // In position order the router also counts (local ranks into pos, the
+  // per-range counts into the scratch), so the permutation is one kernel.
+  bool ranked = false;
+  st = route_enqueue(x, Wg, bias, T, d, E, k, dt, opt, idx, gate, margin, s, err,
+                     by_gate ? nullptr : pos, by_gate ? nullptr : hist, &ranked);
+  if (st == MOE_OK) st = record_stage(1, s);
+  if (st != MOE_OK) return st;
   const int32_t* order = nullptr;
-  if (priority == MOE_PRIORITY_GATE && moe_capacity(T, E, k, cf) >= 0) {
+  if (by_gate) {
     st = moe_priority_order(gate, T, k, reinterpret_cast<int32_t*>(w + L.order),
                             w + L.prio_scratch, priority_scratch_bytes(T), s);
     if (st != MOE_OK) return st;
     order = reinterpret_cast<const int32_t*>(w + L.order);
   }
   st = permute_enqueue(x, idx, order, nullptr, T, d, E, k, moe_capacity(T, E, k, cf), dt, w + L.xp,
-                       L.rows, pos, counts, kept, offsets, w + L.scratch,
-                       permute_scratch_bytes(T, E), s, /*ticket_zeroed=*/true);
+                       L.rows, pos, counts, kept, offsets, hist, ranked_permute_scratch_bytes(E),
+                       s, ranked);
   if (st == MOE_OK) st = record_stage(2, s);
   if (st != MOE_OK) return st;
   st = moe_grouped_ffn(w + L.xp, L.rows, offsets, kept, W1, W3, W2, E, d, H, act, dt, w + L.h,

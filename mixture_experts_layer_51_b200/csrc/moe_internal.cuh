@@ -388,9 +388,30 @@ struct RouteArgs {
   int gating;        // moe_gating
   float gate_scale;  // multiplies every gate
   float* scores = nullptr;  // non-null: write softmax over all E to [E, T] instead of TopK
-  int32_t* err = nullptr;   // device error word for the tensor-core router's bounded waits
+  int32_t* err = nullptr;   // device error word for the routers' bounded waits
+  // Counting half of the permutation, filled by the streaming router only
+  // (launch_route reports whether it did): per (token, slot) the rank among
+  // earlier assignments to the same expert in the token's range [T, k], and
+  // per range the assignments per expert [G, E] (route_ranges).
+  int32_t* lrank = nullptr;
+  int32_t* hist = nullptr;
 };
-cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms);
+// `ranked` (nullable) is set to whether lrank/hist were written.
+cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms,
+                         bool* ranked = nullptr);
+
+// Token ranges shared by the streaming router and the permutation: G ranges
+// of whole 8-token groups, range c = [c*T8/G*8, min(T, (c+1)*T8/G*8)), so
+// ranges differ by at most 8 tokens; MT = rows per router tile (<= 128).
+constexpr int kMaxRouteRanges = 256;
+struct RouteRanges {
+  int G, T8, MT;
+};
+RouteRanges route_ranges(int T, int num_sms);
+// Streaming router (route_stream.cu): bf16, E % 8 == 0.  MOE_ROUTE_STREAM=0
+// turns it off, for measurements.
+bool route_stream_supported(const RouteArgs& a);
+cudaError_t launch_route_stream(const RouteArgs& a, int num_sms, cudaStream_t s);
 // Tensor-core router (route_tc.cu): bf16, E % 8 == 0.  MOE_ROUTE_TC=0 turns
 // it off, for measurements.
 bool route_tc_supported(const RouteArgs& a);
@@ -445,6 +466,29 @@ struct PermuteArgs {
   const int32_t* prior = nullptr;  // per-expert assignments of earlier shards, or null
   bool ticket_zeroed = false;      // the caller already zeroed *ticket on this stream
 };
+// Permutation in two kernels over the route_ranges of T: local ranks and
+// per-range counts (skipped when the router already wrote them into pos and
+// hist), then positions -- prefix over the ranges, capacity, 128-row aligned
+// offsets -- and the row copy.  pos holds the local ranks in between.
+struct RankedPermuteArgs {
+  const void* x;
+  const int32_t* idx;
+  int T, d, E, k;
+  int capacity;                    // INT32_MAX when dropless
+  void* xp;
+  int32_t* pos;
+  int32_t* counts;
+  int32_t* kept_counts;
+  int32_t* offsets;
+  int32_t* hist;                   // [kMaxRouteRanges * E] scratch
+  const int32_t* order = nullptr;  // queue order (token at position i), or null
+  const int32_t* prior = nullptr;  // per-expert assignments of earlier shards, or null
+  bool ranked = false;             // pos / hist already hold the local ranks and counts
+  int num_sms = 148;
+};
+size_t ranked_permute_scratch_bytes(int E);
+cudaError_t launch_ranked_permute(const RankedPermuteArgs& a, moe_dtype dtype, cudaStream_t s);
+
 cudaError_t launch_expert_counts(const int32_t* idx, int T, int E, int k, int32_t* counts,
                                  cudaStream_t s);
 cudaError_t launch_rank_prefix(const int32_t* gathered, int n_ranks, int E, int rank,

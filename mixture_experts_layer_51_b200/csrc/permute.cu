@@ -308,6 +308,228 @@ cudaError_t launch_row_copy(const void* x, const int32_t* pos, int T, int npos, 
                        npos, dvec, static_cast<uint4*>(xp));
 }
 
+// ------------------------------------------------------------------------
+// The permutation over the router's token ranges (route_ranges).  Ranks are
+// counted once per range -- by the streaming router as it selects, or by
+// ranked_local_kernel -- and ranked_place_copy_kernel turns a (token, slot)
+// with expert e and local rank lr into row offsets[e] + base_c[e] + lr, where
+// base_c[e] sums the counts of the ranges before c; it is kept when that
+// queue place is below the expert's capacity.  Every CTA of the second
+// kernel recomputes the prefix it needs from the [G, E] count table (a few
+// KB, read from L2), so no counter, ticket or second launch orders them, and
+// nothing decided by atomics: the placement is deterministic.
+namespace {
+
+constexpr int kRankThreads = 256;
+constexpr int kRankWarps = kRankThreads / 32;
+constexpr int kPlaceWarps = 8;
+
+__device__ __forceinline__ void range_of(int c, int G, int T8, int T, int& r0, int& r1) {
+  r0 = static_cast<int>(static_cast<int64_t>(c) * T8 / G) * 8;
+  r1 = min(T, static_cast<int>(static_cast<int64_t>(c + 1) * T8 / G) * 8);
+}
+
+// One CTA per range: queue positions [r0, r1) (position i serves token
+// order[i], or i), 256 at a time, one thread each.  Writes lrank[t, j] (the
+// rank among the range's earlier assignments to the same expert; -1 for an
+// expert id outside [0, E)) and hist[c, e].
+__global__ void __launch_bounds__(kRankThreads)
+    ranked_local_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ order,
+                        int T, int E, int k, int G, int T8, int32_t* __restrict__ lrank,
+                        int32_t* __restrict__ hist) {
+  __shared__ int cnt[kMaxE];
+  __shared__ int wcnt[kRankWarps][kMaxE];
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x;
+  int r0, r1;
+  range_of(c, G, T8, T, r0, r1);
+  if (tid < E) cnt[tid] = 0;
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = r0; base < r1; base += kRankThreads) {
+    const int i = base + tid;
+    const int t = i < r1 ? (order ? order[i] : i) : -1;
+    int ej[kMaxK], rj[kMaxK];
+    uint64_t mask = 0;
+    for (int j = 0; j < k; ++j) {
+      ej[j] = t >= 0 ? idx[(int64_t)t * k + j] : -1;
+      rj[j] = -1;
+      if (ej[j] >= 0 && ej[j] < E) mask |= 1ull << ej[j];
+    }
+    for (int e = 0; e < E; ++e) {
+      const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
+      if (lane == 0) wcnt[warp][e] = __popc(b);
+      if ((mask >> e) & 1ull) {
+        const int r = __popc(b & lt);
+        for (int j = 0; j < k; ++j)
+          if (ej[j] == e) rj[j] = r;
+      }
+    }
+    __syncthreads();
+    if (t >= 0) {
+      for (int j = 0; j < k; ++j) {
+        int r = -1;
+        if (rj[j] >= 0) {
+          const int e = ej[j];
+          r = cnt[e] + rj[j];
+          for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+        }
+        lrank[(int64_t)t * k + j] = r;
+      }
+    }
+    __syncthreads();
+    if (tid < E) {
+      int sum = 0;
+#pragma unroll
+      for (int w = 0; w < kRankWarps; ++w) sum += wcnt[w][tid];
+      cnt[tid] += sum;
+    }
+    __syncthreads();
+  }
+  if (tid < E) hist[(int64_t)c * E + tid] = cnt[tid];
+}
+
+// S CTAs per range.  Prologue: the prefix of the count table over the ranges
+// before this one, the totals, the capacities (C, or C - prior[e] for a
+// shard of a batch), kept counts and 128-row aligned offsets; CTA 0 writes
+// counts, kept_counts and offsets.  Then one warp per queue position of
+// this CTA's share of the range: pos[t, j] (in: local rank, out: row or -1)
+// and the copy of x[t] to every kept row (16-byte vectors, eight in flight
+// per lane), reading the row once.
+__global__ void __launch_bounds__(kPlaceWarps * 32)
+    ranked_place_copy_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
+                             const int32_t* __restrict__ order, int T, int E, int k, int G, int T8,
+                             int S, int C, const int32_t* __restrict__ prior,
+                             const int32_t* __restrict__ hist, int32_t* __restrict__ pos,
+                             int dvec, uint4* __restrict__ xp, int32_t* __restrict__ counts,
+                             int32_t* __restrict__ kept_counts, int32_t* __restrict__ offsets) {
+  __shared__ int red_b[kPlaceWarps * 32], red_t[kPlaceWarps * 32];
+  __shared__ int s_base[kMaxE], s_cap[kMaxE], s_off[kMaxE + 1], s_kept[kMaxE];
+  __shared__ int dst[kPlaceWarps][kMaxK];
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x / S, sub = blockIdx.x - c * S;
+  {
+    // Thread (part, e) sums ranges part, part + parts, ... of column e.
+    const int parts = (kPlaceWarps * 32) / E;
+    const int e = tid % E, part = tid / E;
+    int sb = 0, st = 0;
+    if (part < parts) {
+      for (int q = part; q < G; q += parts) {
+        const int v = hist[(int64_t)q * E + e];
+        st += v;
+        sb += q < c ? v : 0;
+      }
+    }
+    red_b[tid] = sb;
+    red_t[tid] = st;
+    __syncthreads();
+    if (tid < E) {
+      int b = 0, tot = 0;
+      for (int q = 0; q < parts; ++q) {
+        b += red_b[q * E + tid];
+        tot += red_t[q * E + tid];
+      }
+      int cap = C;
+      if (prior && C != INT32_MAX) cap = max(0, C - prior[tid]);
+      s_base[tid] = b;
+      s_cap[tid] = cap;
+      s_kept[tid] = tot < cap ? tot : cap;
+      if (blockIdx.x == 0) {
+        counts[tid] = tot;
+        kept_counts[tid] = s_kept[tid];
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int off = 0;
+      for (int q = 0; q < E; ++q) {
+        s_off[q] = off;
+        off += (s_kept[q] + kRowAlign - 1) / kRowAlign * kRowAlign;
+      }
+      s_off[E] = off;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0 && tid <= E) offsets[tid] = s_off[tid];
+  }
+  int r0, r1;
+  range_of(c, G, T8, T, r0, r1);
+  const int len = r1 - r0;
+  const int q0 = r0 + static_cast<int>(static_cast<int64_t>(sub) * len / S);
+  const int q1 = r0 + static_cast<int>(static_cast<int64_t>(sub + 1) * len / S);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i = q0 + warp; i < q1; i += kPlaceWarps) {
+    const int t = order ? order[i] : i;
+    int p = -1;
+    if (lane < k) {
+      const int e = idx[(int64_t)t * k + lane];
+      const int lr = pos[(int64_t)t * k + lane];
+      if (e >= 0 && e < E && lr >= 0) {
+        // Kept when the queue place is below the capacity; comparing with
+        // the kept count min(count, capacity) also bounds the row by
+        // offsets[E] whatever the local ranks hold.
+        const int r = s_base[e] + lr;
+        if (r < s_kept[e]) p = s_off[e] + r;
+      }
+      pos[(int64_t)t * k + lane] = p;
+    }
+    const unsigned b = __ballot_sync(0xffffffffu, p >= 0);
+    if (p >= 0) dst[warp][__popc(b & lt)] = p;
+    const int nd = __popc(b);
+    __syncwarp();
+    if (nd > 0) {
+      const uint4* src = x + (int64_t)t * dvec;
+      for (int v0 = lane; v0 < dvec; v0 += 32 * 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (v0 + u * 32 < dvec) v[u] = __ldcs(src + v0 + u * 32);
+        for (int j = 0; j < nd; ++j) {
+          uint4* out = xp + (int64_t)dst[warp][j] * dvec;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (v0 + u * 32 < dvec) out[v0 + u * 32] = v[u];
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+size_t ranked_permute_scratch_bytes(int E) {
+  return static_cast<size_t>(kMaxRouteRanges) * static_cast<size_t>(E) * sizeof(int32_t);
+}
+
+cudaError_t launch_ranked_permute(const RankedPermuteArgs& a, moe_dtype dtype, cudaStream_t s) {
+  if (a.T == 0) {
+    cudaError_t err = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(a.kept_counts, 0, sizeof(int32_t) * a.E, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1), s);
+    return err;
+  }
+  const RouteRanges rg = route_ranges(a.T, a.num_sms);
+  cudaError_t err = cudaSuccess;
+  if (!a.ranked) {
+    err = launch_kernel(ranked_local_kernel, dim3(rg.G), dim3(kRankThreads), 0, s, 1, true, a.idx,
+                        a.order, a.T, a.E, a.k, rg.G, rg.T8, a.pos, a.hist);
+    if (err != cudaSuccess) return err;
+  }
+  // About four CTAs per SM over all ranges, each range's share at least a
+  // few tokens.
+  const int per_range = (rg.T8 * 8 + rg.G - 1) / rg.G;
+  const int S = std::max(1, std::min({8, (4 * a.num_sms + rg.G - 1) / rg.G, per_range / 4}));
+  const int dvec = a.d * (dtype == MOE_BF16 ? 2 : 4) / 16;
+  return launch_kernel(ranked_place_copy_kernel, dim3(rg.G * S), dim3(kPlaceWarps * 32), 0, s, 1,
+                       true, static_cast<const uint4*>(a.x), a.idx, a.order, a.T, a.E, a.k, rg.G,
+                       rg.T8, S, a.capacity, a.prior, static_cast<const int32_t*>(a.hist), a.pos,
+                       dvec, static_cast<uint4*>(a.xp), a.counts, a.kept_counts, a.offsets);
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* v = getenv("MOE_PDL");

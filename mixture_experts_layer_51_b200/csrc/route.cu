@@ -21,6 +21,7 @@
 #include <stdlib.h>
 
 #include "moe_internal.cuh"
+#include "route_select.cuh"
 
 namespace moe {
 namespace {
@@ -96,24 +97,6 @@ __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t,
     for (int j = 1; j < KM; ++j)
       if (j == k && k < E) mg = tv[j - 1] - tv[j];
     margin[t] = mg;
-  }
-}
-
-// Inserts (v, ei) into a list sorted by descending value (ei < 0: nothing
-// to insert).  An unfilled slot (index < 0) always takes the value, so -inf
-// logits are still ranked in expert order; a strict comparison leaves an
-// equal earlier (lower-index) entry in front.
-template <int KM>
-__device__ __forceinline__ void insert_sorted(float (&tv)[KM], int (&ti)[KM], float v, int ei) {
-#pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    const bool take = ei >= 0 && (v > tv[j] || ti[j] < 0);
-    const float tvj = tv[j];
-    const int tij = ti[j];
-    tv[j] = take ? v : tvj;
-    ti[j] = take ? ei : tij;
-    v = take ? tvj : v;
-    ei = take ? tij : ei;
   }
 }
 
@@ -315,17 +298,9 @@ __global__ void __launch_bounds__(kRouteThreads)
   const int t = t0 + static_cast<int>(q) * TPC + rr;
   const float* lrow = fin + rr * LS;
   if (scores) {
-    // Expert-choice affinities: softmax over all E logits.  The P threads
-    // of a token combine their maxima and sums with a fixed butterfly.
-    float m = -INFINITY;
-    for (int e = p; e < E; e += P) m = fmaxf(m, lrow[e]);
-#pragma unroll
-    for (int o = P / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.f;
-    for (int e = p; e < E; e += P) sum += expf(lrow[e] - m);
-#pragma unroll
-    for (int o = P / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = 1.f / sum;
+    // Expert-choice affinities: softmax over all E logits.
+    float m, inv;
+    softmax_stats(lrow, E, P, p, m, inv);
     // Expert-major output scores[e, t]: the tile is written with consecutive
     // threads on consecutive tokens, each value recomputed from the same
     // logit, maximum and reciprocal as the sum used.
@@ -344,76 +319,7 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
     return;
   }
-  // This thread's experts [e_lo, e_hi), then the butterfly merge.
-  float tv[KM];
-  int ti[KM];
-#pragma unroll
-  for (int j = 0; j < KM; ++j) {
-    tv[j] = -INFINITY;
-    ti[j] = -1;
-  }
-  {
-    const int per = (E + P - 1) / P;
-    const int e_lo = min(E, p * per), e_hi = min(E, e_lo + per);
-    for (int e = e_lo; e < e_hi; ++e) insert_sorted<KM>(tv, ti, lrow[e], e);
-  }
-#pragma unroll
-  for (int o = 1; o < P; o <<= 1) {
-    float pv[KM];
-    int pi[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      pv[j] = __shfl_xor_sync(0xffffffffu, tv[j], o);
-      pi[j] = __shfl_xor_sync(0xffffffffu, ti[j], o);
-    }
-    if (p & o) {
-      // The partner holds the lower experts: its list goes first.
-#pragma unroll
-      for (int j = 0; j < KM; ++j) {
-        const float v = tv[j];
-        const int ei = ti[j];
-        tv[j] = pv[j];
-        ti[j] = pi[j];
-        pv[j] = v;
-        pi[j] = ei;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < KM; ++j) insert_sorted<KM>(tv, ti, pv[j], pi[j]);
-  }
-  const float m = tv[0];  // the largest logit
-  float denom = 0.f;
-  if (gating == MOE_GATE_SOFTMAX_TOPK) {
-    // Switch order: the softmax denominator over all E logits.
-    for (int e = p; e < E; e += P) denom += expf(lrow[e] - m);
-#pragma unroll
-    for (int o = P / 2; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
-  } else {
-#pragma unroll
-    for (int j = 0; j < KM; ++j)
-      if (j < k) denom += expf(tv[j] - m);
-  }
-  if (t < T) {
-    const float inv = gate_scale / denom;
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-      if (j < k && j % P == p) {
-        idx[(int64_t)t * k + j] = ti[j];
-        gate[(int64_t)t * k + j] = expf(tv[j] - m) * inv;
-      }
-    }
-    if (margin) {
-      // slot k-1 minus slot k (every gap computed, one kept: no dynamic
-      // index into the list)
-      float mg = INFINITY;
-#pragma unroll
-      for (int j = 1; j < KM; ++j) {
-        const float gap = tv[j - 1] - tv[j];
-        mg = (j == k && k < E) ? gap : mg;
-      }
-      if (p == 0) margin[t] = mg;
-    }
-  }
+  select_token<KM>(lrow, E, k, P, p, t, t < T, gating, gate_scale, idx, gate, margin, nullptr);
 }
 
 // fp32 router: one warp per token; 8 experts at a time, each lane strides d,
@@ -533,7 +439,9 @@ cudaError_t launch_route_bf16(const RouteArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int /*num_sms*/) {
+cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, int num_sms,
+                         bool* ranked) {
+  if (ranked) *ranked = false;
   if (a.T == 0) return cudaSuccess;
   if (dtype == MOE_FP32) {
     route_fp32_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(static_cast<const float*>(a.x),
@@ -541,6 +449,13 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
                                                     a.d, a.E, a.k, a.idx, a.gate, a.margin,
                                                     a.gating, a.gate_scale, a.scores);
     return cudaGetLastError();
+  }
+  if (route_stream_supported(a)) {
+    const cudaError_t err = launch_route_stream(a, num_sms, s);
+    if (err != cudaErrorInvalidValue) {
+      if (ranked) *ranked = err == cudaSuccess && a.lrank && a.hist;
+      return err;  // else: no tensor map, fall through
+    }
   }
   if (route_tc_supported(a)) {
     const cudaError_t err = launch_route_tc(a, s);

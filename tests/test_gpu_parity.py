@@ -53,6 +53,9 @@ def test_full_switch_tiny_fp32():
     dict(T=400, d=192, E=3, k=1, H=72, act="gelu"),  # bf16 GELU, odd sizes
     dict(T=2000, d=128, E=16, k=2, H=256, cf=0.25),  # heavy dropping
     dict(T=513, d=64, E=64, k=8, H=64),          # many tiny experts
+    dict(T=1703, d=320, E=24, k=3, H=128),       # W_g box wider than E (24 of 32), d % 256 != 0
+    dict(T=9999, d=200, E=40, k=5, H=96),        # router tiles of 72 rows, ragged last range
+    dict(T=21011, d=128, E=16, k=2, H=64, cf=1.0),  # two router tiles per range
 ])
 def test_edge_shapes(case):
     act = case.pop("act", "swiglu")

@@ -1,6 +1,8 @@
-"""The tensor-core router (route_tc.cu) forced on where the heuristic would
-not pick it: small batches, ragged sizes, both gate orders, expert choice.
-MOE_ROUTE_TC is read once per process, so each check runs in a child."""
+"""The routers other than the default streaming one, forced on: the
+tensor-core router (route_tc.cu) and the clustered mma.sync router
+(route.cu), on small batches, ragged sizes, both gate orders and expert
+choice.  The choice (MOE_ROUTE_STREAM, MOE_ROUTE_TC) is read once per
+process, so each check runs in a child."""
 
 import os
 import subprocess
@@ -14,10 +16,14 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_tensor_core_router_forced_on_small_batches():
-    """The tensor-core router is chosen for large batches only; forcing it
-    (MOE_ROUTE_TC=1, read once per process, so in a child process) on the
-    small parity layers and a ragged batch must still match the oracle."""
+ALTERNATES = {"tensor_core": {"MOE_ROUTE_STREAM": "0", "MOE_ROUTE_TC": "1"},
+              "mma_sync_clusters": {"MOE_ROUTE_STREAM": "0", "MOE_ROUTE_TC": "0"}}
+
+
+@pytest.mark.parametrize("router", list(ALTERNATES))
+def test_alternate_router_forced_on_small_batches(router):
+    """An alternate router forced on the small parity layers and a ragged
+    batch must still match the oracle."""
     script = textwrap.dedent("""
         import sys
         sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
@@ -36,14 +42,15 @@ def test_tensor_core_router_forced_on_small_batches():
             full_parity(w, make_inputs(w, "cpu"), gating="softmax_topk", gate_scale=2.0)
         print("TC_ROUTER_OK")
     """).format(root=ROOT, tests=os.path.join(ROOT, "tests"))
-    env = dict(os.environ, MOE_ROUTE_TC="1")
+    env = dict(os.environ, **ALTERNATES[router])
     r = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0, r.stderr[-3000:]
     assert "TC_ROUTER_OK" in r.stdout
 
 
-def test_tensor_core_router_expert_choice_forced():
+@pytest.mark.parametrize("router", list(ALTERNATES))
+def test_alternate_router_expert_choice_forced(router):
     script = textwrap.dedent("""
         import sys
         sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
@@ -54,7 +61,7 @@ def test_tensor_core_router_expert_choice_forced():
             T._check(w, T.make_inputs(w, "cpu"))
         print("TC_EC_OK")
     """).format(root=ROOT, tests=os.path.join(ROOT, "tests"))
-    env = dict(os.environ, MOE_ROUTE_TC="1")
+    env = dict(os.environ, **ALTERNATES[router])
     r = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0, r.stderr[-3000:]
