@@ -39,8 +39,10 @@ __host__ __device__ constexpr int stage_bytes(int NT, int BM, int BK) {
 // TopK over one token's E logits (descending; equal logits keep the lower
 // expert first), then softmax over the k selected ones.  `get(e)` returns
 // the logit of expert e.  The running top-(k+1) list lives in registers:
-// each new logit bubbles down a fixed compare-and-swap chain, and a strict
-// comparison leaves an equal earlier (lower-index) entry in front.
+// each new logit bubbles down a fixed compare-and-swap chain; an entry moves
+// in front of another when its logit is larger, or equal with a lower
+// expert, so an entry pushed down keeps its place before an equal logit of
+// a higher expert.
 template <int KM, typename Get>
 __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t, int32_t* idx,
                                                    float* gate, float* margin, int gating,
@@ -59,7 +61,7 @@ __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t,
     for (int j = 0; j < KM; ++j) {
       // An unfilled slot (ti < 0) always takes the value, so -inf logits
       // are still ranked in expert order.
-      if (v > tv[j] || ti[j] < 0) {
+      if (ti[j] < 0 || v > tv[j] || (v == tv[j] && ei < ti[j])) {
         const float tvj = tv[j];
         const int tij = ti[j];
         tv[j] = v;

@@ -10,9 +10,9 @@
 // P threads cooperate on one token (P a power of two, the P lanes adjacent
 // in one warp).  Each keeps the sorted top-(k+1) list of a contiguous range
 // of experts (a compare-and-swap chain), then the lists are merged in a
-// butterfly in which the higher-index half's entries go into the lower half's
-// list, so equal logits keep the lower expert first -- the stable descending
-// order -- and every thread ends with the same list.
+// butterfly in which the lower half's list goes first, so equal logits keep
+// the lower expert first -- the stable descending order -- and every thread
+// ends with the same list.
 #pragma once
 
 #include <math.h>
@@ -21,21 +21,57 @@
 
 namespace moe {
 
-// Inserts (v, ei) into a list sorted by descending value (ei < 0: nothing
-// to insert).  An unfilled slot (index < 0) always takes the value, so -inf
-// logits are still ranked in expert order; a strict comparison leaves an
-// equal earlier (lower-index) entry in front.
+// (v, ei) goes before (w, ej): a larger value, or an equal value and a lower
+// expert -- the stable descending order.
+__device__ __forceinline__ bool ranks_before(float v, int ei, float w, int ej) {
+  return v > w || (v == w && ei < ej);
+}
+
+// Inserts (v, ei) into a list sorted in that order (ei < 0: nothing to
+// insert).  An unfilled slot (index < 0) always takes the entry, so -inf
+// logits are still ranked in expert order.  An entry pushed down the list
+// is compared by value and expert, so it stays in front of an equal logit
+// of a higher expert.
 template <int KM>
 __device__ __forceinline__ void insert_sorted(float (&tv)[KM], int (&ti)[KM], float v, int ei) {
 #pragma unroll
   for (int j = 0; j < KM; ++j) {
-    const bool take = ei >= 0 && (v > tv[j] || ti[j] < 0);
+    const bool take = ei >= 0 && (ti[j] < 0 || ranks_before(v, ei, tv[j], ti[j]));
     const float tvj = tv[j];
     const int tij = ti[j];
     tv[j] = take ? v : tvj;
     ti[j] = take ? ei : tij;
     v = take ? tvj : v;
     ei = take ? tij : ei;
+  }
+}
+
+// Merges two lists sorted as insert_sorted keeps them into the first: the
+// KM leading entries of their union, in the same order; a real entry goes
+// before an unfilled one.  Each step takes the larger head and shifts
+// that list by one -- only the entries that may still be taken move.
+template <int KM>
+__device__ __forceinline__ void merge_sorted(float (&av)[KM], int (&ai)[KM], float (&bv)[KM],
+                                             int (&bi)[KM]) {
+  float ov[KM];
+  int oi[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    const bool ta = ai[0] >= 0 && (bi[0] < 0 || ranks_before(av[0], ai[0], bv[0], bi[0]));
+    ov[j] = ta ? av[0] : bv[0];
+    oi[j] = ta ? ai[0] : bi[0];
+#pragma unroll
+    for (int i = 0; i + 1 < KM - j; ++i) {
+      av[i] = ta ? av[i + 1] : av[i];
+      ai[i] = ta ? ai[i + 1] : ai[i];
+      bv[i] = ta ? bv[i] : bv[i + 1];
+      bi[i] = ta ? bi[i] : bi[i + 1];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    av[j] = ov[j];
+    ai[j] = oi[j];
   }
 }
 
@@ -83,8 +119,7 @@ __device__ __forceinline__ void select_token(const float* lrow, int E, int k, in
         pi[j] = ei;
       }
     }
-#pragma unroll
-    for (int j = 0; j < KM; ++j) insert_sorted<KM>(tv, ti, pv[j], pi[j]);
+    merge_sorted<KM>(tv, ti, pv, pi);
   }
   const float m = tv[0];  // the largest logit
   float denom = 0.f;

@@ -76,6 +76,35 @@ def test_all_tokens_on_one_expert_with_capacity():
     assert (g["pos"][:C, 0] >= 0).all() and (g["pos"][C:, 0] == -1).all()
 
 
+@pytest.mark.parametrize("E,k,dtype", [(8, 3, "bf16"), (16, 5, "bf16"), (32, 5, "bf16"),
+                                       (64, 7, "bf16"), (6, 3, "bf16"), (4, 1, "fp32")])
+def test_exact_logit_ties_keep_the_lower_expert(E, k, dtype):
+    """Router columns duplicated in pairs: every token's logits come in
+    exactly equal pairs (the same products summed in the same order), so with
+    odd k the TopK boundary splits a pair for many tokens.  The pages' order
+    is a stable descending sort (equal logits: lower expert first), so every
+    token's experts, in slot order, must equal the oracle's -- ties are not
+    excluded here.  Covers each router back end (E 8 and 16: mma.sync with a
+    K-split; 32 and 64: tcgen05; 6: the clustered mma.sync router; fp32)."""
+    w = Workload("ties", T=1000, d=256, E=E, k=k, H=64, act="swiglu", dtype=dtype, cf=0.0,
+                 seed=41)
+    inp = make_inputs(w, "cpu")
+    Wg = inp["Wg"].clone()
+    Wg[:, 1::2] = Wg[:, 0::2]
+    inp["Wg"] = Wg
+    g = run_gpu(w, inp)
+    logits = oracle.router_logits(inp["x"], Wg, inp["bias"])
+    idx_o, _, margin = oracle.top_k(logits, k)
+    assert (margin == 0).sum() > w.T // 4, "the boundary should split a pair often"
+    assert np.array_equal(g["idx"], idx_o)
+    assert np.array_equal(g["margin"][margin == 0], margin[margin == 0])
+    kept, _ = check_permutation(g, to_np(inp["x"].float()), w.T, w.E, w.k, w.cf,
+                                g["views"]["xp"])
+    y_tf, _ = oracle.moe_forward_tokens(inp["x"], logits, g["idx"], kept, inp["W1"], inp["W3"],
+                                        inp["W2"], w.act)
+    assert_y_close(g["y"], y_tf, w.dtype)
+
+
 def test_upcycling_identity_on_gpu():
     """Identical experts: the layer equals the dense FFN (within bf16)."""
     w = Workload("upcycle", T=300, d=128, E=8, k=2, H=256, act="swiglu", dtype="bf16", cf=0.0,
