@@ -351,32 +351,35 @@ __global__ void __launch_bounds__(kRankThreads)
   for (int base = r0; base < r1; base += kRankThreads) {
     const int i = base + tid;
     const int t = i < r1 ? (order ? order[i] : i) : -1;
+    // Slot arrays indexed only by unrolled loops up to kMaxK (registers).
     int ej[kMaxK], rj[kMaxK];
     uint64_t mask = 0;
-    for (int j = 0; j < k; ++j) {
-      ej[j] = t >= 0 ? idx[(int64_t)t * k + j] : -1;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      ej[j] = (t >= 0 && j < k) ? idx[(int64_t)t * k + j] : -1;
       rj[j] = -1;
       if (ej[j] >= 0 && ej[j] < E) mask |= 1ull << ej[j];
     }
     for (int e = 0; e < E; ++e) {
       const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
       if (lane == 0) wcnt[warp][e] = __popc(b);
-      if ((mask >> e) & 1ull) {
-        const int r = __popc(b & lt);
-        for (int j = 0; j < k; ++j)
-          if (ej[j] == e) rj[j] = r;
-      }
+      const int r = __popc(b & lt);
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) rj[j] = ((mask >> e) & 1ull) && ej[j] == e ? r : rj[j];
     }
     __syncthreads();
     if (t >= 0) {
-      for (int j = 0; j < k; ++j) {
-        int r = -1;
-        if (rj[j] >= 0) {
-          const int e = ej[j];
-          r = cnt[e] + rj[j];
-          for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (j < k) {
+          int r = -1;
+          if (rj[j] >= 0) {
+            const int e = ej[j];
+            r = cnt[e] + rj[j];
+            for (int w = 0; w < warp; ++w) r += wcnt[w][e];
+          }
+          lrank[(int64_t)t * k + j] = r;
         }
-        lrank[(int64_t)t * k + j] = r;
       }
     }
     __syncthreads();

@@ -60,8 +60,10 @@ __device__ __forceinline__ void merge_sorted(float (&av)[KM], int (&ai)[KM], flo
     const bool ta = ai[0] >= 0 && (bi[0] < 0 || ranks_before(av[0], ai[0], bv[0], bi[0]));
     ov[j] = ta ? av[0] : bv[0];
     oi[j] = ta ? ai[0] : bi[0];
+    // Fixed bounds, so the lists stay in registers; the entries past
+    // KM - 1 - j are never taken again, so shifting them as well is harmless.
 #pragma unroll
-    for (int i = 0; i + 1 < KM - j; ++i) {
+    for (int i = 0; i + 1 < KM; ++i) {
       av[i] = ta ? av[i + 1] : av[i];
       ai[i] = ta ? ai[i + 1] : ai[i];
       bv[i] = ta ? bv[i] : bv[i + 1];

@@ -233,32 +233,38 @@ __device__ __forceinline__ void rs_tile_epilogue(const RsParams& p, RsCtl& c,
   // order: one thread per token of the tile (warps 0-3), a ballot per
   // expert; the warps below come from shared counts, earlier tiles from the
   // running per-expert count.
+  // (The slot loops run to the compile-time bound KM - 1 >= k, so the slot
+  // arrays stay in registers.)
+  constexpr int KS = KM - 1;
   uint64_t mask = 0;
-  int ej[kMaxK], rj[kMaxK];
+  int ej[KS], rj[KS];
   const bool have = !aborted && warp < 4 && tid < rows;
   if (warp < 4) {
-    for (int j = 0; j < p.k; ++j) {
-      ej[j] = have ? c.idx_s[tid][j] : -1;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+      ej[j] = (have && j < p.k) ? c.idx_s[tid][j] : -1;
       rj[j] = 0;
-      if (have) mask |= 1ull << ej[j];
+      if (ej[j] >= 0) mask |= 1ull << ej[j];
     }
     const unsigned lt = (1u << lane) - 1u;
     for (int e = 0; e < p.E; ++e) {
       const unsigned b = __ballot_sync(0xffffffffu, (mask >> e) & 1ull);
       if (lane == 0) c.wcnt[warp][e] = __popc(b);
-      if ((mask >> e) & 1ull) {
-        for (int j = 0; j < p.k; ++j)
-          if (ej[j] == e) rj[j] = __popc(b & lt);
-      }
+      const int r = __popc(b & lt);
+#pragma unroll
+      for (int j = 0; j < KS; ++j) rj[j] = ej[j] == e ? r : rj[j];
     }
   }
   consumer_sync();
   if (have) {
-    for (int j = 0; j < p.k; ++j) {
-      const int e = ej[j];
-      int r = c.cnt[e] + rj[j];
-      for (int w = 0; w < warp; ++w) r += c.wcnt[w][e];
-      p.lrank[static_cast<int64_t>(row0 + tid) * p.k + j] = r;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+      if (j < p.k) {
+        const int e = ej[j];
+        int r = c.cnt[e] + rj[j];
+        for (int w = 0; w < warp; ++w) r += c.wcnt[w][e];
+        p.lrank[static_cast<int64_t>(row0 + tid) * p.k + j] = r;
+      }
     }
   }
   consumer_sync();
@@ -604,13 +610,19 @@ cudaError_t launch_rs(const RouteArgs& a, int num_sms, cudaStream_t s) {
   const RouteRanges rg = route_ranges(a.T, num_sms);
   const bool tc = a.E > 16;
   const int EP = tc ? kRsTcN : (a.E <= 8 ? 8 : 16);
-  // tcgen05 with a long selection (k > 2): two tiles per range (boxes of at
-  // least 32 rows), so the selection of the first overlaps the streaming of
-  // the second.  Smaller tiles would not pay: the W_g rows of a stage, 64
-  // experts wide, take shared memory from the x ring.  Otherwise (and for
-  // mma.sync, whose warps both contract and select) the fewest tiles.
+  // The fewest tiles per range.  (Two tiles on the tcgen05 path would let
+  // the selection of the first overlap the streaming of the second, but each
+  // tile streams all of W_g -- 64 experts wide, as large as half the range's
+  // x at E = 64 -- through the same ring: measured slower, 39 vs 34 us on
+  // the 16384 x 2048, E = 64, top-8 router.)  MOE_RS_TC_SPLIT=1 forces two
+  // tiles, for measurements.
+  static const int force_split = [] {
+    const char* v = getenv("MOE_RS_TC_SPLIT");
+    return v ? (v[0] == '0' ? 0 : 1) : -1;
+  }();
   const int rmax = 8 * ((rg.T8 + rg.G - 1) / rg.G);
-  const int mt_tc = a.k > 2 && !a.scores
+  const bool split = force_split == 1;
+  const int mt_tc = split
                         ? std::min(kRsMaxRows, std::max(std::min(rmax, 32), 8 * ((rmax + 15) / 16)))
                         : rg.MT;
   RsParams p{};
