@@ -119,6 +119,10 @@ struct TcParams {
   const int32_t* kept;
   int32_t* err;
   int debug_stall;  // 1: the MMA issuer first waits on a barrier nobody arms (tests only)
+  // 1: (CTA pairs, four epilogue warps) an expert's last block with at most
+  // TM kept rows runs as an M = 128 pair tile -- 64 rows in each CTA -- so
+  // its second half of padding rows is not computed.
+  int half_tiles;
 };
 
 struct Control {
@@ -148,6 +152,17 @@ __device__ __forceinline__ void decode_tile(const Control& c, int t, int& e, int
   const int mt = c.sched_mt[s];
   n = local / mt;
   m = local - n * mt;
+}
+
+// Whether the block of `m_row` (rows inside expert e's block) runs as an
+// M = 128 pair tile: it is the expert's last and holds at most TM kept rows.
+// Its accumulator then sits in TMEM lanes 0-63 (the CTA's 64 rows, tile
+// columns 0..127) and lanes 64-127 (the same rows, columns 128..255), at
+// TMEM columns 0..127.
+template <int CG>
+__device__ __forceinline__ bool is_half_tile(const TcParams& p, const Control& c, int e,
+                                             int m_row) {
+  return CG == 2 && EPI_WARPS == 4 && p.half_tiles && c.kept[e] - m_row <= TM;
 }
 
 #ifndef MOE_FAST_SILU
@@ -296,11 +311,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         int e, m, n;
         decode_tile(c, t, e, m, n);
-        const int row0 = c.off[e] + m * TILE_M + static_cast<int>(rank) * TM;
+        const bool half_m = is_half_tile<CG>(p, c, e, m * TILE_M);
+        const int row0 =
+            c.off[e] + m * TILE_M + static_cast<int>(rank) * (half_m ? TM / 2 : TM);
         // First 64-column chunk of this CTA's B columns (4-D weight maps).
-        const int c0 = CG == 2 ? (EPI == EPI_SWIGLU ? n * 2 : n * 4 + 2 * static_cast<int>(rank))
+        // SwiGLU pairs: each CTA holds one 64-column chunk of W1 next to the
+        // same chunk of W3 (leader: the tile's first chunk, peer: its
+        // second), so in either tile height every thread's accumulator row
+        // holds the gate and the up value of the same h columns.
+        const int c0 = CG == 2 ? (EPI == EPI_SWIGLU ? n * 2 + static_cast<int>(rank)
+                                                    : n * 4 + 2 * static_cast<int>(rank))
                                : (EPI == EPI_SWIGLU ? n * 2 : n * 4);
-        const CUtensorMap* mb = (CG == 2 && EPI == EPI_SWIGLU && !leader) ? &tmB1 : &tmB0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) {
             ok = false;
@@ -340,14 +361,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             else
               tma_load_2d_pair(a_dst, &tmA, full_leader, k0, row0);
             if (p.b_chunked) {
-              // SwiGLU: leader loads W1 columns (gate half), peer the same
-              // columns of W3 (up half); otherwise the two column halves.
-              tma_load_4d_pair(b_dst, mb, full_leader, 0, k0, c0, e);
+              tma_load_4d_pair(b_dst, &tmB0, full_leader, 0, k0, c0, e);
+              if (EPI == EPI_SWIGLU) tma_load_4d_pair(b_dst + B_CHUNK, &tmB1, full_leader, 0, k0, c0, e);
+            } else if (EPI == EPI_SWIGLU) {
+              const int n0 = n * (TN / 2) + static_cast<int>(rank) * 64;
+              tma_load_3d_pair(b_dst, &tmB0, full_leader, n0, k0, e);
+              tma_load_3d_pair(b_dst + B_BOX_BYTES, &tmB1, full_leader, n0, k0, e);
             } else {
-              const int n0 = EPI == EPI_SWIGLU ? n * (TN / 2)
-                                               : n * TN + static_cast<int>(rank) * (TN / 2);
-              tma_load_3d_pair(b_dst, mb, full_leader, n0, k0, e);
-              tma_load_3d_pair(b_dst + B_BOX_BYTES, mb, full_leader, n0 + 64, k0, e);
+              const int n0 = n * TN + static_cast<int>(rank) * (TN / 2);
+              tma_load_3d_pair(b_dst, &tmB0, full_leader, n0, k0, e);
+              tma_load_3d_pair(b_dst + B_BOX_BYTES, &tmB0, full_leader, n0 + 64, k0, e);
             }
           }
           ++nissued;
@@ -399,7 +422,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_bf16_f32(TILE_M, TN, false, true);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(TILE_M, TN, false, true);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(TILE_M / 2, TN, false, true);
       // Descriptors of stage 0; a stage and a 16-wide K step only move the
       // 14-bit start-address field (addresses < 256 KB never carry out of it).
       const uint64_t adesc0 = smem_desc_sw128(smem_base, 16, 1024);
@@ -429,6 +453,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         issued_any = true;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * TN);
+        int te, tm, tn;
+        decode_tile(c, t, te, tm, tn);
+        const uint32_t idesc = is_half_tile<CG>(p, c, te, tm * TILE_M) ? idesc_half : idesc_full;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase)) {
             ok = false;
@@ -552,26 +579,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * TN);
-      const int blk_row = m * TILE_M + static_cast<int>(rank) * TM;
+      // Full tiles: this warp's 32 rows of the CTA's 128.  Half tiles: 32 of
+      // the CTA's 64 rows (quad & 1) and one half of the tile's columns
+      // (quad >> 1), as the M = 128 pair accumulator lays them out.
+      const bool half_m = is_half_tile<CG>(p, c, e, m * TILE_M);
+      const int rsub = half_m ? (quad & 1) * 32 : quad * 32;
+      const int chalf = half_m ? (quad >> 1) : 0;
+      const int blk_row = m * TILE_M + static_cast<int>(rank) * (half_m ? TM / 2 : TM);
       const bool blk_ok = blk_row < c.kept[e];
-      const int row0 = c.off[e] + blk_row + quad * 32;
-      const int valid_rows = c.kept[e] - (blk_row + quad * 32);  // rows of this warp's box to keep
+      const int row0 = c.off[e] + blk_row + rsub;
+      const int valid_rows = c.kept[e] - (blk_row + rsub);  // rows of this warp's box to keep
       if (EPI == EPI_SWIGLU || EPI == EPI_GELU) {
         // bf16 output (h): one 32-column chunk per TMEM wait, each lane
         // storing its own row's 64 bytes.  (Loading several chunks per wait
         // made this epilogue slower than the MMAs of a short tile: the
         // up projection of the 1024-wide layer lost 40%.)
-        const int n0 = EPI == EPI_SWIGLU ? n * (TN / 2) : n * TN;
-        constexpr int NCH = (EPI == EPI_SWIGLU ? 4 : TN / 32) / EPI_SPLIT;  // chunks of this warp
+        const int n0 = EPI == EPI_SWIGLU ? n * (TN / 2) + chalf * 64 : n * TN + chalf * (TN / 2);
+        const int NCH = half_m ? (EPI == EPI_SWIGLU ? 2 : 4)
+                               : (EPI == EPI_SWIGLU ? 4 : TN / 32) / EPI_SPLIT;  // chunks of this warp
         const bool row_ok = blk_ok && lane < valid_rows;
         __nv_bfloat16* dst_row =
             static_cast<__nv_bfloat16*>(p.out) + static_cast<int64_t>(row0 + lane) * p.ld_out;
 #pragma unroll 1
         for (int ci = 0; ci < NCH; ++ci) {
           const int cc = half * NCH + ci;
+          // TMEM columns of the gate (or GELU input) and up values of the h
+          // columns n0 + 32 cc ..: a pair holds, per CTA, a W1 chunk next to
+          // the same W3 chunk (64 columns each); one CTA, all of W1's
+          // columns, then W3's.
+          int gcol = cc * 32, ucol = TN / 2 + cc * 32;
+          if (EPI == EPI_SWIGLU && CG == 2) {
+            gcol = half_m ? cc * 32 : (cc >> 1) * 128 + (cc & 1) * 32;
+            ucol = gcol + 64;
+          }
           float g[32], u[32];
-          tc_ld_32cols(tbase + cc * 32, g);
-          if (EPI == EPI_SWIGLU) tc_ld_32cols(tbase + TN / 2 + cc * 32, u);
+          tc_ld_32cols(tbase + gcol, g);
+          if (EPI == EPI_SWIGLU) tc_ld_32cols(tbase + ucol, u);
           tc_wait_ld();
           if (ci == NCH - 1) release(acc);
           if (row_ok) {
@@ -595,8 +638,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {
-        const int n0 = n * TN;
-        constexpr int NCH = TN / 32 / EPI_SPLIT;  // 32-column chunks of this warp
+        const int n0 = n * TN + chalf * (TN / 2);
+        const int NCH = half_m ? 4 : TN / 32 / EPI_SPLIT;  // 32-column chunks of this warp
 #pragma unroll 1
         for (int c0 = half * NCH; c0 < (half + 1) * NCH; c0 += 4) {
           float g[4][32];
@@ -770,6 +813,17 @@ bool use_cta_pairs() {
   return pairs;
 }
 
+// Half-height pair tiles for an expert's short last block (see
+// is_half_tile); MOE_TC_HALF_TILES=0 computes it as a full pair tile, for
+// measurements.
+bool half_tiles() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_TC_HALF_TILES");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 template <int EPI>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& out, const TcParams& p, int num_sms, int64_t tiles_max,
@@ -798,7 +852,9 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   const bool up_chunked = a.H % 64 == 0, dn_chunked = a.d % 64 == 0;
   const bool up_wide = pairs && up_chunked && a.d % 64 == 0;
   const bool dn_wide = pairs && dn_chunked && a.H % 64 == 0;
-  const uint32_t up_chunks = pairs ? 2 : (swiglu ? 2 : 4), dn_chunks = pairs ? 2 : 4;
+  // Pairs: SwiGLU loads one chunk of W1 and the same chunk of W3 per CTA,
+  // otherwise two adjacent chunks; one CTA: all chunks of its columns.
+  const uint32_t up_chunks = pairs ? (swiglu ? 1 : 2) : (swiglu ? 2 : 4), dn_chunks = pairs ? 2 : 4;
   bool ok = (up_wide ? make_map_a3d(&mx, a.xp, a.rows, a.d) : make_map_2d(&mx, a.xp, a.rows, a.d, TM)) &&
             (dn_wide ? make_map_a3d(&mh, a.h, a.rows, a.H) : make_map_2d(&mh, a.h, a.rows, a.H, TM));
   const uint32_t up_kr = up_wide ? 128 : 64, dn_kr = dn_wide ? 128 : 64;
@@ -826,6 +882,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   up.kept = a.kept_counts;
   up.err = a.dev_error;
   up.debug_stall = take_debug_stall();
+  up.half_tiles = half_tiles() ? 1 : 0;
   cudaError_t err =
       swiglu ? launch_gemm<EPI_SWIGLU>(mx, mw1, mw3, mh_out, up, num_sms,
                                        mtiles_max * up.n_tiles, up_wide, s)
@@ -847,6 +904,7 @@ moe_status launch_ffn_tc(const FfnArgs& a, cudaStream_t s, int num_sms, cudaEven
   dn.kept = a.kept_counts;
   dn.err = a.dev_error;
   dn.debug_stall = 0;
+  dn.half_tiles = half_tiles() ? 1 : 0;
   err = launch_gemm<EPI_PLAIN>(mh, mw2, mw2, mo_out, dn, num_sms, mtiles_max * dn.n_tiles,
                                    dn_wide, s);
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
