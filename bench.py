@@ -121,11 +121,13 @@ MAX_ROOFLINE_FRAC = 1.05
 
 
 def choose_bf16_peak(peaks, loop_s, clk, src="measured"):
-    """The bf16 denominator that fits the timed region: the sustained
-    (power-capped) figure only when the region is a loop of at least a second
-    whose sampled clocks show sw_power_cap with the median SM clock below 92 %
-    of max; the burst figure otherwise.  Returns (peak, description)."""
-    sustained = (loop_s >= 1.0 and clk is not None and "sw_power_cap" in clk.get("reasons", [])
+    """The bf16 denominator that fits the timed region, decided by the clocks
+    sampled during it: the sustained (power-capped) figure when at least two
+    samples show sw_power_cap and their median SM clock is below 92 % of max;
+    the burst figure otherwise (full clock, a cap that only flickered, or no
+    samples).  Returns (peak, description)."""
+    sustained = (clk is not None and clk.get("samples", 0) >= 2
+                 and "sw_power_cap" in clk.get("reasons", [])
                  and clk.get("sm_mhz", 0) < 0.92 * clk.get("sm_max_mhz", 1))
     clock = (f", median SM clock {clk['sm_mhz']:.0f} of {clk['sm_max_mhz']:.0f} MHz"
              f"{' (' + ', '.join(clk['reasons']) + ')' if clk.get('reasons') else ''}"
@@ -598,6 +600,8 @@ def main(argv=None):
     if w.dtype == "bf16":
         # The achieved rate comes from the stage loop, so its length and the
         # clocks of the headline loop just before it pick the peak.
+        # (The stage loop follows the headline loop at once, so it runs in
+        # the clock regime that loop's samples show.)
         roof_peak, roof_src = choose_bf16_peak(peaks, stage_loop_s, clk, peak_src)
         roofline = {"kernel": f"ffn_tc_kernel<{act_name}> (grouped up projection)",
                     "bound": "tensor",

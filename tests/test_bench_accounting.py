@@ -23,6 +23,17 @@ def test_short_loop_stays_burst_even_if_the_cap_flickers():
     assert bench.choose_bf16_peak(PEAKS, 0.5, clk)[0] == 1610.6
 
 
+def test_throttled_loop_under_a_second_takes_the_sustained_peak():
+    # the 200-step default loop: 0.92 s, median 1597 MHz under the cap
+    clk = {"sm_mhz": 1597.0, "sm_max_mhz": 1965.0, "samples": 6, "reasons": ["sw_power_cap"]}
+    assert bench.choose_bf16_peak(PEAKS, 0.92, clk)[0] == 1373.6
+
+
+def test_a_single_clock_sample_is_not_evidence_of_throttling():
+    clk = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "samples": 1, "reasons": ["sw_power_cap"]}
+    assert bench.choose_bf16_peak(PEAKS, 2.0, clk)[0] == 1610.6
+
+
 def test_long_power_capped_loop_takes_the_sustained_peak():
     clk = {"sm_mhz": 1320.0, "sm_max_mhz": 1965.0, "samples": 12, "reasons": ["sw_power_cap"]}
     peak, src = bench.choose_bf16_peak(PEAKS, 2.4, clk)
