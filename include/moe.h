@@ -366,7 +366,8 @@ moe_status moe_pipeline_wait(moe_pipeline* p, int32_t slot);
 moe_status moe_pipeline_destroy(moe_pipeline* p);
 
 /* One forward captured as a CUDA graph, for small layers whose forward is
- * shorter than the host's launch work (seven kernels and two memsets).
+ * shorter than the host's launch work (a handful of kernels and a memset;
+ * moe_forward_graph_nodes counts them).
  * moe_forward_graph_create records moe_forward_ex with these arguments
  * (stats not available) on a private stream and instantiates it; nothing
  * runs yet.  The graph keeps the pointers it was made with: x, y, ws and the
@@ -386,6 +387,11 @@ moe_status moe_forward_graph_create(const void* x, const void* Wg, const float* 
                                     moe_graph** out);
 moe_status moe_forward_graph_launch(moe_graph* g, void* stream);
 moe_status moe_forward_graph_destroy(moe_graph* g);
+/* What one launch of the graph runs: *kernels = its kernel nodes (every one
+ * a kernel of this library), *others = the rest (memsets).  Host-only, no
+ * GPU work.  Errors: MOE_ERR_ARG for a NULL argument; MOE_ERR_CUDA if the
+ * graph cannot be read. */
+moe_status moe_forward_graph_nodes(const moe_graph* g, int32_t* kernels, int32_t* others);
 
 /* Stage timing.  `events` points to MOE_NUM_STAGE_EVENTS cudaEvent_t
  * handles (passed as void*) created by the caller, or is NULL to stop.  The

@@ -796,6 +796,26 @@ MOE_API moe_status moe_forward_graph_launch(moe_graph* g, void* stream) {
              : MOE_ERR_CUDA;
 }
 
+MOE_API moe_status moe_forward_graph_nodes(const moe_graph* g, int32_t* kernels,
+                                           int32_t* others) {
+  if (!g || !kernels || !others) return MOE_ERR_ARG;
+  size_t n = 0;
+  if (cudaGraphGetNodes(g->graph, nullptr, &n) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaGraphNode_t nodes[64];
+  if (n > 64) return MOE_ERR_CUDA;  // a forward holds a handful of nodes
+  if (n > 0 && cudaGraphGetNodes(g->graph, nodes, &n) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t nk = 0, no = 0;
+  for (size_t i = 0; i < n; ++i) {
+    cudaGraphNodeType t;
+    if (cudaGraphNodeGetType(nodes[i], &t) != cudaSuccess) return MOE_ERR_CUDA;
+    if (t == cudaGraphNodeTypeKernel) ++nk;
+    else ++no;
+  }
+  *kernels = nk;
+  *others = no;
+  return MOE_OK;
+}
+
 MOE_API moe_status moe_forward_graph_destroy(moe_graph* g) {
   if (!g) return MOE_OK;
   moe_status st = MOE_OK;

@@ -36,6 +36,7 @@ EXPORTED = (
     "moe_expert_choice_workspace_bytes", "moe_forward_expert_choice", "moe_pipeline_create",
     "moe_pipeline_submit", "moe_pipeline_wait", "moe_pipeline_destroy",
     "moe_forward_graph_create", "moe_forward_graph_launch", "moe_forward_graph_destroy",
+    "moe_forward_graph_nodes",
     "moe_probe_stream_read",
 )
 MOE_PIPELINE_MAX_DEPTH = 4
@@ -208,6 +209,8 @@ def lib():
     L.moe_forward_graph_launch.argtypes = [_P, _P]
     L.moe_forward_graph_destroy.restype = ctypes.c_int
     L.moe_forward_graph_destroy.argtypes = [_P]
+    L.moe_forward_graph_nodes.restype = ctypes.c_int
+    L.moe_forward_graph_nodes.argtypes = [_P, _P, _P]
     L.moe_forward_expert_choice.restype = ctypes.c_int
     L.moe_forward_expert_choice.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                             _D, ctypes.c_int, ctypes.c_int, _P, _P, _SZ,
@@ -572,6 +575,13 @@ class ForwardGraph:
         _check(lib().moe_forward_graph_launch(self._h, _stream(self.x.device, stream)),
                "moe_forward_graph_launch")
         return self.y
+
+    def nodes(self):
+        """(kernel nodes, other nodes) of one launch (moe_forward_graph_nodes)."""
+        nk, no = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().moe_forward_graph_nodes(self._h, ctypes.byref(nk), ctypes.byref(no)),
+               "moe_forward_graph_nodes")
+        return nk.value, no.value
 
     def close(self):
         if self._h:

@@ -294,3 +294,6 @@ def test_graph_arguments_are_checked_before_any_cuda_call(lib):
     assert not out.value
     assert lib.moe_forward_graph_launch(None, None) == M.MOE_ERR_ARG
     assert lib.moe_forward_graph_destroy(None) == M.MOE_OK
+    nk, no = ctypes.c_int32(-1), ctypes.c_int32(-1)
+    assert lib.moe_forward_graph_nodes(None, ctypes.byref(nk), ctypes.byref(no)) == M.MOE_ERR_ARG
+    assert nk.value == -1 and no.value == -1

@@ -47,3 +47,24 @@ def test_graph_replay_matches_eager(name):
     assert torch.equal(g.y, y_ref2)
     assert not torch.equal(y_ref2, y_ref)
     g.close()
+
+
+def test_graph_holds_the_forward_kernels():
+    """The bf16 layer with a streaming router (E a multiple of 8, at most 64)
+    is five kernels -- router (with the permutation's counting), placement
+    and copy, the two GEMMs, the combine -- and one memset of the error flag;
+    priority routing adds the gate-order kernels."""
+    w = WORKLOADS["top2_bf16"].replace(T=600, d=256, H=384)
+    t = make_inputs(w, "cuda")
+    layer = M.MoELayer(t["Wg"], t["bias"], t["W1"], t["W3"], t["W2"], w.k, w.cf, w.act)
+    g = layer.graph(t["x"])
+    assert g.nodes() == (5, 1)
+    g.close()
+    w, priority = CASES["bpr_ragged"]
+    t = make_inputs(w, "cuda")
+    bpr = M.MoELayer(t["Wg"], t["bias"], t["W1"], t["W3"], t["W2"], w.k, w.cf, w.act,
+                     priority=priority)
+    g = bpr.graph(t["x"])
+    nk, no = g.nodes()
+    assert nk > 5 and no >= 1
+    g.close()

@@ -398,3 +398,17 @@ def test_batch_priority_routing_full_size_openmoe():
             assert pd.max() <= pk.min()
     max_abs, rel = _whole_batch_y(w, g, cpu, logits, kept)
     print(f"BPR openmoe: max_abs={max_abs:.3g} rel_fro={rel:.3g}")
+
+
+def test_plain_read_probe_reads_every_byte():
+    """moe_probe_stream_read (the measurement aid): its sink is the XOR of
+    every 32-bit word of the buffer, so a read that skipped any 16 bytes
+    (or read one twice) would show."""
+    g = torch.Generator().manual_seed(5)
+    for n in (16, 4096, (1 << 22) + 48):
+        buf = torch.randint(-2**31, 2**31 - 1, (n // 4,), generator=g, dtype=torch.int32)
+        sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+        M.moe_probe_stream_read(buf.cuda(), sink)
+        torch.cuda.synchronize()
+        want = np.bitwise_xor.reduce(buf.numpy().view(np.uint32))
+        assert int(sink.item()) & 0xffffffff == int(want), n
