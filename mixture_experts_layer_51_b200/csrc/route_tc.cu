@@ -59,7 +59,7 @@ __device__ __forceinline__ void insert_sorted_tc(float (&tv)[KM], int (&ti)[KM],
   for (int j = 0; j < KM; ++j) {
     // larger value, or equal value and lower expert (an entry pushed down
     // the list keeps its place in front of an equal logit of a higher one)
-    const bool take = ei >= 0 && (ti[j] < 0 || v > tv[j] || (v == tv[j] && ei < ti[j]));
+    const bool take = (ei >= 0) & ((ti[j] < 0) | (v > tv[j]) | ((v == tv[j]) & (ei < ti[j])));
     const float tvj = tv[j];
     const int tij = ti[j];
     tv[j] = take ? v : tvj;

@@ -412,3 +412,29 @@ def test_plain_read_probe_reads_every_byte():
         torch.cuda.synchronize()
         want = np.bitwise_xor.reduce(buf.numpy().view(np.uint32))
         assert int(sink.item()) & 0xffffffff == int(want), n
+
+
+def test_reversed_k_rounds_opt_in():
+    """MOE_TC_SERPENTINE=1 (read once per process, so in a child): the down
+    projection runs the K steps of every other round of a CTA pair in
+    reverse.  The many-tiles layer (256 down-projection tiles on at most 74
+    pairs: both orders) and the small layers still match the oracle."""
+    import os
+    import subprocess
+    import sys
+    import textwrap
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = textwrap.dedent("""
+        import sys
+        sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
+        import test_gpu_parity as T
+        T.test_many_tiles_per_cta_pair()
+        for name in T.SMALL:
+            T.test_small_layer_parity(name)
+        print("REVERSED_K_OK")
+    """).format(root=root, tests=os.path.join(root, "tests"))
+    env = dict(os.environ, MOE_TC_SERPENTINE="1")
+    r = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stderr[-3000:]
+    assert "REVERSED_K_OK" in r.stdout
