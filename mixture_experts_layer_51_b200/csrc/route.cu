@@ -102,19 +102,6 @@ __device__ __forceinline__ void topk_softmax_store(Get get, int E, int k, int t,
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -331,48 +318,77 @@ __global__ void __launch_bounds__(256)
                       const float* __restrict__ bias, int T, int d, int E, int k,
                       int32_t* __restrict__ idx, float* __restrict__ gate,
                       float* __restrict__ margin, int gating, float gate_scale,
-                      float* __restrict__ scores) {
+                      float* __restrict__ scores, int32_t* __restrict__ lrank,
+                      int32_t* __restrict__ hist) {
   __shared__ float lg[8][kMaxE];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  const float* xr = x + (int64_t)t * d;
-  for (int e0 = 0; e0 < E; e0 += 8) {
-    float acc[8];
+  if (t < T) {
+    const float* xr = x + (int64_t)t * d;
+    for (int e0 = 0; e0 < E; e0 += 8) {
+      float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int c = lane; c < d; c += 32) {
-      const float xv = xr[c];
-      const float* w = Wg + (int64_t)c * E + e0;
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int c = lane; c < d; c += 32) {
+        const float xv = xr[c];
+        const float* w = Wg + (int64_t)c * E + e0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (e0 + i < E) acc[i] = fmaf(xv, w[i], acc[i]);
+        for (int i = 0; i < 8; ++i)
+          if (e0 + i < E) acc[i] = fmaf(xv, w[i], acc[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (e0 + i < E) lg[warp][e0 + i] = acc[i];
+      }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (e0 + i < E) lg[warp][e0 + i] = acc[i];
+    __syncwarp();
+    auto get = [&](int e) { return bias ? lg[warp][e] + bias[e] : lg[warp][e]; };
+    if (scores) {
+      // Expert-choice affinities (softmax over all E), same order of
+      // operations in every lane.
+      float m = -INFINITY;
+      for (int e = 0; e < E; ++e) m = fmaxf(m, get(e));
+      float sum = 0.f;
+      for (int e = 0; e < E; ++e) sum += expf(get(e) - m);
+      const float inv = 1.f / sum;
+      for (int e = lane; e < E; e += 32) scores[(int64_t)e * T + t] = expf(get(e) - m) * inv;
+    } else if (lane == 0) {
+      topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
     }
   }
-  __syncwarp();
-  auto get = [&](int e) { return bias ? lg[warp][e] + bias[e] : lg[warp][e]; };
-  if (scores) {
-    // Expert-choice affinities (softmax over all E), same order of
-    // operations in every lane.
-    float m = -INFINITY;
-    for (int e = 0; e < E; ++e) m = fmaxf(m, get(e));
-    float sum = 0.f;
-    for (int e = 0; e < E; ++e) sum += expf(get(e) - m);
-    const float inv = 1.f / sum;
-    for (int e = lane; e < E; e += 32) scores[(int64_t)e * T + t] = expf(get(e) - m) * inv;
-    return;
+  if (!lrank) return;
+  // The counting half of the permutation, when this block's 8 tokens are one
+  // token range: each assignment's rank among the block's earlier ones to
+  // the same expert (-1 for an expert outside [0, E)), and the block's
+  // assignments per expert.  (idx, written above by other warps, is visible
+  // to the block after the barrier.)
+  __syncthreads();
+  const int t0 = blockIdx.x * 8, n = min(8, T - t0);
+  const int tid = threadIdx.x;
+  if (tid < n) {
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)(t0 + tid) * k + j];
+      int r = -1;
+      if (e >= 0 && e < E) {
+        r = 0;
+        for (int q = 0; q < tid * k; ++q) r += idx[(int64_t)t0 * k + q] == e;
+      }
+      lrank[(int64_t)(t0 + tid) * k + j] = r;
+    }
   }
-  if (lane == 0) topk_softmax_store<kMaxK + 1>(get, E, k, t, idx, gate, margin, gating, gate_scale);
+  if (tid < E) {
+    int c = 0;
+    for (int q = 0; q < n * k; ++q) c += idx[(int64_t)t0 * k + q] == tid;
+    hist[(int64_t)blockIdx.x * E + tid] = c;
+  }
 }
 
 template <int NT, int BM, int BK, int STAGES, int CL, int KM>
@@ -446,11 +462,17 @@ cudaError_t launch_route(const RouteArgs& a, moe_dtype dtype, cudaStream_t s, in
   if (ranked) *ranked = false;
   if (a.T == 0) return cudaSuccess;
   if (dtype == MOE_FP32) {
-    route_fp32_kernel<<<(a.T + 7) / 8, 256, 0, s>>>(static_cast<const float*>(a.x),
-                                                    static_cast<const float*>(a.Wg), a.bias, a.T,
-                                                    a.d, a.E, a.k, a.idx, a.gate, a.margin,
-                                                    a.gating, a.gate_scale, a.scores);
-    return cudaGetLastError();
+    // The blocks of 8 tokens are the permutation's token ranges when there
+    // are at most as many groups of 8 as ranges: then the router also counts.
+    const RouteRanges rg = route_ranges(a.T, num_sms);
+    const bool count = a.lrank && a.hist && !a.scores && rg.G == rg.T8;
+    const cudaError_t err = launch_kernel(
+        route_fp32_kernel, dim3((a.T + 7) / 8), dim3(256), 0, s, 1, true,
+        static_cast<const float*>(a.x), static_cast<const float*>(a.Wg), a.bias, a.T, a.d, a.E,
+        a.k, a.idx, a.gate, a.margin, a.gating, a.gate_scale, a.scores,
+        count ? a.lrank : nullptr, count ? a.hist : nullptr);
+    if (ranked) *ranked = err == cudaSuccess && count;
+    return err;
   }
   if (route_stream_supported(a)) {
     const cudaError_t err = launch_route_stream(a, num_sms, s);

@@ -56,11 +56,16 @@ def test_full_switch_tiny_fp32():
     dict(T=1703, d=320, E=24, k=3, H=128),       # W_g box wider than E (24 of 32), d % 256 != 0
     dict(T=9999, d=200, E=40, k=5, H=96),        # router tiles of 72 rows, ragged last range
     dict(T=21011, d=128, E=16, k=2, H=64, cf=1.0),  # two router tiles per range
+    # fp32: the router counts when its 8-token blocks are the token ranges
+    # (T <= 8 x SMs) and leaves it to the permutation otherwise
+    dict(T=333, d=72, E=5, k=2, H=200, cf=1.0, dtype="fp32"),
+    dict(T=2500, d=64, E=4, k=2, H=136, cf=1.25, act="gelu", dtype="fp32"),
 ])
 def test_edge_shapes(case):
     act = case.pop("act", "swiglu")
     cf = case.pop("cf", 0.0)
-    w = Workload("edge", act=act, dtype="bf16", cf=cf, seed=11, **case)
+    dtype = case.pop("dtype", "bf16")
+    w = Workload("edge", act=act, dtype=dtype, cf=cf, seed=11, **case)
     full_parity(w, make_inputs(w, "cpu"))
 
 
@@ -288,6 +293,50 @@ def test_grouped_ffn_against_oracle(act):
         o_ref = h[r].astype(np.float64) @ W2[e].double().numpy()
         bound = 2.0 ** -8 * np.abs(o_ref) + 1e-5 * np.abs(o_ref).max()
         assert np.all(np.abs(o[r] - o_ref) <= bound), f"o expert {e}"
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+@pytest.mark.parametrize("d,H", [(72, 200), (200, 136)])
+def test_grouped_ffn_fp32_against_oracle(act, d, H):
+    """The fp32 grouped FFN (CUDA cores) alone: K of 72 (a partial last K
+    slab) and 200 (seven slabs through the four-stage ring), a partial last
+    column tile, an empty expert, a one-row expert, blocks that end inside
+    a 64-row tile."""
+    torch.manual_seed(1)
+    E = 5
+    kept = [130, 0, 257, 1, 128]
+    off = [0]
+    for c in kept:
+        off.append(off[-1] + (c + 127) // 128 * 128)
+    rows = off[-1]
+    xp = torch.randn(rows, d)
+    W1 = torch.randn(E, d, H) / d ** 0.5
+    W3 = torch.randn(E, d, H) / d ** 0.5 if act == "swiglu" else None
+    W2 = torch.randn(E, H, d) / H ** 0.5
+    dev = torch.device("cuda")
+    offs = torch.tensor(off, dtype=torch.int32, device=dev)
+    kc = torch.tensor(kept, dtype=torch.int32, device=dev)
+    h, o, err = M.moe_grouped_ffn(xp.to(dev), offs, kc, W1.to(dev),
+                                  None if W3 is None else W3.to(dev), W2.to(dev), act)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    h = to_np(h)
+    o = to_np(o)
+    for e in range(E):
+        r = slice(off[e], off[e] + kept[e])
+        if kept[e] == 0:
+            continue
+        x64 = xp[r].double().numpy()
+        if act == "swiglu":
+            h_ref = oracle.silu(x64 @ W1[e].double().numpy()) * (x64 @ W3[e].double().numpy())
+        else:
+            h_ref = oracle.gelu(x64 @ W1[e].double().numpy())
+        # fp32 accumulation of K products of O(1) terms: a few 1e-7 relative
+        # to the row's scale.
+        scale_h = np.abs(h_ref).max()
+        assert np.abs(h[r] - h_ref).max() <= 1e-5 * scale_h, f"h expert {e}"
+        o_ref = h_ref @ W2[e].double().numpy()
+        assert np.abs(o[r] - o_ref).max() <= 1e-5 * np.abs(o_ref).max(), f"o expert {e}"
 
 
 # ------------------------------------------------------ full-size layers
