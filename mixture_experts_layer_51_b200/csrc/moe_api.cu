@@ -368,6 +368,17 @@ MOE_API moe_status moe_unpermute_combine(const void* o, const int32_t* pos, cons
 
 namespace {
 
+// The device pointers a whole forward reads and writes, checked before
+// anything is enqueued: present, and 16-byte aligned where the kernels read
+// or write them in 16-byte vectors or TMA boxes (the bias is read one float
+// at a time).
+bool forward_ptrs_ok(const void* x, const void* Wg, const void* W1, const void* W3,
+                     const void* W2, moe_act act, const void* y) {
+  if (!x || !Wg || !W1 || !W2 || !y || (act == MOE_SWIGLU && !W3)) return false;
+  return aligned16(x) && aligned16(Wg) && aligned16(W1) &&
+         (act != MOE_SWIGLU || aligned16(W3)) && aligned16(W2) && aligned16(y);
+}
+
 moe_status forward_enqueue(const void* x, const void* Wg, const float* bias, const void* W1,
                            const void* W3, const void* W2, int32_t T, int32_t d, int32_t H,
                            int32_t E, int32_t k, double cf, moe_act act, moe_dtype dt, void* y,
@@ -440,7 +451,9 @@ MOE_API moe_status moe_forward_ex(const void* x, const void* Wg, const float* bi
   int priority;
   if (!compute_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
   if (!read_options(opt, &gating, &gate_scale, &priority)) return MOE_ERR_ARG;
-  if (T > 0 && (!y || !ws || ws_bytes < L.total || !aligned16(ws))) return MOE_ERR_ARG;
+  if (T > 0 && (!forward_ptrs_ok(x, Wg, W1, W3, W2, act, y) || !ws || ws_bytes < L.total ||
+                !aligned16(ws)))
+    return MOE_ERR_ARG;
   if (T == 0) {
     if (stats) {
       memset(stats, 0, sizeof(*stats));
@@ -535,7 +548,9 @@ MOE_API moe_status moe_forward_host(const void* x_host, void* y_host, void* x_de
   moe_ws_layout L;
   if (!compute_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
   if (T == 0) return MOE_OK;
-  if (!x_host || !y_host || !x_dev || !y_dev || !ws || ws_bytes < L.total) return MOE_ERR_ARG;
+  if (!x_host || !y_host || !forward_ptrs_ok(x_dev, Wg, W1, W3, W2, act, y_dev) || !ws ||
+      ws_bytes < L.total || !aligned16(ws))
+    return MOE_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t row_bytes = static_cast<size_t>(d) * elt_size(dt);
   const int nchunk = host_chunks(T, cf);
@@ -672,7 +687,8 @@ MOE_API moe_status moe_pipeline_submit(moe_pipeline* p, int32_t slot, const void
       !read_options(opt, &gating, &gate_scale, &priority))
     return MOE_ERR_ARG;
   if (T == 0) return MOE_OK;
-  if (!x_host || !y_host || !x_dev || !y_dev || !ws || ws_bytes < L.total || !aligned16(ws))
+  if (!x_host || !y_host || !forward_ptrs_ok(x_dev, Wg, W1, W3, W2, act, y_dev) || !ws ||
+      ws_bytes < L.total || !aligned16(ws))
     return MOE_ERR_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -743,8 +759,8 @@ MOE_API moe_status moe_forward_graph_create(const void* x, const void* Wg, const
   if (!compute_layout(T, d, H, E, k, cf, dt, act, &L) ||
       !read_options(opt, &gating, &gate_scale, &priority))
     return MOE_ERR_ARG;
-  if (T == 0 || !x || !Wg || !W1 || !W2 || (act == MOE_SWIGLU && !W3) || !y || !ws ||
-      ws_bytes < L.total || !aligned16(ws))
+  if (T == 0 || !forward_ptrs_ok(x, Wg, W1, W3, W2, act, y) || !ws || ws_bytes < L.total ||
+      !aligned16(ws))
     return MOE_ERR_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
@@ -973,7 +989,9 @@ MOE_API moe_status moe_forward_expert_choice(const void* x, const void* Wg, cons
                                              moe_stats* stats, void* stream) {
   moe_ec_ws_layout L;
   if (!ec_layout(T, d, H, E, k, cf, dt, act, &L)) return MOE_ERR_ARG;
-  if (T > 0 && (!y || !ws || ws_bytes < L.total || !aligned16(ws))) return MOE_ERR_ARG;
+  if (T > 0 && (!forward_ptrs_ok(x, Wg, W1, W3, W2, act, y) || !ws || ws_bytes < L.total ||
+                !aligned16(ws)))
+    return MOE_ERR_ARG;
   if (stats) memset(stats, 0, sizeof(*stats));
   if (T == 0) {
     if (stats) stats->capacity = moe_capacity(T, E, k, cf);

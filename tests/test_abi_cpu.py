@@ -130,6 +130,26 @@ def test_invalid_arguments_are_rejected_before_any_cuda_call(lib):
     st = lib.moe_forward(fake, fake, None, fake, fake, fake, 64, 64, 64, 8, 2, 0.0, M.MOE_SWIGLU,
                          M.MOE_BF16, fake, fake, 16, None, None)
     assert st == M.MOE_ERR_ARG
+    # forward: a missing or misaligned weight or output is refused before
+    # anything is enqueued (a workspace large enough, so only that differs)
+    big = 1 << 40
+    odd = P(0x10008)
+    for args in [(fake, fake, None, odd, fake, fake),     # W1 misaligned
+                 (fake, fake, None, fake, None, fake),    # SwiGLU without W3
+                 (fake, fake, None, fake, fake, odd),     # W2 misaligned
+                 (odd, fake, None, fake, fake, fake),     # x misaligned
+                 (fake, None, None, fake, fake, fake)]:   # no router weights
+        st = lib.moe_forward(*args, 64, 64, 64, 8, 2, 0.0, M.MOE_SWIGLU, M.MOE_BF16, fake, fake,
+                             big, None, None)
+        assert st == M.MOE_ERR_ARG, args
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, 64, 64, 64, 8, 2, 0.0, M.MOE_SWIGLU,
+                         M.MOE_BF16, odd, fake, big, None, None)  # y misaligned
+    assert st == M.MOE_ERR_ARG
+    # GELU ignores W3, aligned or not: the call gets past the checks (to the
+    # first CUDA call, which fails here without a GPU)
+    st = lib.moe_forward(fake, fake, None, fake, odd, fake, 64, 64, 64, 8, 2, 0.0, M.MOE_GELU,
+                         M.MOE_BF16, fake, fake, big, None, None)
+    assert st != M.MOE_ERR_ARG
 
 
 def test_empty_batch_is_a_no_op(lib):
