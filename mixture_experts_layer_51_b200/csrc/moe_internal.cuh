@@ -158,6 +158,14 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// Untiled bulk copy shared -> global of `bytes` contiguous bytes (both
+// addresses 16-byte aligned, bytes a multiple of 16), completion tracked by
+// the issuing thread's bulk groups (bulk_commit / bulk_wait_read).
+__device__ __forceinline__ void bulk_store_1d(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
 // Untiled bulk copy global -> shared of `bytes` contiguous bytes (both
 // addresses 16-byte aligned, bytes a multiple of 16), completion on `bar`.
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
@@ -445,6 +453,10 @@ cudaError_t launch_route_tc(const RouteArgs& a, cudaStream_t s);
 // Whether kernels of the forward chain are launched with programmatic
 // dependent launch (default on; MOE_PDL=0 turns it off, for measurements).
 bool pdl_enabled();
+// Whether the placement kernel carries rows out with bulk stores from
+// shared memory (default on for rows up to 8 KB; MOE_PLACE_BULK=0 turns it
+// off, for measurements).
+bool place_bulk();
 
 // cudaLaunchKernelEx with an optional cluster size and, when `pdl` and
 // pdl_enabled(), programmatic stream serialization.

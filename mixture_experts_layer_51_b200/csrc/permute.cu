@@ -399,8 +399,13 @@ __global__ void __launch_bounds__(kRankThreads)
 // shard of a batch), kept counts and 128-row aligned offsets; CTA 0 writes
 // counts, kept_counts and offsets.  Then one warp per queue position of
 // this CTA's share of the range: pos[t, j] (in: local rank, out: row or -1)
-// and the copy of x[t] to every kept row (16-byte vectors, eight in flight
-// per lane), reading the row once.
+// and the copy of x[t] to every kept row, reading the row once.  BULK: the
+// warp copies the row into one of its two shared-memory row slots
+// (cp.async), then one bulk store per kept row carries it out and is left
+// in flight while the warp loads its next token into the other slot (the
+// copy engine keeps far more bytes in flight than the threads' registers
+// could).  Otherwise: 16-byte vectors, eight in flight per lane.
+template <bool BULK>
 __global__ void __launch_bounds__(kPlaceWarps * 32)
     ranked_place_copy_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ idx,
                              const int32_t* __restrict__ order, int T, int E, int k, int G, int T8,
@@ -411,6 +416,7 @@ __global__ void __launch_bounds__(kPlaceWarps * 32)
   __shared__ int red_b[kPlaceWarps * 32], red_t[kPlaceWarps * 32];
   __shared__ int s_base[kMaxE], s_cap[kMaxE], s_off[kMaxE + 1], s_kept[kMaxE];
   __shared__ int dst[kPlaceWarps][kMaxK];
+  extern __shared__ __align__(128) uint8_t s_rows[];  // BULK: [warp][2][row bytes]
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -464,6 +470,9 @@ __global__ void __launch_bounds__(kPlaceWarps * 32)
   const int q0 = r0 + static_cast<int>(static_cast<int64_t>(sub) * len / S);
   const int q1 = r0 + static_cast<int>(static_cast<int64_t>(sub + 1) * len / S);
   const unsigned lt = (1u << lane) - 1u;
+  const uint32_t row_bytes = static_cast<uint32_t>(dvec) * 16u;
+  const uint32_t slot0 = smem_u32(s_rows) + static_cast<uint32_t>(warp) * 2u * row_bytes;
+  int nrow = 0;  // BULK: rows this warp has loaded
   for (int i = q0 + warp; i < q1; i += kPlaceWarps) {
     const int t = order ? order[i] : i;
     int p = -1;
@@ -483,7 +492,26 @@ __global__ void __launch_bounds__(kPlaceWarps * 32)
     if (p >= 0) dst[warp][__popc(b & lt)] = p;
     const int nd = __popc(b);
     __syncwarp();
-    if (nd > 0) {
+    if (BULK && nd > 0) {
+      const uint32_t slot = slot0 + static_cast<uint32_t>(nrow & 1) * row_bytes;
+      // The bulk stores from this slot (two rows ago) have read it.
+      if (lane == 0 && nrow >= 2) bulk_wait_read<1>();
+      __syncwarp();
+      const uint4* src = x + (int64_t)t * dvec;
+      for (int v = lane; v < dvec; v += 32) cp_async16(slot + v * 16, src + v, 16);
+      cp_async_commit();
+      cp_async_wait<0>();
+      // The row is in shared memory (every lane's copies); make it visible
+      // to the copy engine, then one bulk store per kept row.
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        for (int j = 0; j < nd; ++j)
+          bulk_store_1d(xp + (int64_t)dst[warp][j] * dvec, slot, row_bytes);
+        bulk_commit();
+      }
+      ++nrow;
+    } else if (nd > 0) {
       const uint4* src = x + (int64_t)t * dvec;
       for (int v0 = lane; v0 < dvec; v0 += 32 * 8) {
         uint4 v[8];
@@ -500,6 +528,9 @@ __global__ void __launch_bounds__(kPlaceWarps * 32)
     }
     __syncwarp();
   }
+  // Every bulk store has finished with its slot before the CTA (and its
+  // shared memory) goes away.
+  if (BULK && lane == 0) bulk_wait<0>();
 }
 
 }  // namespace
@@ -525,12 +556,37 @@ cudaError_t launch_ranked_permute(const RankedPermuteArgs& a, moe_dtype dtype, c
   // About four CTAs per SM over all ranges, each range's share at least a
   // few tokens.
   const int per_range = (rg.T8 * 8 + rg.G - 1) / rg.G;
-  const int S = std::max(1, std::min({8, (4 * a.num_sms + rg.G - 1) / rg.G, per_range / 4}));
   const int dvec = a.d * (dtype == MOE_BF16 ? 2 : 4) / 16;
-  return launch_kernel(ranked_place_copy_kernel, dim3(rg.G * S), dim3(kPlaceWarps * 32), 0, s, 1,
-                       true, static_cast<const uint4*>(a.x), a.idx, a.order, a.T, a.E, a.k, rg.G,
-                       rg.T8, S, a.capacity, a.prior, static_cast<const int32_t*>(a.hist), a.pos,
-                       dvec, static_cast<uint4*>(a.xp), a.counts, a.kept_counts, a.offsets);
+  // Bulk copies when two row slots per warp fit beside three CTAs per SM
+  // (rows up to 8 KB: d <= 4096 in bf16); as many CTAs per range as fill
+  // the SMs once, so no CTA repeats the prologue in a second wave.
+  const size_t slots = static_cast<size_t>(kPlaceWarps) * 2 * dvec * 16;
+  const int per_sm = slots == 0 ? 4 : static_cast<int>(std::min<size_t>(4, (227u << 10) / slots));
+  const bool bulk = place_bulk() && per_sm >= 1 && slots <= (128u << 10);
+  const int fill = bulk ? per_sm : 4;
+  const int S = std::max(1, std::min({8, (fill * a.num_sms) / rg.G, per_range / 4}));
+  if (bulk) {
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        ranked_place_copy_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 << 10);
+    if (attr != cudaSuccess) return attr;
+    return launch_kernel(ranked_place_copy_kernel<true>, dim3(rg.G * S), dim3(kPlaceWarps * 32),
+                         slots, s, 1, true, static_cast<const uint4*>(a.x), a.idx, a.order, a.T,
+                         a.E, a.k, rg.G, rg.T8, S, a.capacity, a.prior,
+                         static_cast<const int32_t*>(a.hist), a.pos, dvec,
+                         static_cast<uint4*>(a.xp), a.counts, a.kept_counts, a.offsets);
+  }
+  return launch_kernel(ranked_place_copy_kernel<false>, dim3(rg.G * S), dim3(kPlaceWarps * 32), 0,
+                       s, 1, true, static_cast<const uint4*>(a.x), a.idx, a.order, a.T, a.E, a.k,
+                       rg.G, rg.T8, S, a.capacity, a.prior, static_cast<const int32_t*>(a.hist),
+                       a.pos, dvec, static_cast<uint4*>(a.xp), a.counts, a.kept_counts, a.offsets);
+}
+
+bool place_bulk() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_PLACE_BULK");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 bool pdl_enabled() {
