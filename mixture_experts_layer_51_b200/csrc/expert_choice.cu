@@ -43,6 +43,7 @@ namespace {
 constexpr int kSelCta = 8;       // CTAs per expert (one cluster)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kKeyRegs = 16;     // key chunks a thread keeps in registers
 
 // Ascending order of these keys is descending order of the float (the
 // sign-aware flip turns float order into unsigned order; the complement
@@ -103,17 +104,40 @@ __global__ void __launch_bounds__(kSelThreads)
   const int t_begin = min(T, static_cast<int>(r) * per), t_end = min(T, t_begin + per);
   const float* col = scores + (int64_t)e * T;  // this expert's affinities, contiguous
   auto key_at = [&](int t) { return desc_key(__ldg(col + t)); };
+  // A slice of up to kKeyRegs chunks of kSelThreads keys is read once into
+  // registers; the six passes below then read no memory for their keys.
+  // (The condition is the same for every CTA: per is.)
+  const bool cached = per <= kKeyRegs * kSelThreads;
+  uint32_t kc[kKeyRegs];
+#pragma unroll
+  for (int j = 0; j < kKeyRegs; ++j) {
+    const int t = t_begin + j * kSelThreads + tid;
+    kc[j] = (cached && t < t_end) ? key_at(t) : 0u;
+  }
+  // Visits the slice's tokens in chunks of kSelThreads, in position order:
+  // f(t, valid, key).  Every thread makes the same calls (the warp votes and
+  // block barriers inside f need that).
+  auto visit = [&](auto&& f) {
+    if (cached) {
+#pragma unroll
+      for (int j = 0; j < kKeyRegs; ++j) {
+        if (t_begin + j * kSelThreads < t_end) {
+          const int t = t_begin + j * kSelThreads + tid;
+          f(t, t < t_end, kc[j]);
+        }
+      }
+    } else {
+      for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
+        const int t = b0 + tid;
+        f(t, t < t_end, t < t_end ? key_at(t) : 0u);
+      }
+    }
+  };
 
   for (int i = tid; i < 512; i += kSelThreads) (&hist[0][0])[i] = 0;
   __syncthreads();
-  // The histogram of the keys' top byte over this slice.  All lanes run the
-  // same trip count for the warp votes.
-  for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
-    const int t = b0 + tid;
-    uint32_t bin = 256u;
-    if (t < t_end) bin = key_at(t) >> 24;
-    hist_add(hist[0], bin);
-  }
+  // The histogram of the keys' top byte over this slice.
+  visit([&](int, bool valid, uint32_t key) { hist_add(hist[0], valid ? key >> 24 : 256u); });
 
   uint32_t prefix = 0;  // the n-th smallest key of the column, one byte per pass
   int need = n;         // how many keys equal to the final prefix are taken
@@ -123,15 +147,11 @@ __global__ void __launch_bounds__(kSelThreads)
     if (pass > 0) {
       for (int i = tid; i < 256; i += kSelThreads) h[i] = 0;
       __syncthreads();
-      for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
-        const int t = b0 + tid;
+      visit([&](int, bool valid, uint32_t key) {
         uint32_t bin = 256u;
-        if (t < t_end) {
-          const uint32_t key = key_at(t);
-          if ((key >> (shift + 8)) == (prefix >> (shift + 8))) bin = (key >> shift) & 255u;
-        }
+        if (valid && (key >> (shift + 8)) == (prefix >> (shift + 8))) bin = (key >> shift) & 255u;
         hist_add(h, bin);
-      }
+      });
     }
     // Every CTA's histogram of this pass is complete before any is read;
     // the other buffer is rewritten only after the next barrier.
@@ -182,11 +202,10 @@ __global__ void __launch_bounds__(kSelThreads)
   // tokens in position order.  First every slice counts both kinds; the
   // counts of the lower slices give this slice's starting ranks.
   int lt_n = 0, eq_n = 0;
-  for (int t = t_begin + tid; t < t_end; t += kSelThreads) {
-    const uint32_t key = key_at(t);
-    lt_n += (n > 0 && key < prefix);
-    eq_n += (n > 0 && key == prefix);
-  }
+  visit([&](int, bool valid, uint32_t key) {
+    lt_n += (valid && n > 0 && key < prefix);
+    eq_n += (valid && n > 0 && key == prefix);
+  });
   {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -224,23 +243,21 @@ __global__ void __launch_bounds__(kSelThreads)
 
   const int32_t row0 = e * npad;
   int carry_eq = eq_before, carry_sel = row_before;
-  for (int b0 = t_begin; b0 < t_end; b0 += kSelThreads) {
-    const int t = b0 + tid;
-    const uint32_t key = t < t_end ? key_at(t) : 0xffffffffu;
-    const bool eq = n > 0 && t < t_end && key == prefix;
-    const bool lt = n > 0 && t < t_end && key < prefix;
+  visit([&](int t, bool valid, uint32_t key) {
+    const bool eq = n > 0 && valid && key == prefix;
+    const bool lt = n > 0 && valid && key < prefix;
     int tot_eq, tot_sel;
     const int eq_rank = carry_eq + cta_exclusive_scan(eq, wsum_a, &tot_eq);
     const bool chosen = lt || (eq && eq_rank < need);
     const int row = carry_sel + cta_exclusive_scan(chosen, wsum_b, &tot_sel);
-    if (t < t_end) {
+    if (valid) {
       pos_t[(int64_t)e * T + t] = chosen ? row0 + row : -1;
       if (chosen) tok[(int64_t)e * n + row] = t;
     }
     carry_eq += tot_eq;
     carry_sel += tot_sel;
     __syncthreads();  // wsum_a / wsum_b are rewritten by the next chunk
-  }
+  });
   if (r == 0 && tid == 0) kept_counts[e] = n;
   if (blockIdx.x == 0)
     for (int i = tid; i <= E; i += kSelThreads) offsets[i] = i * npad;
