@@ -40,7 +40,11 @@ namespace {
 // histograms of its cluster through distributed shared memory and sums them
 // in rank order, so all CTAs find the same bucket.  The last pass exchanges
 // per-slice counts the same way to give each slice its starting ranks.
-constexpr int kSelCta = 8;       // CTAs per expert (one cluster)
+// CTAs per expert (one cluster).  Four rather than eight: on the 64-expert,
+// 16384-token layer the permutation stage (selection, transpose, copy) took
+// 145.5 us with clusters of four and 159 us with clusters of eight, whose
+// 512 CTAs need more than one round of the SMs; two measured the same as four.
+constexpr int kSelCta = 4;
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kKeyRegs = 16;     // key chunks a thread keeps in registers
