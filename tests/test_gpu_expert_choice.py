@@ -196,3 +196,26 @@ def test_expert_choice_many_ties_across_slices():
     tok = to_np(v["tok"])
     for e in range(w.E):
         assert np.array_equal(tok[e], tokens[e])
+
+
+def test_expert_choice_long_slices_read_keys_from_memory():
+    """T = 40000 tokens: each of the selection's four slices per expert holds
+    10000 keys, more than its threads keep in registers, so the passes read
+    the keys from the affinity matrix instead; the selection must be the
+    same (teacher-forced, bit-exact, with ties from coarse inputs)."""
+    w = Workload("long", T=40000, d=16, E=8, k=2, H=64, act="swiglu", dtype="bf16", cf=1.0,
+                 seed=26)
+    inp = make_inputs(w, "cpu")
+    g = torch.Generator().manual_seed(6)
+    rows = torch.randint(-2, 3, (50, w.d), generator=g).to(torch.bfloat16)
+    inp["x"] = rows[torch.randint(0, 50, (w.T,), generator=g)].contiguous()
+    t, layer, y, st, v = _run(w, inp)
+    assert st.device_error == 0
+    S_gpu = to_np(v["scores"]).T.astype(np.float64)
+    n = v["n"]
+    sel, tokens = oracle.expert_choice_select(S_gpu, n)
+    pos = to_np(v["pos"])
+    assert np.array_equal(pos >= 0, sel)
+    tok = to_np(v["tok"])
+    for e in range(w.E):
+        assert np.array_equal(tok[e], tokens[e])
